@@ -1,0 +1,385 @@
+"""Plain fp64 CPU oracle of the grouped NVFP4 MoE expert forward.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference legs of ``bench.py`` call this module.  The product
+path (CUDA library + binding) never imports it, and it imports nothing from
+the product package.  It is deliberately slow and obvious: numpy in float64,
+the library matmul and stable argsort as its only primitives, no blocking and
+no fusion.
+
+Sources (rustdoc source pages of the "metrale" project; cited by page and item):
+
+* metrale_model_arch/tp_shard/quant_shard.rs, layout comment at the top of the
+  file: NVFP4 ``weight`` [N, K/2] u8 packed E2M1, ``weight_scale``
+  [N, K/group] u8 E4M3, one f32 ``weight_scale_2``.
+* metrale_model_layers/weight_map/quantized/transpose.rs,
+  ``transpose_for_gemm``: the NVFP4 group is 16; the host fallback of
+  ``transpose_for_gemm_gs`` is the byte loop that defines ``transpose_u8``.
+* metrale_model_layers/layers/ops/nvfp4_moe_grouped.rs, module doc: rows are
+  grouped by expert and the active experts listed (``moe_fp8_grouped_sort``);
+  intermediates are laid out by sorted position; the router-weighted blend
+  (``moe_weighted_sum_blend_fp8_grouped``) returns to token order.  Doc of
+  ``moe_expert_gate_up_act_nvfp4_grouped``: the gate+up kernel writes the FP32
+  product of SiLU(gate) and up, ``[positions, n]``.  Doc of
+  ``moe_expert_down_act_nvfp4_grouped``: down runs over that product; rows of
+  its output are sorted positions.
+* metrale_model_arch/nemotron_moe/prefill_weights.rs, the shared-expert comment
+  of ``prepare_prefill_weights``: the E4M3 cast saturates at 448, which fixes
+  the E4M3 variant as the finite "FN" one (max 448, no infinities).
+* metrale_model_layers/weight_map/expert.rs, ``ExpertWeight::null``: a NULL
+  expert is skipped by the MoE kernels.
+
+Readings where the pages are silent (each also listed in the design notes):
+
+* nibble order: the low nibble of byte j holds k = 2j, the high nibble k = 2j+1;
+* E2M1 and E4M3 follow the OCP 8-bit / MX element definitions; the two E4M3
+  NaN codes 0x7F and 0xFF are rejected (ValueError);
+* the weight value is E2M1(code) * E4M3(scale of its 16-block) * weight_scale_2;
+* gate and up are not rounded to BF16 before SiLU: the product is formed from
+  the exact sums ("kept in FP32" on the GPU, fp64 here);
+* SiLU(z) = z / (1 + exp(-z));
+* sort ties are broken by pair id (pair p = token * k + slot), so the sort is
+  stable and unique; ``active_experts`` is ascending and padded with -1;
+  an expert id outside [0, E) drops its pair (pair_pos = -1, contributes 0);
+* a NULL expert's rows of ``act`` and ``y`` are zero.
+
+Parity pins for every function live in ``tests/test_oracle_pins.py``.
+"""
+
+from __future__ import annotations
+
+import math
+from typing import Callable, Dict, List, Optional, Sequence, Tuple
+
+import numpy as np
+
+__all__ = [
+    "E2M1_GROUP",
+    "e2m1_value",
+    "e2m1_table",
+    "e4m3_value",
+    "e4m3_table",
+    "bf16_bits_to_f64",
+    "dequantize_nvfp4",
+    "silu",
+    "route_sort",
+    "gate_up_silu",
+    "down_proj",
+    "blend",
+    "moe_forward",
+    "moe_forward_tokens",
+    "transpose_u8",
+    "RouteSort",
+]
+
+# NVFP4 block-scale group (transpose.rs, transpose_for_gemm).
+E2M1_GROUP = 16
+
+
+# --------------------------------------------------------------------------- #
+# Element formats
+# --------------------------------------------------------------------------- #
+
+def e2m1_value(code: int) -> float:
+    """Value of one 4-bit E2M1 code: 1 sign bit, 2 exponent bits (bias 1), 1 mantissa bit.
+
+    Exponent field 0 is subnormal: mantissa * 2^-1.  No NaN or infinity codes.
+    """
+    if not 0 <= code <= 15:
+        raise ValueError(f"E2M1 code out of range: {code}")
+    sign = -1.0 if code & 0x8 else 1.0
+    exp = (code >> 1) & 0x3
+    man = code & 0x1
+    if exp == 0:
+        mag = man * 0.5
+    else:
+        mag = 2.0 ** (exp - 1) * (1.0 + man / 2.0)
+    return sign * mag
+
+
+def e2m1_table() -> np.ndarray:
+    """All 16 E2M1 codes decoded, float64 [16]."""
+    return np.array([e2m1_value(c) for c in range(16)], dtype=np.float64)
+
+
+def e4m3_value(code: int) -> float:
+    """Value of one E4M3 (FN) code: 1 sign, 4 exponent bits (bias 7), 3 mantissa bits.
+
+    Exponent field 0 is subnormal: mantissa/8 * 2^-6.  The codes 0x7F and 0xFF
+    are NaN and are rejected with ValueError; there are no infinities, so the
+    largest finite magnitude is 0x7E = 448.
+    """
+    if not 0 <= code <= 255:
+        raise ValueError(f"E4M3 code out of range: {code}")
+    if code & 0x7F == 0x7F:
+        raise ValueError(f"E4M3 code 0x{code:02X} is NaN")
+    sign = -1.0 if code & 0x80 else 1.0
+    exp = (code >> 3) & 0xF
+    man = code & 0x7
+    if exp == 0:
+        mag = (man / 8.0) * 2.0 ** -6
+    else:
+        mag = 2.0 ** (exp - 7) * (1.0 + man / 8.0)
+    return sign * mag
+
+
+def e4m3_table() -> np.ndarray:
+    """All 256 E4M3 codes decoded, float64 [256]; the two NaN codes hold NaN."""
+    out = np.empty(256, dtype=np.float64)
+    for c in range(256):
+        try:
+            out[c] = e4m3_value(c)
+        except ValueError:
+            out[c] = np.nan
+    return out
+
+
+_E2M1 = e2m1_table()
+_E4M3 = e4m3_table()
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """BF16 bit patterns (uint16) to float64, exactly."""
+    u = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return u.view(np.float32).astype(np.float64)
+
+
+def dequantize_nvfp4(packed: np.ndarray, scale: np.ndarray, scale2) -> np.ndarray:
+    """Dense float64 [N, K] of one NVFP4 weight.
+
+    W[n, k] = E2M1(nibble k of row n) * E4M3(scale[n, k // 16]) * weight_scale_2,
+    nibble k being the low nibble of packed[n, k // 2] for even k and the high
+    nibble for odd k.  A NaN scale code raises ValueError.
+    """
+    packed = np.asarray(packed, dtype=np.uint8)
+    scale = np.asarray(scale, dtype=np.uint8)
+    n, half_k = packed.shape
+    k = 2 * half_k
+    if scale.shape != (n, k // E2M1_GROUP):
+        raise ValueError(f"scale shape {scale.shape} does not match packed {packed.shape}")
+    if np.any((scale & 0x7F) == 0x7F):
+        raise ValueError("E4M3 block scale holds a NaN code")
+    codes = np.empty((n, k), dtype=np.uint8)
+    codes[:, 0::2] = packed & 0x0F
+    codes[:, 1::2] = packed >> 4
+    w = _E2M1[codes]
+    w *= np.repeat(_E4M3[scale], E2M1_GROUP, axis=1)
+    w *= float(np.float32(scale2))
+    return w
+
+
+def silu(z: np.ndarray) -> np.ndarray:
+    """SiLU(z) = z / (1 + exp(-z)), float64."""
+    z = np.asarray(z, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
+
+
+# --------------------------------------------------------------------------- #
+# Step 1: group the routed pairs by expert
+# --------------------------------------------------------------------------- #
+
+class RouteSort:
+    """Result of :func:`route_sort`.
+
+    expert_offsets  int32 [E+1]  exclusive prefix of per-expert pair counts
+    sorted_pair_ids int32 [P]    pair ids (token * k + slot) in sorted order;
+                                 only the first expert_offsets[E] are defined
+    pair_pos        int32 [P]    sorted position of each pair, -1 if dropped
+    active_experts  int32 [E]    experts with at least one pair, ascending, -1 padded
+    active_count    int          number of such experts
+    dropped         int          pairs whose expert id was outside [0, E)
+    """
+
+    def __init__(self, expert_offsets, sorted_pair_ids, pair_pos, active_experts,
+                 active_count, dropped):
+        self.expert_offsets = expert_offsets
+        self.sorted_pair_ids = sorted_pair_ids
+        self.pair_pos = pair_pos
+        self.active_experts = active_experts
+        self.active_count = active_count
+        self.dropped = dropped
+
+
+def _stable_order(keys: np.ndarray) -> np.ndarray:
+    """Indices that sort ``keys`` ascending, equal keys kept in index order."""
+    return np.argsort(keys, kind="stable")
+
+
+def route_sort(topk_ids: np.ndarray, num_experts: int) -> RouteSort:
+    """Order the routed (token, expert) pairs by expert, ties by pair id.
+
+    Follows the grouping that nvfp4_moe_grouped.rs (module doc) takes from
+    ``moe_fp8_grouped_sort``: rows grouped by expert, the active experts listed,
+    intermediates laid out by sorted position.
+    """
+    ids = np.asarray(topk_ids, dtype=np.int64).reshape(-1)
+    p_total = ids.size
+    valid = (ids >= 0) & (ids < num_experts)
+    valid_pairs = np.nonzero(valid)[0]
+    order = valid_pairs[_stable_order(ids[valid_pairs])]
+    counts = np.bincount(ids[valid_pairs], minlength=num_experts)
+    offsets = np.zeros(num_experts + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    sorted_pair_ids = np.full(p_total, -1, dtype=np.int32)
+    sorted_pair_ids[: order.size] = order
+    pair_pos = np.full(p_total, -1, dtype=np.int32)
+    pair_pos[order] = np.arange(order.size, dtype=np.int32)
+    active = np.nonzero(counts > 0)[0]
+    active_experts = np.full(num_experts, -1, dtype=np.int32)
+    active_experts[: active.size] = active
+    return RouteSort(offsets.astype(np.int32), sorted_pair_ids, pair_pos, active_experts,
+                     int(active.size), int(p_total - order.size))
+
+
+# --------------------------------------------------------------------------- #
+# Steps 2-4
+# --------------------------------------------------------------------------- #
+
+WeightFn = Callable[[int], Optional[Tuple[np.ndarray, np.ndarray, float]]]
+
+
+def _dense(weight_fn: WeightFn, expert: int) -> Optional[np.ndarray]:
+    w = weight_fn(expert)
+    if w is None:
+        return None
+    packed, scale, s2 = w
+    return dequantize_nvfp4(packed, scale, s2)
+
+
+def gate_up_silu(x_bf16: np.ndarray, topk: int, rs: RouteSort,
+                 gate_fn: WeightFn, up_fn: WeightFn, inter: int) -> np.ndarray:
+    """act [P, I] by sorted position: SiLU(x Wg^T) * (x Wu^T), float64.
+
+    nvfp4_moe_grouped.rs, ``moe_expert_gate_up_act_nvfp4_grouped``: for each
+    active expert and each of its rows (a pair, whose token is pair // k), the
+    gate and up projections of that token's row and their SiLU product.  Rows of
+    a NULL expert are zero.  Rows past expert_offsets[E] are zero.
+    """
+    x = bf16_bits_to_f64(x_bf16)
+    p_total = rs.sorted_pair_ids.size
+    act = np.zeros((p_total, inter), dtype=np.float64)
+    for a in range(rs.active_count):
+        e = int(rs.active_experts[a])
+        lo, hi = int(rs.expert_offsets[e]), int(rs.expert_offsets[e + 1])
+        wg, wu = _dense(gate_fn, e), _dense(up_fn, e)
+        if wg is None or wu is None:
+            continue
+        tokens = rs.sorted_pair_ids[lo:hi] // topk
+        xe = x[tokens]
+        g = xe @ wg.T
+        u = xe @ wu.T
+        act[lo:hi] = silu(g) * u
+    return act
+
+
+def down_proj(act: np.ndarray, rs: RouteSort, down_fn: WeightFn, hidden: int) -> np.ndarray:
+    """y [P, H] by sorted position: act Wd^T per expert, float64.
+
+    nvfp4_moe_grouped.rs, ``moe_expert_down_act_nvfp4_grouped``.
+    """
+    p_total = act.shape[0]
+    y = np.zeros((p_total, hidden), dtype=np.float64)
+    for a in range(rs.active_count):
+        e = int(rs.active_experts[a])
+        lo, hi = int(rs.expert_offsets[e]), int(rs.expert_offsets[e + 1])
+        wd = _dense(down_fn, e)
+        if wd is None:
+            continue
+        y[lo:hi] = act[lo:hi] @ wd.T
+    return y
+
+
+def blend(y: np.ndarray, topk_weights: np.ndarray, pair_pos: np.ndarray) -> np.ndarray:
+    """out [M, H] = sum over slots s of w[t, s] * y[pair_pos[t*k + s]], float64.
+
+    The router-weighted blend back into token order named in the module doc of
+    nvfp4_moe_grouped.rs (``moe_weighted_sum_blend_fp8_grouped``).  A dropped
+    pair (pair_pos = -1) contributes nothing.
+    """
+    w = np.asarray(topk_weights, dtype=np.float64)
+    m, k = w.shape
+    out = np.zeros((m, y.shape[1]), dtype=np.float64)
+    for t in range(m):
+        for s in range(k):
+            pos = int(pair_pos[t * k + s])
+            if pos >= 0:
+                out[t] += w[t, s] * y[pos]
+    return out
+
+
+def moe_forward(x_bf16, topk_ids, topk_weights, num_experts, gate_fn, up_fn, down_fn,
+                hidden: int, inter: int) -> Dict[str, object]:
+    """The four steps in order; returns every intermediate."""
+    topk = np.asarray(topk_ids).shape[1]
+    rs = route_sort(topk_ids, num_experts)
+    act = gate_up_silu(x_bf16, topk, rs, gate_fn, up_fn, inter)
+    y = down_proj(act, rs, down_fn, hidden)
+    out = blend(y, topk_weights, rs.pair_pos)
+    return {"sort": rs, "act": act, "y": y, "out": out}
+
+
+def moe_forward_tokens(x_bf16, topk_ids, topk_weights, num_experts, gate_fn, up_fn, down_fn,
+                       tokens: Sequence[int], hidden: int) -> np.ndarray:
+    """out rows for the listed tokens only, computed token by token, float64.
+
+    The same expert forward written per token: for each routed slot of a token,
+    the expert's gated MLP on that token's row, weighted by its router weight.
+    It shares no grouping with :func:`moe_forward`, so the two check each other,
+    and it lets a full-size problem be checked on a sample of tokens.  Expert
+    weights are dequantised once per expert and cached for the call.
+    """
+    x = bf16_bits_to_f64(x_bf16)
+    ids = np.asarray(topk_ids)
+    w = np.asarray(topk_weights, dtype=np.float64)
+    cache: Dict[int, Optional[List[np.ndarray]]] = {}
+    out = np.zeros((len(tokens), hidden), dtype=np.float64)
+    for i, t in enumerate(tokens):
+        for s in range(ids.shape[1]):
+            e = int(ids[t, s])
+            if not 0 <= e < num_experts:
+                continue
+            if e not in cache:
+                mats = [_dense(fn, e) for fn in (gate_fn, up_fn, down_fn)]
+                cache[e] = None if any(m is None for m in mats) else mats
+            if cache[e] is None:
+                continue
+            wg, wu, wd = cache[e]
+            h = silu(wg @ x[t]) * (wu @ x[t])
+            out[i] += w[t, s] * (wd @ h)
+    return out
+
+
+# --------------------------------------------------------------------------- #
+# Load-time twin builder
+# --------------------------------------------------------------------------- #
+
+def transpose_u8(src: np.ndarray, rows: int, cols: int) -> np.ndarray:
+    """Byte transpose [rows, cols] -> [cols, rows].
+
+    The host fallback of ``transpose_for_gemm_gs`` (transpose.rs) defines it:
+    t[j * rows + i] = b[i * cols + j].  Written as that double loop; it is only
+    run on small inputs.
+    """
+    b = np.asarray(src, dtype=np.uint8).reshape(-1)
+    if b.size != rows * cols:
+        raise ValueError("size mismatch")
+    t = np.empty(rows * cols, dtype=np.uint8)
+    for i in range(rows):
+        for j in range(cols):
+            t[j * rows + i] = b[i * cols + j]
+    return t.reshape(cols, rows)
+
+
+def relative_l2(got: np.ndarray, ref: np.ndarray) -> float:
+    """||got - ref||_2 / ||ref||_2 (0 when both are zero)."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    den = float(np.linalg.norm(ref))
+    num = float(np.linalg.norm(got - ref))
+    if den == 0.0:
+        return 0.0 if num == 0.0 else math.inf
+    return num / den
+
+
+__all__.append("relative_l2")

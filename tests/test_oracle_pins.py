@@ -1,0 +1,405 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself.
+
+Each test ties one oracle function to a library routine, a closed form, a
+brute-force evaluation on a tiny input, or an invariant of the expert forward,
+chosen so that a plausible slip (swapped nibbles, a wrong scale index, a
+transposed operand, a lost token index, an unstable sort) fails at least one
+of them.  The last tests plant such slips in a copy of the oracle and check
+that the pins catch them.
+"""
+
+import math
+import os
+
+import ml_dtypes
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from workloads import make_problem
+from workloads.generators import MATRIX_DOWN, MATRIX_GATE, MATRIX_UP, MoEConfig
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "e4m3_e2m1_spot_values.txt")
+
+
+def _golden():
+    rows = []
+    with open(GOLDEN) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            fmt, code, val = line.split()
+            rows.append((fmt, int(code, 16), float(val)))
+    return rows
+
+
+# --------------------------------------------------------------------------- #
+# Element formats
+# --------------------------------------------------------------------------- #
+
+def test_e2m1_spot_values_from_spec():
+    for fmt, code, val in _golden():
+        if fmt == "e2m1":
+            assert orc.e2m1_value(code) == val
+
+
+def test_e2m1_table_matches_ml_dtypes():
+    lib = np.arange(16, dtype=np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    np.testing.assert_array_equal(orc.e2m1_table(), lib)
+
+
+def test_e4m3_spot_values_from_spec():
+    for fmt, code, val in _golden():
+        if fmt != "e4m3":
+            continue
+        if math.isnan(val):
+            with pytest.raises(ValueError):
+                orc.e4m3_value(code)
+        else:
+            got = orc.e4m3_value(code)
+            assert got == val and math.copysign(1.0, got) == math.copysign(1.0, val)
+
+
+def test_e4m3_exhaustive_against_torch_and_ml_dtypes():
+    codes = np.arange(256, dtype=np.uint8)
+    ref_t = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    ref_m = codes.view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    table = orc.e4m3_table()
+    finite = 0
+    for c in range(256):
+        if (c & 0x7F) == 0x7F:
+            assert math.isnan(ref_t[c]) and math.isnan(table[c])
+            with pytest.raises(ValueError):
+                orc.e4m3_value(c)
+            continue
+        finite += 1
+        assert table[c] == ref_t[c] == ref_m[c], hex(c)
+    assert finite == 254
+    assert np.nanmax(table) == 448.0
+
+
+def test_every_e2m1_e4m3_product_is_exact_in_bf16_and_f16():
+    # The weight value before weight_scale_2 is a product of the two codes; it
+    # must survive a BF16 (and an F16) round trip unchanged, which is what lets a
+    # 16-bit tensor-core operand carry it exactly.
+    e2 = orc.e2m1_table()
+    e4 = orc.e4m3_table()
+    prods = np.array([a * b for a in e2 for b in e4 if not math.isnan(b)])
+    as_bf16 = torch.from_numpy(prods).to(torch.bfloat16).to(torch.float64).numpy()
+    as_f16 = prods.astype(np.float16).astype(np.float64)
+    np.testing.assert_array_equal(as_bf16, prods)
+    np.testing.assert_array_equal(as_f16, prods)
+
+
+def test_bf16_decode_matches_torch():
+    bits = np.random.default_rng(3).integers(0, 1 << 16, 4096, dtype=np.uint16)
+    bits = bits[((bits >> 7) & 0xFF) != 0xFF]  # skip inf / NaN patterns
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(orc.bf16_bits_to_f64(bits), ref)
+
+
+def test_silu_special_values():
+    assert orc.silu(np.array(0.0)) == 0.0
+    assert abs(float(orc.silu(np.array(1.0))) - 0.7310585786300049) < 1e-15
+    assert abs(float(orc.silu(np.array(-1.0))) - (-0.2689414213699951)) < 1e-15
+    assert float(orc.silu(np.array(60.0))) == pytest.approx(60.0, rel=1e-15)
+    assert abs(float(orc.silu(np.array(-60.0)))) < 1e-24
+    assert float(orc.silu(np.array(-1000.0))) == 0.0  # no overflow warning escapes
+
+
+# --------------------------------------------------------------------------- #
+# Dequantisation
+# --------------------------------------------------------------------------- #
+
+def test_nibble_order_low_nibble_is_even_k():
+    # byte 0x21: low nibble 1 (0.5) at k=0, high nibble 2 (1.0) at k=1.
+    packed = np.zeros((1, 8), dtype=np.uint8)
+    packed[0, 0] = 0x21
+    scale = np.full((1, 1), 0x38, dtype=np.uint8)  # 1.0
+    w = orc.dequantize_nvfp4(packed, scale, np.float32(1.0))
+    assert w[0, 0] == 0.5 and w[0, 1] == 1.0 and not w[0, 2:].any()
+
+
+def test_dequant_unit_scales_reduce_to_library_fp4():
+    rng = np.random.default_rng(7)
+    packed = rng.integers(0, 256, (5, 16), dtype=np.uint8)
+    scale = np.full((5, 2), 0x38, dtype=np.uint8)
+    w = orc.dequantize_nvfp4(packed, scale, np.float32(1.0))
+    lo = (packed & 0xF).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    hi = (packed >> 4).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    np.testing.assert_array_equal(w[:, 0::2], lo)
+    np.testing.assert_array_equal(w[:, 1::2], hi)
+
+
+def test_dequant_block_scale_touches_only_its_16_block():
+    rng = np.random.default_rng(8)
+    packed = rng.integers(0, 256, (4, 32), dtype=np.uint8)  # K = 64: 4 blocks
+    scale = rng.integers(0x18, 0x49, (4, 4), dtype=np.uint8)
+    base = orc.dequantize_nvfp4(packed, scale, np.float32(1 / 448))
+    bumped = scale.copy()
+    bumped[2, 1] += 8  # exponent + 1: that block doubles
+    w = orc.dequantize_nvfp4(packed, bumped, np.float32(1 / 448))
+    expect = base.copy()
+    expect[2, 16:32] *= 2.0
+    np.testing.assert_array_equal(w, expect)
+
+
+def test_dequant_scale2_is_a_plain_factor():
+    rng = np.random.default_rng(9)
+    packed = rng.integers(0, 256, (3, 8), dtype=np.uint8)
+    scale = rng.integers(0x18, 0x49, (3, 1), dtype=np.uint8)
+    a = orc.dequantize_nvfp4(packed, scale, np.float32(1.0))
+    b = orc.dequantize_nvfp4(packed, scale, np.float32(0.375))
+    np.testing.assert_array_equal(b, a * 0.375)
+
+
+def test_dequant_rejects_nan_scale():
+    packed = np.zeros((1, 8), dtype=np.uint8)
+    with pytest.raises(ValueError):
+        orc.dequantize_nvfp4(packed, np.array([[0x7F]], dtype=np.uint8), np.float32(1.0))
+    with pytest.raises(ValueError):
+        orc.dequantize_nvfp4(packed, np.array([[0xFF]], dtype=np.uint8), np.float32(1.0))
+
+
+# --------------------------------------------------------------------------- #
+# Route sort
+# --------------------------------------------------------------------------- #
+
+def _brute_sort(ids, num_experts):
+    flat = [int(v) for v in np.asarray(ids).reshape(-1)]
+    order = []
+    for e in range(num_experts):
+        for p, v in enumerate(flat):
+            if v == e:
+                order.append(p)
+    return order
+
+
+@pytest.mark.parametrize("m,k,e", [(1, 2, 8), (7, 3, 5), (33, 8, 128), (64, 4, 3)])
+def test_route_sort_brute_force(m, k, e):
+    rng = np.random.default_rng(m * 1000 + e)
+    ids = rng.integers(0, e, (m, k)).astype(np.int32)
+    rs = orc.route_sort(ids, e)
+    order = _brute_sort(ids, e)
+    assert list(rs.sorted_pair_ids[: len(order)]) == order
+    assert rs.expert_offsets[-1] == m * k and rs.dropped == 0
+    counts = np.diff(rs.expert_offsets)
+    for ex in range(e):
+        assert counts[ex] == int((ids == ex).sum())
+    for pos, p in enumerate(order):
+        assert rs.pair_pos[p] == pos
+    active = [ex for ex in range(e) if counts[ex] > 0]
+    assert rs.active_count == len(active)
+    assert list(rs.active_experts) == active + [-1] * (e - len(active))
+
+
+def test_route_sort_drops_out_of_range_ids():
+    ids = np.array([[0, 5], [-1, 2], [9, 2]], dtype=np.int32)
+    rs = orc.route_sort(ids, 4)
+    assert rs.dropped == 3
+    assert list(rs.sorted_pair_ids[:3]) == [0, 3, 5]
+    assert list(rs.pair_pos) == [0, -1, -1, 1, -1, 2]
+    assert list(rs.expert_offsets) == [0, 1, 1, 3, 3]
+    assert rs.active_count == 2 and list(rs.active_experts) == [0, 2, -1, -1]
+
+
+# --------------------------------------------------------------------------- #
+# The expert forward
+# --------------------------------------------------------------------------- #
+
+def _tiny_cfg(**kw):
+    base = dict(name="pin", hidden=32, inter=16, experts=3, topk=2, tokens=5,
+                router="uniform", seed=77)
+    base.update(kw)
+    return MoEConfig(**base)
+
+
+def _run(prob, **kw):
+    cfg = prob.cfg
+    fns = [lambda e, m=m: prob.expert_weight(m, e) for m in (MATRIX_GATE, MATRIX_UP, MATRIX_DOWN)]
+    return orc.moe_forward(prob.x_bf16, prob.topk_ids, prob.topk_weights, cfg.experts,
+                           *fns, hidden=cfg.hidden, inter=cfg.inter, **kw)
+
+
+def _scalar_weight(prob, m, e, n, k):
+    packed, scale, s2 = prob.expert_weight(m, e)
+    byte = int(packed[n, k // 2])
+    code = (byte >> 4) if (k % 2) else (byte & 0xF)
+    return orc.e2m1_value(code) * orc.e4m3_value(int(scale[n, k // 16])) * float(s2)
+
+
+def test_expert_forward_brute_force_scalar_loops():
+    prob = make_problem(_tiny_cfg())
+    cfg = prob.cfg
+    res = _run(prob)
+    x = orc.bf16_bits_to_f64(prob.x_bf16)
+    for t in range(cfg.tokens):
+        acc = [0.0] * cfg.hidden
+        for s in range(cfg.topk):
+            e = int(prob.topk_ids[t, s])
+            wt = float(prob.topk_weights[t, s])
+            h = []
+            for n in range(cfg.inter):
+                g = sum(_scalar_weight(prob, MATRIX_GATE, e, n, k) * x[t, k] for k in range(cfg.hidden))
+                u = sum(_scalar_weight(prob, MATRIX_UP, e, n, k) * x[t, k] for k in range(cfg.hidden))
+                h.append(g / (1.0 + math.exp(-g)) * u)
+            for j in range(cfg.hidden):
+                acc[j] += wt * sum(_scalar_weight(prob, MATRIX_DOWN, e, j, i) * h[i] for i in range(cfg.inter))
+        np.testing.assert_allclose(res["out"][t], acc, rtol=1e-12, atol=1e-12)
+
+
+def test_single_expert_weight_one_is_dense_gated_mlp():
+    prob = make_problem(_tiny_cfg(experts=1, topk=1, tokens=4, hidden=48, inter=32))
+    res = _run(prob)
+    assert np.all(prob.topk_weights == 1.0)
+    x = orc.bf16_bits_to_f64(prob.x_bf16)
+    wg = orc.dequantize_nvfp4(*prob.expert_weight(MATRIX_GATE, 0))
+    wu = orc.dequantize_nvfp4(*prob.expert_weight(MATRIX_UP, 0))
+    wd = orc.dequantize_nvfp4(*prob.expert_weight(MATRIX_DOWN, 0))
+    dense = (orc.silu(x @ wg.T) * (x @ wu.T)) @ wd.T
+    np.testing.assert_allclose(res["out"], dense, rtol=1e-13, atol=1e-13)
+
+
+def test_unit_vector_input_picks_a_weight_column():
+    # x = e_j: gate/up reduce to column j of Wg / Wu, which fails for a
+    # transposed operand or a wrong k index.
+    prob = make_problem(_tiny_cfg(experts=2, topk=1, tokens=3))
+    j = [3, 17, 30]
+    prob.x_bf16[:] = 0
+    for t in range(3):
+        prob.x_bf16[t, j[t]] = 0x3F80  # 1.0
+    res = _run(prob)
+    rs = res["sort"]
+    for t in range(3):
+        e = int(prob.topk_ids[t, 0])
+        wg = orc.dequantize_nvfp4(*prob.expert_weight(MATRIX_GATE, e))
+        wu = orc.dequantize_nvfp4(*prob.expert_weight(MATRIX_UP, e))
+        expect = orc.silu(wg[:, j[t]]) * wu[:, j[t]]
+        np.testing.assert_array_equal(res["act"][rs.pair_pos[t]], expect)
+
+
+def test_token_permutation_invariance():
+    prob = make_problem(_tiny_cfg(tokens=9, experts=4, topk=2, seed=5))
+    base = _run(prob)["out"]
+    perm = np.random.default_rng(1).permutation(9)
+    prob.x_bf16 = prob.x_bf16[perm].copy()
+    prob.topk_ids = prob.topk_ids[perm].copy()
+    prob.topk_weights = prob.topk_weights[perm].copy()
+    out = _run(prob)["out"]
+    np.testing.assert_allclose(out, base[perm], rtol=1e-13, atol=1e-13)
+
+
+def test_blend_is_linear_and_one_hot_selects_a_pair():
+    prob = make_problem(_tiny_cfg(tokens=4, experts=3, topk=2, seed=6))
+    res = _run(prob)
+    y, pos = res["y"], res["sort"].pair_pos
+    w1 = np.random.default_rng(2).random((4, 2))
+    w2 = np.random.default_rng(3).random((4, 2))
+    np.testing.assert_allclose(orc.blend(y, w1 + w2, pos),
+                               orc.blend(y, w1, pos) + orc.blend(y, w2, pos), rtol=1e-13)
+    onehot = np.zeros((4, 2))
+    onehot[:, 1] = 1.0
+    sel = orc.blend(y, onehot, pos)
+    for t in range(4):
+        np.testing.assert_array_equal(sel[t], y[pos[t * 2 + 1]])
+
+
+def test_grouped_forward_equals_per_token_forward():
+    prob = make_problem(_tiny_cfg(tokens=11, experts=6, topk=3, hidden=64, inter=48, seed=11))
+    cfg = prob.cfg
+    res = _run(prob)
+    fns = [lambda e, m=m: prob.expert_weight(m, e) for m in (MATRIX_GATE, MATRIX_UP, MATRIX_DOWN)]
+    per_tok = orc.moe_forward_tokens(prob.x_bf16, prob.topk_ids, prob.topk_weights, cfg.experts,
+                                     *fns, tokens=range(cfg.tokens), hidden=cfg.hidden)
+    np.testing.assert_allclose(res["out"], per_tok, rtol=1e-12, atol=1e-12)
+
+
+def test_null_expert_contributes_zero():
+    prob = make_problem(_tiny_cfg(tokens=6, experts=3, topk=2, seed=12), null_experts=[1])
+    res = _run(prob)
+    rs = res["sort"]
+    lo, hi = rs.expert_offsets[1], rs.expert_offsets[2]
+    assert hi > lo  # expert 1 is routed to
+    assert not res["act"][lo:hi].any() and not res["y"][lo:hi].any()
+    # Same as zero weights for that expert's slots.
+    w = prob.topk_weights.astype(np.float64).copy()
+    w[prob.topk_ids == 1] = 0.0
+    np.testing.assert_allclose(res["out"], orc.blend(res["y"], w, rs.pair_pos), rtol=1e-13)
+
+
+def test_down_is_linear_in_scale2():
+    prob = make_problem(_tiny_cfg(seed=13))
+    a = _run(prob)["y"]
+    prob.scale2[MATRIX_DOWN, :] *= np.float32(4.0)
+    b = _run(prob)["y"]
+    np.testing.assert_allclose(b, 4.0 * a, rtol=1e-14)
+
+
+# --------------------------------------------------------------------------- #
+# transpose_u8
+# --------------------------------------------------------------------------- #
+
+@pytest.mark.parametrize("rows,cols", [(1, 1), (3, 5), (16, 9), (33, 64)])
+def test_transpose_u8_against_numpy_and_involution(rows, cols):
+    src = np.random.default_rng(rows * cols).integers(0, 256, (rows, cols), dtype=np.uint8)
+    t = orc.transpose_u8(src, rows, cols)
+    np.testing.assert_array_equal(t, src.T)
+    np.testing.assert_array_equal(orc.transpose_u8(t, cols, rows), src)
+
+
+# --------------------------------------------------------------------------- #
+# Planted mistakes: the pins above must catch them
+# --------------------------------------------------------------------------- #
+
+def test_pins_catch_swapped_nibble_order(monkeypatch):
+    real = orc.dequantize_nvfp4
+
+    def swapped(packed, scale, s2):
+        p = np.asarray(packed, dtype=np.uint8)
+        return real(((p & 0xF) << 4) | (p >> 4), scale, s2)
+
+    monkeypatch.setattr(orc, "dequantize_nvfp4", swapped)
+    with pytest.raises(AssertionError):
+        test_nibble_order_low_nibble_is_even_k()
+
+
+def test_pins_catch_a_transposed_operand(monkeypatch):
+    import oracle.nvfp4_moe_oracle as mod
+    real = mod._dense
+
+    def transposed(fn, e):
+        w = real(fn, e)
+        if w is None or w.shape[0] != w.shape[1]:
+            return w
+        return np.ascontiguousarray(w.T)
+
+    monkeypatch.setattr(mod, "_dense", transposed)
+    prob = make_problem(_tiny_cfg(hidden=32, inter=32, experts=2, topk=1, tokens=3))
+    j = [3, 17, 30]
+    prob.x_bf16[:] = 0
+    for t in range(3):
+        prob.x_bf16[t, j[t]] = 0x3F80
+    res = _run(prob)
+    rs = res["sort"]
+    bad = 0
+    for t in range(3):
+        e = int(prob.topk_ids[t, 0])
+        wg = real(lambda ex: prob.expert_weight(MATRIX_GATE, ex), e)
+        wu = real(lambda ex: prob.expert_weight(MATRIX_UP, ex), e)
+        expect = orc.silu(wg[:, j[t]]) * wu[:, j[t]]
+        bad += int(not np.array_equal(res["act"][rs.pair_pos[t]], expect))
+    assert bad > 0
+
+
+def test_pins_catch_an_unstable_sort(monkeypatch):
+    import oracle.nvfp4_moe_oracle as mod
+
+    def ties_reversed(keys):
+        keys = np.asarray(keys)
+        return np.lexsort((-np.arange(keys.size), keys))
+
+    monkeypatch.setattr(mod, "_stable_order", ties_reversed)
+    with pytest.raises(AssertionError):
+        test_route_sort_brute_force(33, 8, 128)
