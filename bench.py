@@ -1,0 +1,488 @@
+#!/usr/bin/env python3
+"""Throughput of the grouped NVFP4 MoE expert forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+One step = one layer forward: route sort, gate+up SiLU, down, blend (the four
+C-ABI calls) over one batch of the workload's synthetic tokens, weights and
+inputs resident in HBM.  The weights rotate over R device replicas (R x the
+routed bytes of a step >= 4 x L2), so every step streams its expert weights
+from HBM.  Steps are replayed from CUDA graphs and timed with CUDA events on
+the launching stream; under torchrun (N > 1) each rank runs an independent
+replica of the workload (weak scaling, no collective on the data path) and the
+time is the max over ranks.
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle
+on the host cores instead (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 MoE layer tokens/s and routed-weight HBM GB/s (% of peak), 1 B200"
+DEFAULT_CONFIG = "decode_m1"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+# Default timed steps per workload: about a second of GPU time each.
+DEFAULT_STEPS = {"tiny": 20000, "decode_m1": 20000, "decode_m32": 5000, "decode_m256": 500,
+                 "prefill_m8192": 200}
+
+# DRAM bytes of one launch of the dominant kernel, from an ncu capture of the
+# same kernel build (None until captured, and reset when the kernel changes).
+NCU_TRAFFIC_BYTES = {}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--path", type=int, default=0, help="0 auto, 1 decode, 2 prefill")
+    ap.add_argument("--split", type=int, default=0)
+    return ap.parse_args(argv)
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", 0)), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def dist_info():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def reduce_max(value: float, group=None) -> float:
+    """Max of a float over the ranks of the default process group (identity without one)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    backend = dist.get_backend(group)
+    dev = torch.device("cuda", torch.cuda.current_device()) if backend == "nccl" else torch.device("cpu")
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# --------------------------------------------------------------------------- #
+# Clock sampling during the timed region
+# --------------------------------------------------------------------------- #
+
+class ClockSampler:
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", str(self.dev)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, begin: bool):
+        if begin:
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for ts, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            rows.append((ts, parts))
+        inside = [r for r in rows if self.t0 is not None and self.t0 - 0.06 <= r[0] <= self.t1 + 0.06]
+        use = inside or rows[-3:]
+        if not use:
+            return None
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(p[2]) for _, p in use if num(p[2]) is not None]
+        smax = [num(p[3]) for _, p in use if num(p[3]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, p in use for i in range(4) if p[6 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(use), "samples_in_timed_region": len(inside)}
+
+
+# --------------------------------------------------------------------------- #
+# Our implementation
+# --------------------------------------------------------------------------- #
+
+def _replicate(layer, copies):
+    """`copies` extra device copies of a layer's weights (distinct memory, same values)."""
+    import nvfp4_weight_quantized_moe_b200 as nvm
+    out = [layer]
+    for _ in range(copies):
+        projs = []
+        for p in (layer.gate, layer.up, layer.down):
+            projs.append(nvm.NVFP4Projection(p.packed.clone(), p.scale.clone(), p.scale2.clone()))
+        out.append(nvm.NVFP4MoE(*projs, layer.topk))
+    return out
+
+
+def run_ours(args, rank, world, local):
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    import nvfp4_weight_quantized_moe_b200 as nvm
+    from workloads import make_problem
+    from workloads.device import upload_inputs, upload_layer
+
+    prob = make_problem(args.config)
+    cfg = prob.cfg
+    steps = args.steps if args.steps is not None else DEFAULT_STEPS.get(cfg.name, 1000)
+    warmup = max(args.warmup, 3)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.Stream(device=dev)
+
+    base = upload_layer(prob, dev)
+    x, ids, w = upload_inputs(prob, dev)
+    bufs = base.buffers(cfg.tokens)
+    # Active experts of this batch (identical for every replica: same routing).
+    with torch.cuda.stream(stream):
+        base.forward(x, ids, w, bufs, path=args.path, split=args.split)
+    stream.synchronize()
+    active = int(bufs.active_count.item())
+    per_expert = base.gate.nbytes_per_expert
+    routed_bytes = 3 * active * per_expert
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    replicas = max(1, math.ceil(4 * l2 / max(routed_bytes, 1)))
+    free = torch.cuda.mem_get_info(dev)[0]
+    layer_bytes = 3 * cfg.experts * per_expert
+    replicas = int(min(replicas, max(1, (free * 0.6) // layer_bytes), 64))
+    layers = _replicate(base, replicas - 1)
+
+    def step(lay):
+        lay.forward(x, ids, w, bufs, path=args.path, split=args.split)
+
+    # Graphs: one of R steps (one per replica) plus single-step graphs for remainders.
+    with torch.cuda.stream(stream):
+        for lay in layers:
+            step(lay)
+    stream.synchronize()
+    g_all = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_all, stream=stream):
+        for lay in layers:
+            step(lay)
+    g_one = []
+    for lay in layers:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(lay)
+        g_one.append(g)
+
+    def run_steps(n):
+        full, rem = divmod(n, len(layers))
+        for _ in range(full):
+            g_all.replay()
+        for i in range(rem):
+            g_one[i].replay()
+
+    with torch.cuda.stream(stream):
+        run_steps(warmup)
+    stream.synchronize()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler.mark(True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        run_steps(steps)
+        ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    sampler.mark(False)
+    barrier()
+    clocks = sampler.stop()
+    elapsed_ms = reduce_max(ev0.elapsed_time(ev1))
+    ms_per_step = elapsed_ms / steps
+    tokens_per_s = world * cfg.tokens * steps / (elapsed_ms / 1e3)
+
+    hbm, tflops, tflops_sus, peak_kind = measured_peaks()
+    routed_gbs = world * routed_bytes / (ms_per_step * 1e-3) / 1e9
+
+    # Dominant kernel, timed alone: gate+up SiLU, one launch per replica.
+    prefill = _uses_prefill(args, cfg)
+    gu_graph = torch.cuda.CUDAGraph()
+    cap = nvm.active_cap(cfg.experts, cfg.pairs)
+
+    def gate_up(lay):
+        nvm.gate_up_silu(x, lay.gate.tables, lay.up.tables, bufs.act, bufs.expert_offsets,
+                         bufs.sorted_pair_ids, bufs.active_experts, bufs.active_count,
+                         cfg.inter, cfg.hidden, cap, cfg.tokens, cfg.topk, path=args.path,
+                         split=args.split)
+    with torch.cuda.graph(gu_graph, stream=stream):
+        for lay in layers:
+            gate_up(lay)
+    reps = max(3, min(2000, int(200.0 / max(0.7 * ms_per_step * len(layers), 1e-4))))
+    with torch.cuda.stream(stream):
+        gu_graph.replay()
+        ev0.record(stream)
+        for _ in range(reps):
+            gu_graph.replay()
+        ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    gu_ms = ev0.elapsed_time(ev1) / (reps * len(layers))
+    gu_bytes = 2 * active * per_expert
+    gu_flops = 2.0 * 2 * cfg.pairs * cfg.hidden * cfg.inter
+    if prefill:
+        achieved = gu_flops / (gu_ms * 1e-3) / 1e12
+        roofline = {"kernel": "nvfp4_moe_gate_up_silu (tcgen05 prefill path)", "bound": "tensor",
+                    "achieved": achieved, "peak": tflops, "unit": "TFLOP/s",
+                    "frac": achieved / tflops, "peak_source": f"{peak_kind} bf16 burst",
+                    "algorithmic_flops_per_launch": gu_flops, "launch_ms": gu_ms,
+                    "traffic": NCU_TRAFFIC_BYTES.get(cfg.name)}
+    else:
+        achieved = gu_bytes / (gu_ms * 1e-3) / 1e9
+        roofline = {"kernel": "nvfp4_moe_gate_up_silu (decode path)", "bound": "hbm",
+                    "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                    "peak_source": f"{peak_kind} HBM copy", "algorithmic_bytes_per_launch": gu_bytes,
+                    "launch_ms": gu_ms, "traffic": NCU_TRAFFIC_BYTES.get(cfg.name)}
+
+    e2e = None if args.no_e2e else run_e2e(layers, prob, bufs, dev, stream, steps, warmup, args, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(prob)
+
+    line = {
+        "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
+        "steps": steps, "warmup": warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16-mma/f32-acc", "data": "synthetic",
+        "config": {"workload": cfg.name, "hidden": cfg.hidden, "inter": cfg.inter,
+                   "experts": cfg.experts, "topk": cfg.topk, "tokens": cfg.tokens,
+                   "router": cfg.router, "active_experts": active,
+                   "path": "prefill-tcgen05" if prefill else "decode-mma",
+                   "weight_replicas": len(layers),
+                   "l2": f"weights rotate over {len(layers)} device replicas; "
+                         f"{len(layers)} x {routed_bytes/1e6:.1f} MB routed >= 4 x L2 ({l2/1e6:.0f} MB)"
+                         if len(layers) > 1 else f"routed bytes {routed_bytes/1e6:.0f} MB > 4 x L2",
+                   "parallelism": f"replicas x{world}"},
+        "routed_weight_gbs": {"value": routed_gbs, "peak": hbm, "frac": routed_gbs / hbm,
+                              "bytes_per_step": routed_bytes},
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 4 * steps,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        del g_all, g_one, gu_graph
+        dist.destroy_process_group()
+
+
+def _uses_prefill(args, cfg):
+    return False
+
+
+def run_e2e(layers, prob, bufs, dev, stream, steps, warmup, args, world):
+    """Same metric through the public API from pinned host buffers: per step the
+    host->device copy of x / topk_ids / topk_weights, the forward, and the
+    device->host copy of the FP32 output, all inside the timed region."""
+    import torch
+    cfg = prob.cfg
+    hx = torch.from_numpy(prob.x_bf16.view(np.int16)).view(torch.bfloat16).pin_memory()
+    hids = torch.from_numpy(np.ascontiguousarray(prob.topk_ids)).pin_memory()
+    hw = torch.from_numpy(np.ascontiguousarray(prob.topk_weights)).pin_memory()
+    hout = torch.empty((cfg.tokens, cfg.hidden), dtype=torch.float32).pin_memory()
+    dx = torch.empty_like(hx, device=dev)
+    dids = torch.empty_like(hids, device=dev)
+    dw = torch.empty_like(hw, device=dev)
+    n = max(1, min(steps, 2000))
+
+    def one(i):
+        dx.copy_(hx, non_blocking=True)
+        dids.copy_(hids, non_blocking=True)
+        dw.copy_(hw, non_blocking=True)
+        layers[i % len(layers)].forward(dx, dids, dw, bufs, path=args.path, split=args.split)
+        hout.copy_(bufs.out[: cfg.tokens], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(max(3, warmup)):
+            one(i)
+    stream.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for i in range(n):
+            one(i)
+        ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = reduce_max(ev0.elapsed_time(ev1))
+    h2d = hx.numel() * 2 + hids.numel() * 4 + hw.numel() * 4
+    d2h = hout.numel() * 4
+    return {"value": world * cfg.tokens * n / (ms * 1e-3), "unit": "tokens/s", "steps": n,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "api": "NVFP4MoE.forward (four C-ABI calls, eager launches)"}
+
+
+# --------------------------------------------------------------------------- #
+# The CPU oracle as baseline / reference arm
+# --------------------------------------------------------------------------- #
+
+def _oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        return 1
+
+
+def _oracle_sample(prob):
+    """A bounded slice of the workload for the oracle: at most 2 tokens' full forward."""
+    from workloads import make_problem
+    import dataclasses
+    cfg = prob.cfg
+    m = min(cfg.tokens, 2 if cfg.tokens > 1 else 1)
+    sub = make_problem(cfg)
+    sub.x_bf16 = prob.x_bf16[:m].copy()
+    sub.topk_ids = prob.topk_ids[:m].copy()
+    sub.topk_weights = prob.topk_weights[:m].copy()
+    sub.cfg = dataclasses.replace(cfg, tokens=m)
+    return sub
+
+
+def _oracle_step(sub):
+    import oracle as orc
+    cfg = sub.cfg
+    fns = [lambda e, mm=mm: sub.expert_weight(mm, e, cache=True) for mm in (0, 1, 2)]
+    orc.moe_forward(sub.x_bf16, sub.topk_ids, sub.topk_weights, cfg.experts, *fns,
+                    hidden=cfg.hidden, inter=cfg.inter)
+
+
+def cpu_baseline(prob, budget_s=12.0):
+    sub = _oracle_sample(prob)
+    _oracle_step(sub)  # draws (and caches) the sample's expert bytes
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        _oracle_step(sub)
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": sub.cfg.tokens * n / dt, "unit": "tokens/s", "cores": _oracle_threads(),
+            "kind": "oracle",
+            "sample": f"{n} fp64 oracle forwards of the first {sub.cfg.tokens} token(s) of "
+                      f"{prob.cfg.name} (route sort, dequantise the routed experts, gate+up SiLU, "
+                      f"down, blend), weight bytes pre-drawn, {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    from workloads import make_problem
+    prob = make_problem(args.config)
+    steps = args.steps if args.steps is not None else 5
+    warmup = max(args.warmup, 3)
+    sub = _oracle_sample(prob)
+    for _ in range(min(warmup, 1) if steps > 20 else warmup):
+        _oracle_step(sub)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        _oracle_step(sub)
+    dt = time.perf_counter() - t0
+    value = sub.cfg.tokens * steps / dt
+    cores = _oracle_threads()
+    sample = (f"each step: fp64 oracle forward of the first {sub.cfg.tokens} token(s) of "
+              f"{prob.cfg.name}")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": 0, "steps": steps, "warmup": warmup, "ms_per_step": dt * 1e3 / steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": prob.cfg.name, "hidden": prob.cfg.hidden, "inter": prob.cfg.inter,
+                       "experts": prob.cfg.experts, "topk": prob.cfg.topk, "tokens": prob.cfg.tokens},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local = dist_info()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

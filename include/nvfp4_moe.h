@@ -1,0 +1,215 @@
+/*
+ * nvfp4_moe.h - C ABI of the grouped NVFP4 MoE expert forward (sm_100a).
+ *
+ * The forward has four steps, one entry point each, run in this order on one
+ * CUDA stream:
+ *
+ *   1. nvfp4_moe_route_sort    group the routed (token, expert) pairs by expert
+ *   2. nvfp4_moe_gate_up_silu  act = SiLU(x Wg^T) * (x Wu^T), FP32, per sorted row
+ *   3. nvfp4_moe_down          y   = act Wd^T, FP32, per sorted row
+ *   4. nvfp4_moe_blend         out[t] = sum_s w[t,s] * y[pos(t,s)], token order
+ *
+ * plus the load-time twin builder nvfp4_moe_transpose_u8.
+ *
+ * Sources.  The operations and layouts are those of the rustdoc source pages of
+ * the "metrale" project:
+ *   - metrale_model_layers/layers/ops/nvfp4_moe_grouped.rs: module doc (rows
+ *     grouped by expert by `moe_fp8_grouped_sort`, active experts listed,
+ *     intermediates laid out by sorted position, blend
+ *     `moe_weighted_sum_blend_fp8_grouped`), `Nvfp4ExpertTables`,
+ *     `moe_expert_gate_up_act_nvfp4_grouped`, `moe_expert_down_act_nvfp4_grouped`;
+ *   - metrale_model_arch/tp_shard/quant_shard.rs, layout comment: NVFP4 weight
+ *     [N, K/2] u8 packed E2M1, weight_scale [N, K/16] u8 E4M3, one f32
+ *     weight_scale_2;
+ *   - metrale_model_layers/weight_map/quantized/transpose.rs,
+ *     `transpose_for_gemm_gs` and its host byte loop (transpose_u8);
+ *   - metrale_model_layers/weight_map/expert.rs, `ExpertWeight::null`: the MoE
+ *     kernels skip a NULL expert.
+ *
+ * Conventions common to every entry point.
+ *   - All tensor pointers are DEVICE pointers, owned by the caller, row-major
+ *     and contiguous.  The library allocates no memory, never synchronises the
+ *     stream and never reads device data on the host.
+ *   - Return value: NVFP4_MOE_OK, or an error code from nvfp4_moe_status.
+ *     Argument errors are detected on the host before any launch (nothing is
+ *     launched then); a failed launch returns NVFP4_MOE_ECUDA.  Nothing is
+ *     thrown across the ABI, and no kernel traps.
+ *   - NVFP4 weight value:  W[n,k] = E2M1(nibble k of row n)
+ *                                   * E4M3(scale[n, k/16]) * weight_scale_2.
+ *     NIBBLE ORDER: byte j of a row holds k = 2j in its LOW nibble and
+ *     k = 2j+1 in its HIGH nibble.  E4M3 is the finite "FN" variant (max 448);
+ *     its NaN codes 0x7F / 0xFF are not valid block scales.
+ *   - A pair is p = token * topk + slot.  A "sorted position" is a pair's index
+ *     after grouping by expert (ascending expert id, ties by ascending p).
+ *   - A NULL expert (NULL entry in its packed_ptrs table) is skipped: its rows
+ *     of act / y are written as zeros.
+ *   - Shape rules: hidden and intermediate are multiples of 256 (one 16-byte
+ *     scale load covers 256 k); 1 <= topk <= num_experts <= 1024.
+ */
+#ifndef NVFP4_MOE_H_
+#define NVFP4_MOE_H_
+
+#include <stdint.h>
+#include <cuda_runtime.h>
+
+#if defined(NVFP4_MOE_BUILD) && defined(__GNUC__)
+#define NVFP4_MOE_API __attribute__((visibility("default")))
+#else
+#define NVFP4_MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NVFP4_MOE_OK = 0,
+  NVFP4_MOE_EINVAL = 1, /* NULL pointer or invalid argument value            */
+  NVFP4_MOE_ESHAPE = 2, /* shape outside the supported set (see above)       */
+  NVFP4_MOE_ECUDA = 3   /* a CUDA call or kernel launch failed               */
+} nvfp4_moe_status;
+
+/*
+ * One NVFP4 projection across the routed experts (Nvfp4ExpertTables in
+ * nvfp4_moe_grouped.rs).  All three are DEVICE arrays of length num_experts:
+ *   packed_ptrs[e]  device pointer to expert e's packed E2M1 bytes  u8 [N, K/2]
+ *                   (16-byte aligned), or NULL for a NULL expert;
+ *   scale_ptrs[e]   device pointer to its E4M3 block scales          u8 [N, K/16]
+ *                   (16-byte aligned);
+ *   scale2[e]       its f32 weight_scale_2.
+ */
+typedef struct {
+  const void* const* packed_ptrs;
+  const void* const* scale_ptrs;
+  const float* scale2;
+} nvfp4_expert_tables;
+
+/*
+ * Launch options of the two projection steps (nvfp4_moe_*_ex).  Zero-filled
+ * options, or a NULL pointer, mean "choose from the shape":
+ *   path   0 auto; 1 decode path (register-fed warp MMA over streamed weights,
+ *          for few rows per expert); 2 prefill path (tcgen05 MMA with TMEM
+ *          accumulators over shared-memory-dequantised weight tiles).
+ *   split  decode path only: 0 auto, or 1, 2, 4 = warps of a CTA that split K.
+ * Both paths compute the same function; the choice affects only speed and the
+ * FP32 summation order.
+ */
+typedef struct {
+  int32_t path;
+  int32_t split;
+} nvfp4_moe_launch_opts;
+
+/*
+ * Step 1: group the routed pairs by expert (moe_fp8_grouped_sort, named in the
+ * module doc of nvfp4_moe_grouped.rs).
+ *
+ *   topk_ids        i32 [num_tokens, topk]  expert id of each pair
+ *   expert_offsets  i32 [num_experts + 1]   out: exclusive prefix of per-expert
+ *                                           pair counts; [E] = kept pairs
+ *   sorted_pair_ids i32 [P]                 out: pair id at each sorted position;
+ *                                           positions >= kept pairs hold -1
+ *   pair_pos        i32 [P]                 out: sorted position of each pair
+ *                                           (inverse of sorted_pair_ids), -1 if dropped
+ *   active_experts  i32 [num_experts]       out: experts with >= 1 pair, ascending,
+ *                                           padded with -1
+ *   active_count    i32 [1]                 out: number of active experts
+ *   status          i32 [1] or NULL         out: 0, or 1 if some id was outside
+ *                                           [0, num_experts) (that pair is dropped)
+ * P = num_tokens * topk, at most 1<<24.  The result is unique (bit-exact).
+ */
+NVFP4_MOE_API int nvfp4_moe_route_sort(const int32_t* topk_ids, uint32_t num_tokens, uint32_t topk,
+                         uint32_t num_experts, int32_t* expert_offsets,
+                         int32_t* sorted_pair_ids, int32_t* pair_pos,
+                         int32_t* active_experts, int32_t* active_count,
+                         int32_t* status, cudaStream_t stream);
+
+/*
+ * Step 2: grouped gate+up with the SiLU product kept in FP32
+ * (moe_expert_gate_up_act_nvfp4_grouped in nvfp4_moe_grouped.rs).
+ *
+ *   x           bf16 bits [num_tokens, k_hidden]
+ *   gate, up    tables of [n_inter, k_hidden] NVFP4 weights
+ *   act         f32 [P, n_inter]  out: row r = sorted position r:
+ *               act[r, n] = SiLU(g) * u, g = sum_k Wg[n,k] x[t,k], u likewise,
+ *               t = sorted_pair_ids[r] / topk.  Rows >= kept pairs are untouched.
+ *   expert_offsets, sorted_pair_ids, active_experts, active_count: from step 1.
+ *   cap         upper bound on active experts used to size the launch; pass
+ *               nvfp4_moe_active_cap(num_experts, P).
+ * Gate and up are not rounded to BF16 before SiLU.  n_inter % 64 == 0.
+ */
+NVFP4_MOE_API int nvfp4_moe_gate_up_silu(const uint16_t* x, nvfp4_expert_tables gate,
+                           nvfp4_expert_tables up, float* act,
+                           const int32_t* expert_offsets, const int32_t* sorted_pair_ids,
+                           const int32_t* active_experts, const int32_t* active_count,
+                           uint32_t n_inter, uint32_t k_hidden, uint32_t cap,
+                           uint32_t num_tokens, uint32_t topk, cudaStream_t stream);
+
+/* nvfp4_moe_gate_up_silu with explicit launch options (NULL = automatic). */
+NVFP4_MOE_API int nvfp4_moe_gate_up_silu_ex(const uint16_t* x, nvfp4_expert_tables gate,
+                              nvfp4_expert_tables up, float* act,
+                              const int32_t* expert_offsets, const int32_t* sorted_pair_ids,
+                              const int32_t* active_experts, const int32_t* active_count,
+                              uint32_t n_inter, uint32_t k_hidden, uint32_t cap,
+                              uint32_t num_tokens, uint32_t topk,
+                              const nvfp4_moe_launch_opts* opts, cudaStream_t stream);
+
+/*
+ * Step 3: grouped down projection over the FP32 SiLU products
+ * (moe_expert_down_act_nvfp4_grouped in nvfp4_moe_grouped.rs).
+ *
+ *   act     f32 [num_pairs, k_inter]  from step 2 (rows are sorted positions)
+ *   down    table of [n_hidden, k_inter] NVFP4 weights
+ *   y       f32 [num_pairs, n_hidden] out: y[r, j] = sum_i Wd[j,i] act[r,i].
+ *           Rows >= kept pairs are untouched.
+ * n_hidden % 128 == 0.
+ */
+NVFP4_MOE_API int nvfp4_moe_down(const float* act, nvfp4_expert_tables down, float* y,
+                   const int32_t* expert_offsets, const int32_t* active_experts,
+                   const int32_t* active_count, uint32_t n_hidden, uint32_t k_inter,
+                   uint32_t cap, uint32_t num_pairs, cudaStream_t stream);
+
+/* nvfp4_moe_down with explicit launch options (NULL = automatic). */
+NVFP4_MOE_API int nvfp4_moe_down_ex(const float* act, nvfp4_expert_tables down, float* y,
+                      const int32_t* expert_offsets, const int32_t* active_experts,
+                      const int32_t* active_count, uint32_t n_hidden, uint32_t k_inter,
+                      uint32_t cap, uint32_t num_pairs, const nvfp4_moe_launch_opts* opts,
+                      cudaStream_t stream);
+
+/*
+ * Step 4: router-weighted blend back into token order
+ * (moe_weighted_sum_blend_fp8_grouped, named in the module doc of
+ * nvfp4_moe_grouped.rs).
+ *
+ *   y            f32 [P, hidden]            from step 3
+ *   topk_weights f32 [num_tokens, topk]
+ *   pair_pos     i32 [P]                    from step 1 (-1 = dropped pair)
+ *   out_f32      f32 [num_tokens, hidden]   out: sum over s = 0..topk-1, in that
+ *                                           order, of w[t,s] * y[pair_pos[t*topk+s]]
+ *   out_bf16     bf16 bits [num_tokens, hidden] or NULL: out_f32 rounded to
+ *                nearest even.
+ * hidden % 4 == 0.  Deterministic: no atomics.
+ */
+NVFP4_MOE_API int nvfp4_moe_blend(const float* y, const float* topk_weights, const int32_t* pair_pos,
+                    float* out_f32, uint16_t* out_bf16, uint32_t num_tokens, uint32_t topk,
+                    uint32_t hidden, cudaStream_t stream);
+
+/*
+ * Load-time twin builder: byte transpose [rows, cols] -> [cols, rows]
+ * (transpose_u8, used by transpose_for_gemm_gs in transpose.rs, whose host
+ * fallback loop t[j*rows + i] = b[i*cols + j] defines it).  src and dst must
+ * not overlap.  Bit-exact.
+ */
+NVFP4_MOE_API int nvfp4_moe_transpose_u8(const uint8_t* src, uint8_t* dst, uint32_t rows, uint32_t cols,
+                           cudaStream_t stream);
+
+/* Host helper: launch bound on active experts, min(num_experts, num_pairs). */
+NVFP4_MOE_API uint32_t nvfp4_moe_active_cap(uint32_t num_experts, uint32_t num_pairs);
+
+/* Static, human-readable name of a status code. */
+NVFP4_MOE_API const char* nvfp4_moe_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_MOE_H_ */

@@ -1,0 +1,24 @@
+"""Grouped NVFP4 weight-quantised MoE expert forward for B200 (sm_100a).
+
+The compute lives in ``libnvfp4moe.so`` (hand-written CUDA, C ABI in
+include/nvfp4_moe.h); this package is its thin Python binding plus device
+containers.  Importing it without the built library raises ImportError.
+"""
+
+from ._binding import (  # noqa: F401
+    LIB_PATH,
+    PATH_AUTO,
+    PATH_DECODE,
+    PATH_PREFILL,
+    ExpertTables,
+    LaunchOpts,
+    NVFP4MoEError,
+    active_cap,
+    blend,
+    down,
+    exported_symbols,
+    gate_up_silu,
+    route_sort,
+    transpose_u8,
+)
+from .layer import MoEBuffers, NVFP4MoE, NVFP4Projection  # noqa: F401

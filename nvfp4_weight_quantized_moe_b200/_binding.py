@@ -1,0 +1,169 @@
+"""ctypes binding of the C ABI in include/nvfp4_moe.h.
+
+Argument marshalling only: each function checks dtypes, devices and
+contiguity of the torch tensors it is given, passes their device pointers and
+sizes to the library entry point of the same name, and raises
+``NVFP4MoEError`` on a non-zero status.  Every step of the forward runs in
+the library's CUDA kernels; there is no fallback.  If the library is missing
+the import fails.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG_DIR, "libnvfp4moe.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m nvfp4_weight_quantized_moe_b200.build` "
+        "(nvcc, sm_100a). There is no CPU fallback.")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+c_void_p = ctypes.c_void_p
+c_u32 = ctypes.c_uint32
+c_int = ctypes.c_int
+
+
+class ExpertTables(ctypes.Structure):
+    """nvfp4_expert_tables: three device arrays of length num_experts."""
+    _fields_ = [("packed_ptrs", c_void_p), ("scale_ptrs", c_void_p), ("scale2", c_void_p)]
+
+
+class LaunchOpts(ctypes.Structure):
+    """nvfp4_moe_launch_opts."""
+    _fields_ = [("path", ctypes.c_int32), ("split", ctypes.c_int32)]
+
+
+PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
+
+_sig = {
+    "nvfp4_moe_route_sort": (c_int, [c_void_p, c_u32, c_u32, c_u32, c_void_p, c_void_p, c_void_p,
+                                     c_void_p, c_void_p, c_void_p, c_void_p]),
+    "nvfp4_moe_gate_up_silu": (c_int, [c_void_p, ExpertTables, ExpertTables, c_void_p, c_void_p,
+                                       c_void_p, c_void_p, c_void_p, c_u32, c_u32, c_u32, c_u32,
+                                       c_u32, c_void_p]),
+    "nvfp4_moe_gate_up_silu_ex": (c_int, [c_void_p, ExpertTables, ExpertTables, c_void_p, c_void_p,
+                                          c_void_p, c_void_p, c_void_p, c_u32, c_u32, c_u32, c_u32,
+                                          c_u32, ctypes.POINTER(LaunchOpts), c_void_p]),
+    "nvfp4_moe_down": (c_int, [c_void_p, ExpertTables, c_void_p, c_void_p, c_void_p, c_void_p,
+                               c_u32, c_u32, c_u32, c_u32, c_void_p]),
+    "nvfp4_moe_down_ex": (c_int, [c_void_p, ExpertTables, c_void_p, c_void_p, c_void_p, c_void_p,
+                                  c_u32, c_u32, c_u32, c_u32, ctypes.POINTER(LaunchOpts), c_void_p]),
+    "nvfp4_moe_blend": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_u32, c_u32,
+                                c_u32, c_void_p]),
+    "nvfp4_moe_transpose_u8": (c_int, [c_void_p, c_void_p, c_u32, c_u32, c_void_p]),
+    "nvfp4_moe_active_cap": (c_u32, [c_u32, c_u32]),
+    "nvfp4_moe_status_string": (ctypes.c_char_p, [c_int]),
+}
+for _name, (_res, _args) in _sig.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+
+class NVFP4MoEError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        msg = _lib.nvfp4_moe_status_string(status).decode()
+        super().__init__(f"{fn} returned {status} ({msg})")
+        self.status = status
+
+
+def exported_symbols():
+    """Names the binding resolves in the library."""
+    return sorted(_sig)
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise NVFP4MoEError(fn, status)
+
+
+def _ptr(t: Optional[torch.Tensor], dtype=None, name="tensor") -> Optional[int]:
+    if t is None:
+        return None
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _opts(path: int, split: int):
+    if path == 0 and split == 0:
+        return None
+    return ctypes.byref(LaunchOpts(path, split))
+
+
+def active_cap(num_experts: int, num_pairs: int) -> int:
+    return int(_lib.nvfp4_moe_active_cap(num_experts, num_pairs))
+
+
+def route_sort(topk_ids, num_experts, expert_offsets, sorted_pair_ids, pair_pos,
+               active_experts, active_count, status=None, stream=None) -> None:
+    m, k = topk_ids.shape
+    _check("nvfp4_moe_route_sort", _lib.nvfp4_moe_route_sort(
+        _ptr(topk_ids, torch.int32, "topk_ids"), m, k, num_experts,
+        _ptr(expert_offsets, torch.int32, "expert_offsets"),
+        _ptr(sorted_pair_ids, torch.int32, "sorted_pair_ids"),
+        _ptr(pair_pos, torch.int32, "pair_pos"),
+        _ptr(active_experts, torch.int32, "active_experts"),
+        _ptr(active_count, torch.int32, "active_count"),
+        _ptr(status, torch.int32, "status"), _stream(stream)))
+
+
+def gate_up_silu(x, gate: ExpertTables, up: ExpertTables, act, expert_offsets, sorted_pair_ids,
+                 active_experts, active_count, n_inter, k_hidden, cap, num_tokens, topk,
+                 path=0, split=0, stream=None) -> None:
+    if x.dtype not in (torch.bfloat16, torch.uint16, torch.int16):
+        raise TypeError("x: expected bf16 (or its uint16 bits)")
+    _check("nvfp4_moe_gate_up_silu_ex", _lib.nvfp4_moe_gate_up_silu_ex(
+        _ptr(x, None, "x"), gate, up, _ptr(act, torch.float32, "act"),
+        _ptr(expert_offsets, torch.int32, "expert_offsets"),
+        _ptr(sorted_pair_ids, torch.int32, "sorted_pair_ids"),
+        _ptr(active_experts, torch.int32, "active_experts"),
+        _ptr(active_count, torch.int32, "active_count"),
+        n_inter, k_hidden, cap, num_tokens, topk, _opts(path, split), _stream(stream)))
+
+
+def down(act, down_w: ExpertTables, y, expert_offsets, active_experts, active_count,
+         n_hidden, k_inter, cap, num_pairs, path=0, split=0, stream=None) -> None:
+    _check("nvfp4_moe_down_ex", _lib.nvfp4_moe_down_ex(
+        _ptr(act, torch.float32, "act"), down_w, _ptr(y, torch.float32, "y"),
+        _ptr(expert_offsets, torch.int32, "expert_offsets"),
+        _ptr(active_experts, torch.int32, "active_experts"),
+        _ptr(active_count, torch.int32, "active_count"),
+        n_hidden, k_inter, cap, num_pairs, _opts(path, split), _stream(stream)))
+
+
+def blend(y, topk_weights, pair_pos, out_f32, out_bf16=None, stream=None) -> None:
+    m, k = topk_weights.shape
+    hidden = out_f32.shape[1]
+    _check("nvfp4_moe_blend", _lib.nvfp4_moe_blend(
+        _ptr(y, torch.float32, "y"), _ptr(topk_weights, torch.float32, "topk_weights"),
+        _ptr(pair_pos, torch.int32, "pair_pos"), _ptr(out_f32, torch.float32, "out_f32"),
+        _ptr(out_bf16, None, "out_bf16"), m, k, hidden, _stream(stream)))
+
+
+def transpose_u8(src, dst, stream=None) -> None:
+    rows, cols = src.shape
+    if tuple(dst.shape) != (cols, rows):
+        raise ValueError("dst must be [cols, rows]")
+    _check("nvfp4_moe_transpose_u8", _lib.nvfp4_moe_transpose_u8(
+        _ptr(src, torch.uint8, "src"), _ptr(dst, torch.uint8, "dst"), rows, cols, _stream(stream)))

@@ -1,0 +1,207 @@
+// C ABI of the grouped NVFP4 MoE expert forward: argument checks on the host,
+// path choice, launches.  Declarations and argument contracts: include/nvfp4_moe.h.
+
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "../../include/nvfp4_moe.h"
+#include "kernels.h"
+
+namespace nvm {
+
+cudaError_t ensure_dynamic_smem(const void* kernel, int bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> done;
+  std::lock_guard<std::mutex> lock(mu);
+  auto key = std::make_pair(kernel, dev);
+  auto it = done.find(key);
+  if (it != done.end() && it->second >= bytes) return cudaSuccess;
+  err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (err == cudaSuccess) done[key] = bytes;
+  return err;
+}
+
+namespace {
+
+constexpr uint32_t kMaxExperts = 1024;
+constexpr uint64_t kMaxPairs = 1ull << 24;
+
+bool tables_ok(const nvfp4_expert_tables& t) {
+  return t.packed_ptrs != nullptr && t.scale_ptrs != nullptr && t.scale2 != nullptr;
+}
+
+int status_of(cudaError_t err) { return err == cudaSuccess ? NVFP4_MOE_OK : NVFP4_MOE_ECUDA; }
+
+// Decode-path K split from the average rows per active expert: one row per
+// expert needs the four warps of a CTA on one output tile to have enough loads
+// in flight; many rows per expert give each warp its own tile.
+int auto_split(uint64_t pairs, uint32_t cap) {
+  const uint64_t rows_per_expert = cap ? pairs / cap : pairs;
+  if (rows_per_expert < 2) return 4;
+  if (rows_per_expert < 8) return 2;
+  return 1;
+}
+
+bool split_ok(int s) { return s == 1 || s == 2 || s == 4; }
+
+}  // namespace
+}  // namespace nvm
+
+using namespace nvm;
+
+extern "C" {
+
+uint32_t nvfp4_moe_active_cap(uint32_t num_experts, uint32_t num_pairs) {
+  return num_experts < num_pairs ? num_experts : num_pairs;
+}
+
+const char* nvfp4_moe_status_string(int status) {
+  switch (status) {
+    case NVFP4_MOE_OK: return "ok";
+    case NVFP4_MOE_EINVAL: return "invalid argument (NULL pointer or bad value)";
+    case NVFP4_MOE_ESHAPE: return "unsupported shape";
+    case NVFP4_MOE_ECUDA: return "CUDA launch or runtime error";
+    default: return "unknown status";
+  }
+}
+
+int nvfp4_moe_route_sort(const int32_t* topk_ids, uint32_t num_tokens, uint32_t topk,
+                         uint32_t num_experts, int32_t* expert_offsets,
+                         int32_t* sorted_pair_ids, int32_t* pair_pos,
+                         int32_t* active_experts, int32_t* active_count,
+                         int32_t* status, cudaStream_t stream) {
+  if (expert_offsets == nullptr || active_experts == nullptr || active_count == nullptr)
+    return NVFP4_MOE_EINVAL;
+  if (num_experts == 0 || num_experts > kMaxExperts || topk == 0 || topk > num_experts)
+    return NVFP4_MOE_ESHAPE;
+  const uint64_t pairs = (uint64_t)num_tokens * topk;
+  if (pairs > kMaxPairs) return NVFP4_MOE_ESHAPE;
+  if (pairs > 0 && (topk_ids == nullptr || sorted_pair_ids == nullptr || pair_pos == nullptr))
+    return NVFP4_MOE_EINVAL;
+  return status_of(launch_route_sort(topk_ids, (uint32_t)pairs, num_experts, expert_offsets,
+                                     sorted_pair_ids, pair_pos, active_experts, active_count,
+                                     status, stream));
+}
+
+int nvfp4_moe_gate_up_silu_ex(const uint16_t* x, nvfp4_expert_tables gate,
+                              nvfp4_expert_tables up, float* act,
+                              const int32_t* expert_offsets, const int32_t* sorted_pair_ids,
+                              const int32_t* active_experts, const int32_t* active_count,
+                              uint32_t n_inter, uint32_t k_hidden, uint32_t cap,
+                              uint32_t num_tokens, uint32_t topk,
+                              const nvfp4_moe_launch_opts* opts, cudaStream_t stream) {
+  if (n_inter == 0 || n_inter % 64 != 0 || k_hidden == 0 || k_hidden % 256 != 0 || topk == 0 ||
+      cap > 65535)
+    return NVFP4_MOE_ESHAPE;
+  const uint64_t pairs = (uint64_t)num_tokens * topk;
+  if (pairs > kMaxPairs) return NVFP4_MOE_ESHAPE;
+  if (pairs == 0 || cap == 0) return NVFP4_MOE_OK;
+  if (x == nullptr || act == nullptr || expert_offsets == nullptr || sorted_pair_ids == nullptr ||
+      active_experts == nullptr || active_count == nullptr || !tables_ok(gate) || !tables_ok(up))
+    return NVFP4_MOE_EINVAL;
+  const int path = opts ? opts->path : 0;
+  int split = opts ? opts->split : 0;
+  if (path != 0 && path != 1) return NVFP4_MOE_EINVAL;
+  if (split == 0) split = auto_split(pairs, cap);
+  if (!split_ok(split)) return NVFP4_MOE_EINVAL;
+  GroupedArgs a{};
+  a.src = x;
+  a.packed0 = gate.packed_ptrs;
+  a.scale0 = gate.scale_ptrs;
+  a.s2_0 = gate.scale2;
+  a.packed1 = up.packed_ptrs;
+  a.scale1 = up.scale_ptrs;
+  a.s2_1 = up.scale2;
+  a.out = act;
+  a.offsets = expert_offsets;
+  a.sorted_pair_ids = sorted_pair_ids;
+  a.active_experts = active_experts;
+  a.active_count = active_count;
+  a.N = n_inter;
+  a.K = k_hidden;
+  a.topk = topk;
+  return status_of(launch_grouped(kModeGateUp, split, 4 / split, a, cap, stream));
+}
+
+int nvfp4_moe_gate_up_silu(const uint16_t* x, nvfp4_expert_tables gate,
+                           nvfp4_expert_tables up, float* act,
+                           const int32_t* expert_offsets, const int32_t* sorted_pair_ids,
+                           const int32_t* active_experts, const int32_t* active_count,
+                           uint32_t n_inter, uint32_t k_hidden, uint32_t cap,
+                           uint32_t num_tokens, uint32_t topk, cudaStream_t stream) {
+  return nvfp4_moe_gate_up_silu_ex(x, gate, up, act, expert_offsets, sorted_pair_ids,
+                                   active_experts, active_count, n_inter, k_hidden, cap,
+                                   num_tokens, topk, nullptr, stream);
+}
+
+int nvfp4_moe_down_ex(const float* act, nvfp4_expert_tables down, float* y,
+                      const int32_t* expert_offsets, const int32_t* active_experts,
+                      const int32_t* active_count, uint32_t n_hidden, uint32_t k_inter,
+                      uint32_t cap, uint32_t num_pairs, const nvfp4_moe_launch_opts* opts,
+                      cudaStream_t stream) {
+  if (n_hidden == 0 || n_hidden % 128 != 0 || k_inter == 0 || k_inter % 256 != 0 || cap > 65535)
+    return NVFP4_MOE_ESHAPE;
+  if (num_pairs > kMaxPairs) return NVFP4_MOE_ESHAPE;
+  if (num_pairs == 0 || cap == 0) return NVFP4_MOE_OK;
+  if (act == nullptr || y == nullptr || expert_offsets == nullptr || active_experts == nullptr ||
+      active_count == nullptr || !tables_ok(down))
+    return NVFP4_MOE_EINVAL;
+  const int path = opts ? opts->path : 0;
+  int split = opts ? opts->split : 0;
+  if (path != 0 && path != 1) return NVFP4_MOE_EINVAL;
+  if (split == 0) split = auto_split(num_pairs, cap);
+  if (!split_ok(split)) return NVFP4_MOE_EINVAL;
+  GroupedArgs a{};
+  a.src = act;
+  a.packed0 = down.packed_ptrs;
+  a.scale0 = down.scale_ptrs;
+  a.s2_0 = down.scale2;
+  a.out = y;
+  a.offsets = expert_offsets;
+  a.active_experts = active_experts;
+  a.active_count = active_count;
+  a.N = n_hidden;
+  a.K = k_inter;
+  a.topk = 1;
+  return status_of(launch_grouped(kModeDown, split, 4 / split, a, cap, stream));
+}
+
+int nvfp4_moe_down(const float* act, nvfp4_expert_tables down, float* y,
+                   const int32_t* expert_offsets, const int32_t* active_experts,
+                   const int32_t* active_count, uint32_t n_hidden, uint32_t k_inter,
+                   uint32_t cap, uint32_t num_pairs, cudaStream_t stream) {
+  return nvfp4_moe_down_ex(act, down, y, expert_offsets, active_experts, active_count, n_hidden,
+                           k_inter, cap, num_pairs, nullptr, stream);
+}
+
+int nvfp4_moe_blend(const float* y, const float* topk_weights, const int32_t* pair_pos,
+                    float* out_f32, uint16_t* out_bf16, uint32_t num_tokens, uint32_t topk,
+                    uint32_t hidden, cudaStream_t stream) {
+  // One grid row per token: at most 65535 tokens per call.
+  if (hidden == 0 || hidden % 4 != 0 || topk == 0 || num_tokens > 65535 ||
+      (uint64_t)num_tokens * topk > kMaxPairs)
+    return NVFP4_MOE_ESHAPE;
+  if (num_tokens == 0) return NVFP4_MOE_OK;
+  if (y == nullptr || topk_weights == nullptr || pair_pos == nullptr || out_f32 == nullptr)
+    return NVFP4_MOE_EINVAL;
+  return status_of(launch_blend(y, topk_weights, pair_pos, out_f32, out_bf16, num_tokens, topk,
+                                hidden, stream));
+}
+
+int nvfp4_moe_transpose_u8(const uint8_t* src, uint8_t* dst, uint32_t rows, uint32_t cols,
+                           cudaStream_t stream) {
+  if (rows == 0 || cols == 0) return NVFP4_MOE_OK;
+  if (src == nullptr || dst == nullptr) return NVFP4_MOE_EINVAL;
+  if (rows > 65535u * 32u || cols > 2147483647u / 2) return NVFP4_MOE_ESHAPE;
+  const uint64_t bytes = (uint64_t)rows * cols;
+  const uintptr_t s = reinterpret_cast<uintptr_t>(src), d = reinterpret_cast<uintptr_t>(dst);
+  if (s < d + bytes && d < s + bytes) return NVFP4_MOE_EINVAL;  // overlapping buffers
+  return status_of(launch_transpose_u8(src, dst, rows, cols, stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,51 @@
+// Internal launch interface between the C ABI (abi.cu) and the kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace nvm {
+
+enum { kModeGateUp = 0, kModeDown = 1 };
+
+// Arguments of the grouped projection kernels.  Mode gate+up reads BF16 x
+// [M, K] and two weight tables (gate, up) with the same [N, K]; mode down
+// reads FP32 act [P, K] and one table.  `out` is [P, N] FP32 by sorted position.
+struct GroupedArgs {
+  const void* src;
+  const void* const* packed0;
+  const void* const* scale0;
+  const float* s2_0;
+  const void* const* packed1;
+  const void* const* scale1;
+  const float* s2_1;
+  float* out;
+  const int32_t* offsets;
+  const int32_t* sorted_pair_ids;
+  const int32_t* active_experts;
+  const int32_t* active_count;
+  uint32_t N, K, topk;
+};
+
+// Decode-shaped path (register-fed tensor-core MMA), grouped_mma.cu.
+// split in {1, 2, 4} with tiles = 4 / split.
+cudaError_t launch_grouped(int mode, int split, int tiles, const GroupedArgs& a, uint32_t cap,
+                           cudaStream_t stream);
+int grouped_rows_per_cta(int mode, int split);
+
+cudaError_t launch_route_sort(const int32_t* topk_ids, uint32_t num_pairs, uint32_t num_experts,
+                              int32_t* expert_offsets, int32_t* sorted_pair_ids, int32_t* pair_pos,
+                              int32_t* active_experts, int32_t* active_count, int32_t* status,
+                              cudaStream_t stream);
+
+cudaError_t launch_blend(const float* y, const float* topk_weights, const int32_t* pair_pos,
+                         float* out_f32, uint16_t* out_bf16, uint32_t num_tokens, uint32_t topk,
+                         uint32_t hidden, cudaStream_t stream);
+
+cudaError_t launch_transpose_u8(const uint8_t* src, uint8_t* dst, uint32_t rows, uint32_t cols,
+                                cudaStream_t stream);
+
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device).
+cudaError_t ensure_dynamic_smem(const void* kernel, int bytes);
+
+}  // namespace nvm

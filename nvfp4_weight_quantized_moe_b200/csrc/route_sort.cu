@@ -1,0 +1,144 @@
+// Step 1 of the expert forward: group the routed (token, expert) pairs by
+// expert and list the active experts (the grouping `moe_fp8_grouped_sort`
+// provides, per the module doc of metrale_model_layers/layers/ops/
+// nvfp4_moe_grouped.rs).
+//
+// One CTA of 1024 threads does a stable counting sort in shared memory:
+//   1. per-expert counts (shared-memory atomics; counts are order-free);
+//   2. one block-wide exclusive scan gives expert_offsets and, over the
+//      "count > 0" flags, the ascending list of active experts;
+//   3. the pairs are placed in passes of 1024 in pair order.  Inside a warp,
+//      __match_any_sync finds the lanes with the same expert and the rank of a
+//      lane among them; per-warp counts per expert, scanned over the 32 warps in
+//      warp order, give each warp's base, so a pair's position is
+//      cursor[e] + warp base + lane rank: ascending pair id within an expert,
+//      the same result on every run.
+// Out-of-range ids are dropped (pair_pos = -1) and flagged in `status`.
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nvm {
+
+namespace {
+
+constexpr int kSortThreads = 1024;
+
+// Block-wide exclusive scan of one int per thread (1024 threads).
+NVM_DEV int block_exclusive_scan(int v, int* warp_tmp, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) warp_tmp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int w = warp_tmp[lane];
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += t;
+    }
+    warp_tmp[lane] = wi - w;  // exclusive warp base
+    if (lane == 31) warp_tmp[32] = wi;
+  }
+  __syncthreads();
+  const int ex = incl - v + warp_tmp[warp];
+  total = warp_tmp[32];
+  __syncthreads();
+  return ex;
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kSortThreads)
+    route_sort_kernel(const int32_t* __restrict__ ids, int P, int E, int32_t* __restrict__ offsets,
+                      int32_t* __restrict__ sorted, int32_t* __restrict__ pair_pos,
+                      int32_t* __restrict__ active, int32_t* __restrict__ active_count,
+                      int32_t* __restrict__ status) {
+  extern __shared__ int sm[];
+  int* cnt = sm;                                            // [E]
+  int* cursor = sm + E;                                     // [E]
+  uint16_t* wc = reinterpret_cast<uint16_t*>(sm + 2 * E);   // [32][E]
+  __shared__ int tmp[33];
+  __shared__ int bad;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < E; i += kSortThreads) cnt[i] = 0;
+  if (tid == 0) bad = 0;
+  __syncthreads();
+  for (int p = tid; p < P; p += kSortThreads) {
+    const int v = ids[p];
+    if ((unsigned)v < (unsigned)E) atomicAdd(&cnt[v], 1);
+    else bad = 1;
+  }
+  __syncthreads();
+
+  const int c = tid < E ? cnt[tid] : 0;
+  int kept = 0, nactive = 0;
+  const int off = block_exclusive_scan(c, tmp, kept);
+  const int arank = block_exclusive_scan(c > 0 ? 1 : 0, tmp, nactive);
+  if (tid < E) {
+    offsets[tid] = off;
+    cursor[tid] = off;
+    if (c > 0) active[arank] = tid;
+  }
+  if (tid == 0) {
+    offsets[E] = kept;
+    *active_count = nactive;
+    if (status != nullptr) *status = bad;
+  }
+  for (int i = nactive + tid; i < E; i += kSortThreads) active[i] = -1;
+  for (int i = kept + tid; i < P; i += kSortThreads) sorted[i] = -1;
+
+  for (int base = 0; base < P; base += kSortThreads) {
+    for (int i = tid; i < 32 * E; i += kSortThreads) wc[i] = 0;
+    const int p = base + tid;
+    const int v = p < P ? ids[p] : -1;
+    const bool valid = (unsigned)v < (unsigned)E;
+    const unsigned peers = __match_any_sync(0xffffffffu, valid ? v : -1);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    __syncthreads();
+    if (valid && rank == 0) wc[warp * E + v] = (uint16_t)__popc(peers);
+    __syncthreads();
+    if (tid < E) {
+      int run = 0;
+      for (int w = 0; w < 32; ++w) {
+        const int t = wc[w * E + tid];
+        wc[w * E + tid] = (uint16_t)run;
+        run += t;
+      }
+      cnt[tid] = run;
+    }
+    __syncthreads();
+    if (valid) {
+      const int pos = cursor[v] + wc[warp * E + v] + rank;
+      sorted[pos] = p;
+      pair_pos[p] = pos;
+    } else if (p < P) {
+      pair_pos[p] = -1;
+    }
+    __syncthreads();
+    if (tid < E) cursor[tid] += cnt[tid];
+    __syncthreads();
+  }
+}
+
+cudaError_t launch_route_sort(const int32_t* topk_ids, uint32_t num_pairs, uint32_t num_experts,
+                              int32_t* expert_offsets, int32_t* sorted_pair_ids, int32_t* pair_pos,
+                              int32_t* active_experts, int32_t* active_count, int32_t* status,
+                              cudaStream_t stream) {
+  const int smem = (int)num_experts * (2 * 4 + 32 * 2);
+  cudaError_t err = ensure_dynamic_smem(reinterpret_cast<const void*>(route_sort_kernel), smem);
+  if (err != cudaSuccess) return err;
+  route_sort_kernel<<<1, kSortThreads, smem, stream>>>(topk_ids, (int)num_pairs, (int)num_experts,
+                                                       expert_offsets, sorted_pair_ids, pair_pos,
+                                                       active_experts, active_count, status);
+  return cudaGetLastError();
+}
+
+}  // namespace nvm

@@ -323,28 +323,29 @@ def moe_forward_tokens(x_bf16, topk_ids, topk_weights, num_experts, gate_fn, up_
                        tokens: Sequence[int], hidden: int) -> np.ndarray:
     """out rows for the listed tokens only, computed token by token, float64.
 
-    The same expert forward written per token: for each routed slot of a token,
-    the expert's gated MLP on that token's row, weighted by its router weight.
+    The same expert forward written per token: each routed slot of a token adds
+    the expert's gated MLP of that token's row, weighted by its router weight.
     It shares no grouping with :func:`moe_forward`, so the two check each other,
-    and it lets a full-size problem be checked on a sample of tokens.  Expert
-    weights are dequantised once per expert and cached for the call.
+    and it lets a full-size problem be checked on a sample of tokens.  Experts
+    are visited one at a time (each dequantised once, then released), so only
+    one expert's dense weights are held at a time.
     """
     x = bf16_bits_to_f64(x_bf16)
     ids = np.asarray(topk_ids)
     w = np.asarray(topk_weights, dtype=np.float64)
-    cache: Dict[int, Optional[List[np.ndarray]]] = {}
     out = np.zeros((len(tokens), hidden), dtype=np.float64)
+    uses: Dict[int, List[Tuple[int, int, int]]] = {}
     for i, t in enumerate(tokens):
         for s in range(ids.shape[1]):
             e = int(ids[t, s])
-            if not 0 <= e < num_experts:
-                continue
-            if e not in cache:
-                mats = [_dense(fn, e) for fn in (gate_fn, up_fn, down_fn)]
-                cache[e] = None if any(m is None for m in mats) else mats
-            if cache[e] is None:
-                continue
-            wg, wu, wd = cache[e]
+            if 0 <= e < num_experts:
+                uses.setdefault(e, []).append((i, int(t), s))
+    for e in sorted(uses):
+        mats = [_dense(fn, e) for fn in (gate_fn, up_fn, down_fn)]
+        if any(m is None for m in mats):
+            continue
+        wg, wu, wd = mats
+        for i, t, s in uses[e]:
             h = silu(wg @ x[t]) * (wu @ x[t])
             out[i] += w[t, s] * (wd @ h)
     return out

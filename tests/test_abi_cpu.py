@@ -1,0 +1,89 @@
+"""CPU checks of the C ABI: the library loads, exports every declared symbol,
+and rejects bad arguments on the host before any CUDA call.  No compute runs."""
+
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        names |= set(re.findall(r"NVFP4_MOE_API\s+[\w\s\*]*?\b(nvfp4_moe_\w+)\s*\(", text))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from nvfp4_weight_quantized_moe_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def test_header_declares_the_five_steps():
+    names = _declared()
+    for n in ("nvfp4_moe_route_sort", "nvfp4_moe_gate_up_silu", "nvfp4_moe_down",
+              "nvfp4_moe_blend", "nvfp4_moe_transpose_u8"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_binding_resolves_every_declared_symbol(lib):
+    import nvfp4_weight_quantized_moe_b200 as m
+    assert set(m.exported_symbols()) == _declared()
+
+
+def test_host_validation_rejects_bad_shapes_without_a_gpu(lib):
+    import nvfp4_weight_quantized_moe_b200._binding as B
+    L = B._lib
+    t = B.ExpertTables(None, None, None)
+    # route_sort: E = 0, E > 1024, topk > E
+    args = [None, 1, 2, 0, ctypes.c_void_p(8), None, None, ctypes.c_void_p(8), ctypes.c_void_p(8), None, None]
+    assert L.nvfp4_moe_route_sort(*args) == 2
+    args[3] = 2048
+    assert L.nvfp4_moe_route_sort(*args) == 2
+    args[3] = 1
+    assert L.nvfp4_moe_route_sort(*args) == 2
+    # route_sort: missing outputs
+    assert L.nvfp4_moe_route_sort(None, 1, 1, 4, None, None, None, None, None, None, None) == 1
+    # gate_up: K not a multiple of 256, N not a multiple of 64
+    assert L.nvfp4_moe_gate_up_silu(None, t, t, None, None, None, None, None, 64, 100, 1, 1, 1, None) == 2
+    assert L.nvfp4_moe_gate_up_silu(None, t, t, None, None, None, None, None, 48, 256, 1, 1, 1, None) == 2
+    # gate_up: NULL tables with work to do
+    assert L.nvfp4_moe_gate_up_silu(None, t, t, None, None, None, None, None, 64, 256, 1, 1, 1, None) == 1
+    # gate_up: no tokens is a no-op
+    assert L.nvfp4_moe_gate_up_silu(None, t, t, None, None, None, None, None, 64, 256, 1, 0, 1, None) == 0
+    # down: N not a multiple of 128
+    assert L.nvfp4_moe_down(None, t, None, None, None, None, 64, 256, 1, 1, None) == 2
+    # blend: hidden % 4
+    assert L.nvfp4_moe_blend(None, None, None, None, None, 1, 1, 6, None) == 2
+    assert L.nvfp4_moe_blend(None, None, None, None, None, 0, 1, 8, None) == 0
+    # transpose: overlap and NULL
+    assert L.nvfp4_moe_transpose_u8(None, None, 4, 4, None) == 1
+    assert L.nvfp4_moe_transpose_u8(ctypes.c_void_p(4096), ctypes.c_void_p(4100), 4, 4, None) == 1
+    # launch options: bad path / split
+    bad = B.LaunchOpts(7, 0)
+    ok_t = B.ExpertTables(8, 8, 8)
+    p8 = ctypes.c_void_p(8)
+    assert L.nvfp4_moe_gate_up_silu_ex(p8, ok_t, ok_t, p8, p8, p8, p8, p8, 64, 256, 1, 1, 1,
+                                       ctypes.byref(bad), None) == 1
+    bad = B.LaunchOpts(1, 3)
+    assert L.nvfp4_moe_down_ex(p8, ok_t, p8, p8, p8, p8, 128, 256, 1, 1, ctypes.byref(bad), None) == 1
+
+
+def test_active_cap_and_status_strings(lib):
+    import nvfp4_weight_quantized_moe_b200 as m
+    assert m.active_cap(128, 8) == 8 and m.active_cap(8, 65536) == 8
+    L = m._binding._lib
+    for s in range(4):
+        assert L.nvfp4_moe_status_string(s)
