@@ -59,6 +59,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--path", type=int, default=0, help="0 auto, 1 decode, 2 prefill")
     ap.add_argument("--split", type=int, default=0)
+    ap.add_argument("--tiles", type=int, default=0)
+    ap.add_argument("--depth", type=int, default=0)
+    ap.add_argument("--replicas", type=int, default=0,
+                    help="weight replicas to rotate over (0: enough to exceed 4 x L2)")
     return ap.parse_args(argv)
 
 
@@ -209,7 +213,7 @@ def run_ours(args, rank, world, local):
     bufs = base.buffers(cfg.tokens)
     # Active experts of this batch (identical for every replica: same routing).
     with torch.cuda.stream(stream):
-        base.forward(x, ids, w, bufs, path=args.path, split=args.split)
+        base.forward(x, ids, w, bufs, **_opts(args))
     stream.synchronize()
     active = int(bufs.active_count.item())
     per_expert = base.gate.nbytes_per_expert
@@ -219,10 +223,12 @@ def run_ours(args, rank, world, local):
     free = torch.cuda.mem_get_info(dev)[0]
     layer_bytes = 3 * cfg.experts * per_expert
     replicas = int(min(replicas, max(1, (free * 0.6) // layer_bytes), 64))
+    if args.replicas > 0:
+        replicas = args.replicas
     layers = _replicate(base, replicas - 1)
 
     def step(lay):
-        lay.forward(x, ids, w, bufs, path=args.path, split=args.split)
+        lay.forward(x, ids, w, bufs, **_opts(args))
 
     # Graphs: one of R steps (one per replica) plus single-step graphs for remainders.
     with torch.cuda.stream(stream):
@@ -281,8 +287,7 @@ def run_ours(args, rank, world, local):
     def gate_up(lay):
         nvm.gate_up_silu(x, lay.gate.tables, lay.up.tables, bufs.act, bufs.expert_offsets,
                          bufs.sorted_pair_ids, bufs.active_experts, bufs.active_count,
-                         cfg.inter, cfg.hidden, cap, cfg.tokens, cfg.topk, path=args.path,
-                         split=args.split)
+                         cfg.inter, cfg.hidden, cap, cfg.tokens, cfg.topk, **_opts(args))
     with torch.cuda.graph(gu_graph, stream=stream):
         for lay in layers:
             gate_up(lay)
@@ -345,6 +350,10 @@ def run_ours(args, rank, world, local):
         dist.destroy_process_group()
 
 
+def _opts(args):
+    return dict(path=args.path, split=args.split, tiles=args.tiles, depth=args.depth)
+
+
 def _uses_prefill(args, cfg):
     return False
 
@@ -368,7 +377,7 @@ def run_e2e(layers, prob, bufs, dev, stream, steps, warmup, args, world):
         dx.copy_(hx, non_blocking=True)
         dids.copy_(hids, non_blocking=True)
         dw.copy_(hw, non_blocking=True)
-        layers[i % len(layers)].forward(dx, dids, dw, bufs, path=args.path, split=args.split)
+        layers[i % len(layers)].forward(dx, dids, dw, bufs, **_opts(args))
         hout.copy_(bufs.out[: cfg.tokens], non_blocking=True)
 
     with torch.cuda.stream(stream):

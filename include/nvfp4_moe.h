@@ -85,18 +85,24 @@ typedef struct {
 } nvfp4_expert_tables;
 
 /*
- * Launch options of the two projection steps (nvfp4_moe_*_ex).  Zero-filled
- * options, or a NULL pointer, mean "choose from the shape":
- *   path   0 auto; 1 decode path (register-fed warp MMA over streamed weights,
- *          for few rows per expert); 2 prefill path (tcgen05 MMA with TMEM
- *          accumulators over shared-memory-dequantised weight tiles).
- *   split  decode path only: 0 auto, or 1, 2, 4 = warps of a CTA that split K.
- * Both paths compute the same function; the choice affects only speed and the
- * FP32 summation order.
+ * Launch options of the two projection steps (nvfp4_moe_*_ex).  A NULL pointer,
+ * or a zero field, means "choose from the shape":
+ *   path     0 auto; 1 decode path (register-fed warp MMA over streamed weights,
+ *            for few rows per expert); 2 prefill path (tcgen05 MMA with TMEM
+ *            accumulators over shared-memory-dequantised weight tiles).
+ *   split    decode path: warps of a CTA that split K, 1, 2 or 4 (2 and 4
+ *            with tiles = 1 and depth = 2).
+ *   tiles    decode path: 8-row token tiles per pass over an expert, 1, 2 or 4
+ *            (gate+up) / 1 or 2 (down); 4 takes depth = 2.
+ *   depth    decode path: weight chunks each warp keeps in flight, 2 or 3.
+ * Every choice computes the same function; it affects speed and the FP32
+ * summation order only.
  */
 typedef struct {
   int32_t path;
   int32_t split;
+  int32_t tiles;
+  int32_t depth;
 } nvfp4_moe_launch_opts;
 
 /*
@@ -157,23 +163,24 @@ NVFP4_MOE_API int nvfp4_moe_gate_up_silu_ex(const uint16_t* x, nvfp4_expert_tabl
  * Step 3: grouped down projection over the FP32 SiLU products
  * (moe_expert_down_act_nvfp4_grouped in nvfp4_moe_grouped.rs).
  *
- *   act     f32 [num_pairs, k_inter]  from step 2 (rows are sorted positions)
+ *   act     f32 [P, k_inter]   from step 2 (rows are sorted positions)
  *   down    table of [n_hidden, k_inter] NVFP4 weights
- *   y       f32 [num_pairs, n_hidden] out: y[r, j] = sum_i Wd[j,i] act[r,i].
+ *   y       f32 [P, n_hidden]  out: y[r, j] = sum_i Wd[j,i] act[r,i].
  *           Rows >= kept pairs are untouched.
+ *   cap, num_tokens, topk: as for step 2 (P = num_tokens * topk).
  * n_hidden % 128 == 0.
  */
 NVFP4_MOE_API int nvfp4_moe_down(const float* act, nvfp4_expert_tables down, float* y,
                    const int32_t* expert_offsets, const int32_t* active_experts,
                    const int32_t* active_count, uint32_t n_hidden, uint32_t k_inter,
-                   uint32_t cap, uint32_t num_pairs, cudaStream_t stream);
+                   uint32_t cap, uint32_t num_tokens, uint32_t topk, cudaStream_t stream);
 
 /* nvfp4_moe_down with explicit launch options (NULL = automatic). */
 NVFP4_MOE_API int nvfp4_moe_down_ex(const float* act, nvfp4_expert_tables down, float* y,
                       const int32_t* expert_offsets, const int32_t* active_experts,
                       const int32_t* active_count, uint32_t n_hidden, uint32_t k_inter,
-                      uint32_t cap, uint32_t num_pairs, const nvfp4_moe_launch_opts* opts,
-                      cudaStream_t stream);
+                      uint32_t cap, uint32_t num_tokens, uint32_t topk,
+                      const nvfp4_moe_launch_opts* opts, cudaStream_t stream);
 
 /*
  * Step 4: router-weighted blend back into token order

@@ -38,7 +38,8 @@ class ExpertTables(ctypes.Structure):
 
 class LaunchOpts(ctypes.Structure):
     """nvfp4_moe_launch_opts."""
-    _fields_ = [("path", ctypes.c_int32), ("split", ctypes.c_int32)]
+    _fields_ = [("path", ctypes.c_int32), ("split", ctypes.c_int32), ("tiles", ctypes.c_int32),
+                ("depth", ctypes.c_int32)]
 
 
 PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
@@ -53,9 +54,10 @@ _sig = {
                                           c_void_p, c_void_p, c_void_p, c_u32, c_u32, c_u32, c_u32,
                                           c_u32, ctypes.POINTER(LaunchOpts), c_void_p]),
     "nvfp4_moe_down": (c_int, [c_void_p, ExpertTables, c_void_p, c_void_p, c_void_p, c_void_p,
-                               c_u32, c_u32, c_u32, c_u32, c_void_p]),
+                               c_u32, c_u32, c_u32, c_u32, c_u32, c_void_p]),
     "nvfp4_moe_down_ex": (c_int, [c_void_p, ExpertTables, c_void_p, c_void_p, c_void_p, c_void_p,
-                                  c_u32, c_u32, c_u32, c_u32, ctypes.POINTER(LaunchOpts), c_void_p]),
+                                  c_u32, c_u32, c_u32, c_u32, c_u32, ctypes.POINTER(LaunchOpts),
+                                  c_void_p]),
     "nvfp4_moe_blend": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_u32, c_u32,
                                 c_u32, c_void_p]),
     "nvfp4_moe_transpose_u8": (c_int, [c_void_p, c_void_p, c_u32, c_u32, c_void_p]),
@@ -105,10 +107,10 @@ def _stream(stream) -> Optional[int]:
     return int(stream)
 
 
-def _opts(path: int, split: int):
-    if path == 0 and split == 0:
+def _opts(path=0, split=0, tiles=0, depth=0):
+    if not (path or split or tiles or depth):
         return None
-    return ctypes.byref(LaunchOpts(path, split))
+    return ctypes.byref(LaunchOpts(path, split, tiles, depth))
 
 
 def active_cap(num_experts: int, num_pairs: int) -> int:
@@ -130,7 +132,7 @@ def route_sort(topk_ids, num_experts, expert_offsets, sorted_pair_ids, pair_pos,
 
 def gate_up_silu(x, gate: ExpertTables, up: ExpertTables, act, expert_offsets, sorted_pair_ids,
                  active_experts, active_count, n_inter, k_hidden, cap, num_tokens, topk,
-                 path=0, split=0, stream=None) -> None:
+                 path=0, split=0, tiles=0, depth=0, stream=None) -> None:
     if x.dtype not in (torch.bfloat16, torch.uint16, torch.int16):
         raise TypeError("x: expected bf16 (or its uint16 bits)")
     _check("nvfp4_moe_gate_up_silu_ex", _lib.nvfp4_moe_gate_up_silu_ex(
@@ -139,17 +141,20 @@ def gate_up_silu(x, gate: ExpertTables, up: ExpertTables, act, expert_offsets, s
         _ptr(sorted_pair_ids, torch.int32, "sorted_pair_ids"),
         _ptr(active_experts, torch.int32, "active_experts"),
         _ptr(active_count, torch.int32, "active_count"),
-        n_inter, k_hidden, cap, num_tokens, topk, _opts(path, split), _stream(stream)))
+        n_inter, k_hidden, cap, num_tokens, topk, _opts(path, split, tiles, depth),
+        _stream(stream)))
 
 
 def down(act, down_w: ExpertTables, y, expert_offsets, active_experts, active_count,
-         n_hidden, k_inter, cap, num_pairs, path=0, split=0, stream=None) -> None:
+         n_hidden, k_inter, cap, num_tokens, topk, path=0, split=0, tiles=0, depth=0,
+         stream=None) -> None:
     _check("nvfp4_moe_down_ex", _lib.nvfp4_moe_down_ex(
         _ptr(act, torch.float32, "act"), down_w, _ptr(y, torch.float32, "y"),
         _ptr(expert_offsets, torch.int32, "expert_offsets"),
         _ptr(active_experts, torch.int32, "active_experts"),
         _ptr(active_count, torch.int32, "active_count"),
-        n_hidden, k_inter, cap, num_pairs, _opts(path, split), _stream(stream)))
+        n_hidden, k_inter, cap, num_tokens, topk, _opts(path, split, tiles, depth),
+        _stream(stream)))
 
 
 def blend(y, topk_weights, pair_pos, out_f32, out_bf16=None, stream=None) -> None:

@@ -37,17 +37,39 @@ bool tables_ok(const nvfp4_expert_tables& t) {
 
 int status_of(cudaError_t err) { return err == cudaSuccess ? NVFP4_MOE_OK : NVFP4_MOE_ECUDA; }
 
-// Decode-path K split from the average rows per active expert: one row per
-// expert needs the four warps of a CTA on one output tile to have enough loads
-// in flight; many rows per expert give each warp its own tile.
-int auto_split(uint64_t pairs, uint32_t cap) {
-  const uint64_t rows_per_expert = cap ? pairs / cap : pairs;
-  if (rows_per_expert < 2) return 4;
-  if (rows_per_expert < 8) return 2;
-  return 1;
-}
+constexpr int kSmsEstimate = 148;
 
-bool split_ok(int s) { return s == 1 || s == 2 || s == 4; }
+// Decode-path launch shape from the host-known sizes.  Rows per expert are at
+// most min(tokens, pairs) (a token picks an expert once), so small batches hold
+// every row of an expert in one pass; larger ones size the pass for twice the
+// mean.  With one tile, the CTA's warps split K when the grid would otherwise
+// leave SMs short of weight streams.
+DecodePlan plan_decode(int mode, uint64_t tokens, uint64_t pairs, uint32_t num_experts,
+                       uint32_t cap, uint32_t n, const nvfp4_moe_launch_opts* o) {
+  DecodePlan p{};
+  const uint64_t max_rows = tokens < pairs ? tokens : pairs;
+  if (max_rows <= 32) {
+    p.tiles = (int)((max_rows + 7) / 8);
+  } else {
+    const uint64_t mean = (pairs + num_experts - 1) / num_experts;
+    p.tiles = (int)((2 * mean + 7) / 8);
+  }
+  if (p.tiles < 1) p.tiles = 1;
+  if (p.tiles == 3 || p.tiles > 4) p.tiles = 4;
+  if (mode == kModeDown && p.tiles > 2) p.tiles = 2;
+  if (o && o->tiles) p.tiles = o->tiles;
+  const uint64_t active = cap < pairs ? cap : pairs;
+  auto ctas = [&](int split) {
+    const uint64_t rpc = (uint64_t)grouped_rows_per_cta(mode, split);
+    return ((n + rpc - 1) / rpc) * active;
+  };
+  p.split = 1;
+  if (p.tiles == 1 && ctas(1) < 2 * kSmsEstimate) p.split = ctas(2) < 2 * kSmsEstimate ? 4 : 2;
+  if (o && o->split) p.split = o->split;
+  p.depth = (p.split == 1 && p.tiles <= 2) ? 3 : 2;
+  if (o && o->depth) p.depth = o->depth;
+  return p;
+}
 
 }  // namespace
 }  // namespace nvm
@@ -105,10 +127,9 @@ int nvfp4_moe_gate_up_silu_ex(const uint16_t* x, nvfp4_expert_tables gate,
       active_experts == nullptr || active_count == nullptr || !tables_ok(gate) || !tables_ok(up))
     return NVFP4_MOE_EINVAL;
   const int path = opts ? opts->path : 0;
-  int split = opts ? opts->split : 0;
   if (path != 0 && path != 1) return NVFP4_MOE_EINVAL;
-  if (split == 0) split = auto_split(pairs, cap);
-  if (!split_ok(split)) return NVFP4_MOE_EINVAL;
+  const DecodePlan plan = plan_decode(kModeGateUp, num_tokens, pairs, cap, cap, n_inter, opts);
+  if (!grouped_plan_supported(kModeGateUp, plan)) return NVFP4_MOE_EINVAL;
   GroupedArgs a{};
   a.src = x;
   a.packed0 = gate.packed_ptrs;
@@ -125,7 +146,7 @@ int nvfp4_moe_gate_up_silu_ex(const uint16_t* x, nvfp4_expert_tables gate,
   a.N = n_inter;
   a.K = k_hidden;
   a.topk = topk;
-  return status_of(launch_grouped(kModeGateUp, split, 4 / split, a, cap, stream));
+  return status_of(launch_grouped(kModeGateUp, plan, a, cap, stream));
 }
 
 int nvfp4_moe_gate_up_silu(const uint16_t* x, nvfp4_expert_tables gate,
@@ -142,20 +163,21 @@ int nvfp4_moe_gate_up_silu(const uint16_t* x, nvfp4_expert_tables gate,
 int nvfp4_moe_down_ex(const float* act, nvfp4_expert_tables down, float* y,
                       const int32_t* expert_offsets, const int32_t* active_experts,
                       const int32_t* active_count, uint32_t n_hidden, uint32_t k_inter,
-                      uint32_t cap, uint32_t num_pairs, const nvfp4_moe_launch_opts* opts,
-                      cudaStream_t stream) {
-  if (n_hidden == 0 || n_hidden % 128 != 0 || k_inter == 0 || k_inter % 256 != 0 || cap > 65535)
+                      uint32_t cap, uint32_t num_tokens, uint32_t topk,
+                      const nvfp4_moe_launch_opts* opts, cudaStream_t stream) {
+  if (n_hidden == 0 || n_hidden % 128 != 0 || k_inter == 0 || k_inter % 256 != 0 || topk == 0 ||
+      cap > 65535)
     return NVFP4_MOE_ESHAPE;
-  if (num_pairs > kMaxPairs) return NVFP4_MOE_ESHAPE;
-  if (num_pairs == 0 || cap == 0) return NVFP4_MOE_OK;
+  const uint64_t pairs = (uint64_t)num_tokens * topk;
+  if (pairs > kMaxPairs) return NVFP4_MOE_ESHAPE;
+  if (pairs == 0 || cap == 0) return NVFP4_MOE_OK;
   if (act == nullptr || y == nullptr || expert_offsets == nullptr || active_experts == nullptr ||
       active_count == nullptr || !tables_ok(down))
     return NVFP4_MOE_EINVAL;
   const int path = opts ? opts->path : 0;
-  int split = opts ? opts->split : 0;
   if (path != 0 && path != 1) return NVFP4_MOE_EINVAL;
-  if (split == 0) split = auto_split(num_pairs, cap);
-  if (!split_ok(split)) return NVFP4_MOE_EINVAL;
+  const DecodePlan plan = plan_decode(kModeDown, num_tokens, pairs, cap, cap, n_hidden, opts);
+  if (!grouped_plan_supported(kModeDown, plan)) return NVFP4_MOE_EINVAL;
   GroupedArgs a{};
   a.src = act;
   a.packed0 = down.packed_ptrs;
@@ -167,16 +189,16 @@ int nvfp4_moe_down_ex(const float* act, nvfp4_expert_tables down, float* y,
   a.active_count = active_count;
   a.N = n_hidden;
   a.K = k_inter;
-  a.topk = 1;
-  return status_of(launch_grouped(kModeDown, split, 4 / split, a, cap, stream));
+  a.topk = topk;
+  return status_of(launch_grouped(kModeDown, plan, a, cap, stream));
 }
 
 int nvfp4_moe_down(const float* act, nvfp4_expert_tables down, float* y,
                    const int32_t* expert_offsets, const int32_t* active_experts,
                    const int32_t* active_count, uint32_t n_hidden, uint32_t k_inter,
-                   uint32_t cap, uint32_t num_pairs, cudaStream_t stream) {
+                   uint32_t cap, uint32_t num_tokens, uint32_t topk, cudaStream_t stream) {
   return nvfp4_moe_down_ex(act, down, y, expert_offsets, active_experts, active_count, n_hidden,
-                           k_inter, cap, num_pairs, nullptr, stream);
+                           k_inter, cap, num_tokens, topk, nullptr, stream);
 }
 
 int nvfp4_moe_blend(const float* y, const float* topk_weights, const int32_t* pair_pos,

@@ -27,10 +27,19 @@ struct GroupedArgs {
   uint32_t N, K, topk;
 };
 
-// Decode-shaped path (register-fed tensor-core MMA), grouped_mma.cu.
-// split in {1, 2, 4} with tiles = 4 / split.
-cudaError_t launch_grouped(int mode, int split, int tiles, const GroupedArgs& a, uint32_t cap,
+// Launch shape of the decode path (grouped_mma.cu):
+//   split  warps of a CTA that split K over the same rows (1, 2 or 4)
+//   tiles  8-token tiles held per pass over an expert (1, 2 or 4)
+//   depth  weight chunks in flight per warp (2 or 3)
+struct DecodePlan {
+  int split;
+  int tiles;
+  int depth;
+};
+
+cudaError_t launch_grouped(int mode, const DecodePlan& plan, const GroupedArgs& a, uint32_t cap,
                            cudaStream_t stream);
+bool grouped_plan_supported(int mode, const DecodePlan& plan);
 int grouped_rows_per_cta(int mode, int split);
 
 cudaError_t launch_route_sort(const int32_t* topk_ids, uint32_t num_pairs, uint32_t num_experts,

@@ -90,8 +90,11 @@ class NVFP4MoE:
 
     def forward(self, x: torch.Tensor, topk_ids: torch.Tensor, topk_weights: torch.Tensor,
                 bufs: Optional[MoEBuffers] = None, path: int = 0, split: int = 0,
-                stream=None) -> MoEBuffers:
-        """Run the four steps on ``stream``; results land in ``bufs`` (returned)."""
+                tiles: int = 0, depth: int = 0, stream=None) -> MoEBuffers:
+        """Run the four steps on ``stream``; results land in ``bufs`` (returned).
+
+        path / split / tiles / depth are the launch options of the two
+        projections (0 = chosen from the shape); see nvfp4_moe_launch_opts."""
         m = x.shape[0]
         if bufs is None:
             bufs = self.buffers(m)
@@ -103,9 +106,9 @@ class NVFP4MoE:
         B.gate_up_silu(x, self.gate.tables, self.up.tables, bufs.act, bufs.expert_offsets,
                        bufs.sorted_pair_ids, bufs.active_experts, bufs.active_count,
                        self.inter, self.hidden, cap, m, self.topk, path=path, split=split,
-                       stream=stream)
+                       tiles=tiles, depth=depth, stream=stream)
         B.down(bufs.act, self.down.tables, bufs.y, bufs.expert_offsets, bufs.active_experts,
-               bufs.active_count, self.hidden, self.inter, cap, p, path=path, split=split,
-               stream=stream)
+               bufs.active_count, self.hidden, self.inter, cap, m, self.topk, path=path,
+               split=split, tiles=tiles, depth=depth, stream=stream)
         B.blend(bufs.y, topk_weights, bufs.pair_pos, bufs.out, bufs.out_bf16, stream=stream)
         return bufs

@@ -64,7 +64,7 @@ def test_host_validation_rejects_bad_shapes_without_a_gpu(lib):
     # gate_up: no tokens is a no-op
     assert L.nvfp4_moe_gate_up_silu(None, t, t, None, None, None, None, None, 64, 256, 1, 0, 1, None) == 0
     # down: N not a multiple of 128
-    assert L.nvfp4_moe_down(None, t, None, None, None, None, 64, 256, 1, 1, None) == 2
+    assert L.nvfp4_moe_down(None, t, None, None, None, None, 64, 256, 1, 1, 1, None) == 2
     # blend: hidden % 4
     assert L.nvfp4_moe_blend(None, None, None, None, None, 1, 1, 6, None) == 2
     assert L.nvfp4_moe_blend(None, None, None, None, None, 0, 1, 8, None) == 0
@@ -72,13 +72,16 @@ def test_host_validation_rejects_bad_shapes_without_a_gpu(lib):
     assert L.nvfp4_moe_transpose_u8(None, None, 4, 4, None) == 1
     assert L.nvfp4_moe_transpose_u8(ctypes.c_void_p(4096), ctypes.c_void_p(4100), 4, 4, None) == 1
     # launch options: bad path / split
-    bad = B.LaunchOpts(7, 0)
+    bad = B.LaunchOpts(7, 0, 0, 0)
     ok_t = B.ExpertTables(8, 8, 8)
     p8 = ctypes.c_void_p(8)
     assert L.nvfp4_moe_gate_up_silu_ex(p8, ok_t, ok_t, p8, p8, p8, p8, p8, 64, 256, 1, 1, 1,
                                        ctypes.byref(bad), None) == 1
-    bad = B.LaunchOpts(1, 3)
-    assert L.nvfp4_moe_down_ex(p8, ok_t, p8, p8, p8, p8, 128, 256, 1, 1, ctypes.byref(bad), None) == 1
+    for opts in ((1, 8, 0, 0), (1, 3, 0, 0), (1, 0, 3, 0), (1, 0, 0, 5), (1, 1, 4, 0), (1, 4, 2, 2)):
+        # split 8 or 3, tiles 3, depth 5, down with 4 tiles, split with 2 tiles
+        bad = B.LaunchOpts(*opts)
+        assert L.nvfp4_moe_down_ex(p8, ok_t, p8, p8, p8, p8, 128, 256, 1, 1, 1,
+                                   ctypes.byref(bad), None) == 1, opts
 
 
 def test_active_cap_and_status_strings(lib):

@@ -42,7 +42,7 @@ def _fns(prob):
     return [lambda e, m=m: prob.expert_weight(m, e, cache=True) for m in (MATRIX_GATE, MATRIX_UP, MATRIX_DOWN)]
 
 
-def _gpu_forward(prob, path=0, split=0, layer=None):
+def _gpu_forward(prob, layer=None, **opts):
     from workloads.device import upload_inputs, upload_layer
     layer = layer or upload_layer(prob)
     x, ids, w = upload_inputs(prob)
@@ -50,7 +50,7 @@ def _gpu_forward(prob, path=0, split=0, layer=None):
     bufs.act.fill_(float("nan"))
     bufs.y.fill_(float("nan"))
     bufs.out.fill_(float("nan"))
-    layer.forward(x, ids, w, bufs, path=path, split=split)
+    layer.forward(x, ids, w, bufs, **opts)
     torch.cuda.synchronize()
     return layer, bufs
 
@@ -184,13 +184,41 @@ SMALL = {
 }
 
 
-@pytest.mark.parametrize("split", [0, 1, 2, 4])
+# Decode launch shapes: (split, tiles, depth); zeros pick from the shape.
+PLANS = [(0, 0, 0), (4, 1, 2), (2, 1, 2), (1, 1, 2), (1, 1, 3), (1, 2, 2), (1, 2, 3)]
+
+
+@pytest.mark.parametrize("plan", PLANS, ids=lambda p: "s%d-t%d-d%d" % p)
 @pytest.mark.parametrize("name", list(SMALL))
-def test_forward_small(name, split):
+def test_forward_small(name, plan):
     _need_gpu()
     prob = make_problem(SMALL[name])
-    _, bufs = _gpu_forward(prob, path=1 if split else 0, split=split)
+    split, tiles, depth = plan
+    _, bufs = _gpu_forward(prob, path=1 if any(plan) else 0, split=split, tiles=tiles, depth=depth)
     _check_full(prob, bufs)
+
+
+def test_gate_up_four_tiles():
+    """Gate+up holding 32 rows per pass (the 17..32-token shape)."""
+    _need_gpu()
+    prob = make_problem(SMALL["hot"])
+    import nvfp4_weight_quantized_moe_b200 as nvm
+    from workloads.device import upload_inputs, upload_layer
+    cfg = prob.cfg
+    layer = upload_layer(prob)
+    x, ids, w = upload_inputs(prob)
+    bufs = layer.buffers(cfg.tokens)
+    nvm.route_sort(ids, cfg.experts, bufs.expert_offsets, bufs.sorted_pair_ids, bufs.pair_pos,
+                   bufs.active_experts, bufs.active_count, bufs.status)
+    cap = nvm.active_cap(cfg.experts, cfg.pairs)
+    nvm.gate_up_silu(x, layer.gate.tables, layer.up.tables, bufs.act, bufs.expert_offsets,
+                     bufs.sorted_pair_ids, bufs.active_experts, bufs.active_count, cfg.inter,
+                     cfg.hidden, cap, cfg.tokens, cfg.topk, path=1, split=1, tiles=4, depth=2)
+    torch.cuda.synchronize()
+    ref = orc.moe_forward(prob.x_bf16, prob.topk_ids, prob.topk_weights, cfg.experts, *_fns(prob),
+                          hidden=cfg.hidden, inter=cfg.inter)
+    kept = int(ref["sort"].expert_offsets[-1])
+    _close(bufs.act.cpu().numpy()[:kept], ref["act"][:kept], "act")
 
 
 def test_null_experts_write_zero_rows():
