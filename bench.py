@@ -43,9 +43,14 @@ FALLBACK_BF16_TFLOPS = 1590.0
 DEFAULT_STEPS = {"tiny": 20000, "decode_m1": 20000, "decode_m32": 5000, "decode_m256": 500,
                  "prefill_m8192": 200}
 
-# DRAM bytes of one launch of the dominant kernel, from an ncu capture of the
-# same kernel build (None until captured, and reset when the kernel changes).
-NCU_TRAFFIC_BYTES = {}
+# DRAM bytes (read + write) of one launch of the dominant kernel (gate+up
+# SiLU) from an ncu capture of the same kernel build and launch shape; see the
+# grouped_mma_*_ncu_full summaries.  Absent for workloads not captured, and
+# cleared whenever that kernel changes.
+NCU_TRAFFIC_BYTES = {
+    "decode_m1": 28355840,      # 28.36 MB read, 0 written (routed gate+up bytes: 28.31 MB)
+    "decode_m32": 316248320,    # 311.60 MB read, 4.64 MB written
+}
 
 
 def parse_args(argv=None):

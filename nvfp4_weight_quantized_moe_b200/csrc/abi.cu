@@ -48,11 +48,12 @@ DecodePlan plan_decode(int mode, uint64_t tokens, uint64_t pairs, uint32_t num_e
                        uint32_t cap, uint32_t n, const nvfp4_moe_launch_opts* o) {
   DecodePlan p{};
   const uint64_t max_rows = tokens < pairs ? tokens : pairs;
-  if (max_rows <= 32) {
+  const uint64_t mean = (pairs + num_experts - 1) / num_experts;
+  if (max_rows <= 16) {
     p.tiles = (int)((max_rows + 7) / 8);
   } else {
-    const uint64_t mean = (pairs + num_experts - 1) / num_experts;
     p.tiles = (int)((2 * mean + 7) / 8);
+    if (p.tiles < 2) p.tiles = 2;
   }
   if (p.tiles < 1) p.tiles = 1;
   if (p.tiles == 3 || p.tiles > 4) p.tiles = 4;
@@ -64,9 +65,9 @@ DecodePlan plan_decode(int mode, uint64_t tokens, uint64_t pairs, uint32_t num_e
     return ((n + rpc - 1) / rpc) * active;
   };
   p.split = 1;
-  if (p.tiles == 1 && ctas(1) < 2 * kSmsEstimate) p.split = ctas(2) < 2 * kSmsEstimate ? 4 : 2;
+  if (p.tiles == 1 && ctas(1) < 2 * kSmsEstimate) p.split = ctas(2) < kSmsEstimate ? 4 : 2;
   if (o && o->split) p.split = o->split;
-  p.depth = (p.split == 1 && p.tiles <= 2) ? 3 : 2;
+  p.depth = 2;
   if (o && o->depth) p.depth = o->depth;
   return p;
 }
