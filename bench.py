@@ -48,8 +48,8 @@ DEFAULT_STEPS = {"tiny": 20000, "decode_m1": 20000, "decode_m32": 5000, "decode_
 # grouped_mma_*_ncu_full summaries.  Absent for workloads not captured, and
 # cleared whenever that kernel changes.
 NCU_TRAFFIC_BYTES = {
-    "decode_m1": 28355840,      # 28.36 MB read, 0 written (routed gate+up bytes: 28.31 MB)
-    "decode_m32": 316248320,    # 311.60 MB read, 4.64 MB written
+    ("decode_m1", "mma.sync"): 28355840,     # 28.36 MB read, 0 written (routed gate+up: 28.31 MB)
+    ("decode_m32", "mma.sync"): 316248320,   # 311.60 MB read, 4.64 MB written
 }
 
 
@@ -66,6 +66,8 @@ def parse_args(argv=None):
     ap.add_argument("--split", type=int, default=0)
     ap.add_argument("--tiles", type=int, default=0)
     ap.add_argument("--depth", type=int, default=0)
+    ap.add_argument("--no-workspace", action="store_true",
+                    help="use the calls without workspace (decode path only)")
     ap.add_argument("--replicas", type=int, default=0,
                     help="weight replicas to rotate over (0: enough to exceed 4 x L2)")
     return ap.parse_args(argv)
@@ -216,10 +218,13 @@ def run_ours(args, rank, world, local):
     base = upload_layer(prob, dev)
     x, ids, w = upload_inputs(prob, dev)
     bufs = base.buffers(cfg.tokens)
+    ws = None if args.no_workspace else base.workspace(cfg.tokens)
     # Active experts of this batch (identical for every replica: same routing).
     with torch.cuda.stream(stream):
-        base.forward(x, ids, w, bufs, **_opts(args))
+        base.forward(x, ids, w, bufs, workspace=ws, **_opts(args))
     stream.synchronize()
+    if nvm.device_error() != 0:
+        raise RuntimeError("device error word set by the forward")
     active = int(bufs.active_count.item())
     per_expert = base.gate.nbytes_per_expert
     routed_bytes = 3 * active * per_expert
@@ -233,7 +238,7 @@ def run_ours(args, rank, world, local):
     layers = _replicate(base, replicas - 1)
 
     def step(lay):
-        lay.forward(x, ids, w, bufs, **_opts(args))
+        lay.forward(x, ids, w, bufs, workspace=ws, **_opts(args))
 
     # Graphs: one of R steps (one per replica) plus single-step graphs for remainders.
     with torch.cuda.stream(stream):
@@ -285,14 +290,21 @@ def run_ours(args, rank, world, local):
     routed_gbs = world * routed_bytes / (ms_per_step * 1e-3) / 1e9
 
     # Dominant kernel, timed alone: gate+up SiLU, one launch per replica.
-    prefill = _uses_prefill(args, cfg)
+    tc = ws is not None and args.path != 1
+    prefill = tc and _uses_prefill(args, cfg)
     gu_graph = torch.cuda.CUDAGraph()
     cap = nvm.active_cap(cfg.experts, cfg.pairs)
 
     def gate_up(lay):
-        nvm.gate_up_silu(x, lay.gate.tables, lay.up.tables, bufs.act, bufs.expert_offsets,
-                         bufs.sorted_pair_ids, bufs.active_experts, bufs.active_count,
-                         cfg.inter, cfg.hidden, cap, cfg.tokens, cfg.topk, **_opts(args))
+        if ws is None:
+            nvm.gate_up_silu(x, lay.gate.tables, lay.up.tables, bufs.act, bufs.expert_offsets,
+                             bufs.sorted_pair_ids, bufs.active_experts, bufs.active_count,
+                             cfg.inter, cfg.hidden, cap, cfg.tokens, cfg.topk, **_opts(args))
+        else:
+            nvm.gate_up_silu_ws(x, lay.gate.tables, lay.up.tables, bufs.act, bufs.expert_offsets,
+                                bufs.sorted_pair_ids, bufs.active_experts, bufs.active_count,
+                                cfg.inter, cfg.hidden, cap, cfg.tokens, cfg.topk, cfg.experts, ws,
+                                **_opts(args))
     with torch.cuda.graph(gu_graph, stream=stream):
         for lay in layers:
             gate_up(lay)
@@ -309,19 +321,21 @@ def run_ours(args, rank, world, local):
     gu_flops = 2.0 * 2 * cfg.pairs * cfg.hidden * cfg.inter
     if prefill:
         achieved = gu_flops / (gu_ms * 1e-3) / 1e12
-        roofline = {"kernel": "nvfp4_moe_gate_up_silu (tcgen05 prefill path)", "bound": "tensor",
+        roofline = {"kernel": "nvfp4_moe_gate_up_silu_ws (tcgen05, 128-row passes)", "bound": "tensor",
                     "achieved": achieved, "peak": tflops, "unit": "TFLOP/s",
                     "frac": achieved / tflops, "peak_source": f"{peak_kind} bf16 burst",
                     "algorithmic_flops_per_launch": gu_flops, "launch_ms": gu_ms,
-                    "traffic": NCU_TRAFFIC_BYTES.get(cfg.name)}
+                    "traffic": NCU_TRAFFIC_BYTES.get((cfg.name, "tcgen05"))}
     else:
         achieved = gu_bytes / (gu_ms * 1e-3) / 1e9
-        roofline = {"kernel": "nvfp4_moe_gate_up_silu (decode path)", "bound": "hbm",
+        roofline = {"kernel": "nvfp4_moe_gate_up_silu_ws (tcgen05, 16-row passes)" if tc else
+                    "nvfp4_moe_gate_up_silu (register-fed mma.sync)", "bound": "hbm",
                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                     "peak_source": f"{peak_kind} HBM copy", "algorithmic_bytes_per_launch": gu_bytes,
-                    "launch_ms": gu_ms, "traffic": NCU_TRAFFIC_BYTES.get(cfg.name)}
+                    "launch_ms": gu_ms,
+                    "traffic": NCU_TRAFFIC_BYTES.get((cfg.name, "tcgen05" if tc else "mma.sync"))}
 
-    e2e = None if args.no_e2e else run_e2e(layers, prob, bufs, dev, stream, steps, warmup, args, world)
+    e2e = None if args.no_e2e else run_e2e(layers, prob, bufs, ws, dev, stream, steps, warmup, args, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -334,7 +348,7 @@ def run_ours(args, rank, world, local):
         "config": {"workload": cfg.name, "hidden": cfg.hidden, "inter": cfg.inter,
                    "experts": cfg.experts, "topk": cfg.topk, "tokens": cfg.tokens,
                    "router": cfg.router, "active_experts": active,
-                   "path": "prefill-tcgen05" if prefill else "decode-mma",
+                   "path": ("tcgen05-nt128" if prefill else "tcgen05-nt16") if tc else "mma.sync",
                    "weight_replicas": len(layers),
                    "l2": f"weights rotate over {len(layers)} device replicas; "
                          f"{len(layers)} x {routed_bytes/1e6:.1f} MB routed >= 4 x L2 ({l2/1e6:.0f} MB)"
@@ -345,7 +359,7 @@ def run_ours(args, rank, world, local):
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": 4 * steps,
+        "gpu_launches": (6 if ws is not None else 4) * steps,
         "clocks": clocks,
     }
     if rank == 0:
@@ -360,10 +374,13 @@ def _opts(args):
 
 
 def _uses_prefill(args, cfg):
-    return False
+    """Many rows per expert: the tcgen05 kernel runs 128-row passes and is tensor-bound."""
+    if args.tiles:
+        return args.tiles * 8 > 16
+    return (cfg.pairs + cfg.experts - 1) // cfg.experts > 16
 
 
-def run_e2e(layers, prob, bufs, dev, stream, steps, warmup, args, world):
+def run_e2e(layers, prob, bufs, ws, dev, stream, steps, warmup, args, world):
     """Same metric through the public API from pinned host buffers: per step the
     host->device copy of x / topk_ids / topk_weights, the forward, and the
     device->host copy of the FP32 output, all inside the timed region."""
@@ -382,7 +399,7 @@ def run_e2e(layers, prob, bufs, dev, stream, steps, warmup, args, world):
         dx.copy_(hx, non_blocking=True)
         dids.copy_(hids, non_blocking=True)
         dw.copy_(hw, non_blocking=True)
-        layers[i % len(layers)].forward(dx, dids, dw, bufs, **_opts(args))
+        layers[i % len(layers)].forward(dx, dids, dw, bufs, workspace=ws, **_opts(args))
         hout.copy_(bufs.out[: cfg.tokens], non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -404,7 +421,7 @@ def run_e2e(layers, prob, bufs, dev, stream, steps, warmup, args, world):
     d2h = hout.numel() * 4
     return {"value": world * cfg.tokens * n / (ms * 1e-3), "unit": "tokens/s", "steps": n,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "api": "NVFP4MoE.forward (four C-ABI calls, eager launches)"}
+            "api": "NVFP4MoE.forward (C-ABI calls, eager launches)"}
 
 
 # --------------------------------------------------------------------------- #

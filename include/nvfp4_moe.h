@@ -49,6 +49,7 @@
 #ifndef NVFP4_MOE_H_
 #define NVFP4_MOE_H_
 
+#include <stddef.h>
 #include <stdint.h>
 #include <cuda_runtime.h>
 
@@ -181,6 +182,51 @@ NVFP4_MOE_API int nvfp4_moe_down_ex(const float* act, nvfp4_expert_tables down, 
                       const int32_t* active_count, uint32_t n_hidden, uint32_t k_inter,
                       uint32_t cap, uint32_t num_tokens, uint32_t topk,
                       const nvfp4_moe_launch_opts* opts, cudaStream_t stream);
+
+/*
+ * Bytes of caller-owned device workspace the tcgen05 path needs for one call
+ * of nvfp4_moe_gate_up_silu_ws / nvfp4_moe_down_ws with these sizes (the two
+ * steps use disjoint parts of it, so one buffer serves both).
+ */
+NVFP4_MOE_API size_t nvfp4_moe_workspace_bytes(uint32_t num_tokens, uint32_t topk, uint32_t hidden,
+                                               uint32_t inter);
+
+/*
+ * Steps 2 and 3 with a workspace, which opens the tcgen05 path (path 2, or
+ * path 0 when the output width is a multiple of 128 for gate+up, 256 for
+ * down; path 2 with another width returns NVFP4_MOE_ESHAPE): activations are packed
+ * once into f16 (x per token; act per sorted row as an f16 hi + lo pair, each
+ * row scaled by a power of two into the f16 range), and the projection kernel
+ * decodes each weight row straight into tensor memory for tcgen05.mma with
+ * FP32 accumulators in tensor memory.  Arguments as for the calls without
+ * _ws, plus num_experts (the length of the expert tables; it bounds the
+ * offsets read) and `workspace`: device memory of at least
+ * nvfp4_moe_workspace_bytes(num_tokens, topk, hidden, inter) bytes, 256-byte
+ * aligned, owned by the caller, overwritten by the call.  For the tcgen05
+ * path opts->tiles selects the token rows per pass (2 -> 16, 16 -> 128; 0 =
+ * from the shape).  Results equal the other path's within FP32 rounding.
+ * Calls on one stream may share the workspace; concurrent calls may not.
+ */
+NVFP4_MOE_API int nvfp4_moe_gate_up_silu_ws(
+    const uint16_t* x, nvfp4_expert_tables gate, nvfp4_expert_tables up, float* act,
+    const int32_t* expert_offsets, const int32_t* sorted_pair_ids, const int32_t* active_experts,
+    const int32_t* active_count, uint32_t n_inter, uint32_t k_hidden, uint32_t cap,
+    uint32_t num_tokens, uint32_t topk, uint32_t num_experts, const nvfp4_moe_launch_opts* opts,
+    void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+NVFP4_MOE_API int nvfp4_moe_down_ws(
+    const float* act, nvfp4_expert_tables down, float* y, const int32_t* expert_offsets,
+    const int32_t* active_experts, const int32_t* active_count, uint32_t n_hidden, uint32_t k_inter,
+    uint32_t cap, uint32_t num_tokens, uint32_t topk, uint32_t num_experts,
+    const nvfp4_moe_launch_opts* opts, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Device error word of the library: 0, or 1 if a tcgen05-path kernel gave up
+ * waiting on one of its barriers (its outputs are then not valid).  Kernels
+ * never trap; they set this word and exit.  Reading it synchronises the
+ * device; clear != 0 resets it to 0.  Returns -1 if the read itself failed.
+ */
+NVFP4_MOE_API int nvfp4_moe_device_error(int clear);
 
 /*
  * Step 4: router-weighted blend back into token order

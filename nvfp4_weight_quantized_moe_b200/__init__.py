@@ -15,10 +15,14 @@ from ._binding import (  # noqa: F401
     NVFP4MoEError,
     active_cap,
     blend,
+    device_error,
     down,
+    down_ws,
     exported_symbols,
     gate_up_silu,
+    gate_up_silu_ws,
     route_sort,
     transpose_u8,
+    workspace_bytes,
 )
 from .layer import MoEBuffers, NVFP4MoE, NVFP4Projection  # noqa: F401

@@ -61,6 +61,15 @@ _sig = {
     "nvfp4_moe_blend": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_u32, c_u32,
                                 c_u32, c_void_p]),
     "nvfp4_moe_transpose_u8": (c_int, [c_void_p, c_void_p, c_u32, c_u32, c_void_p]),
+    "nvfp4_moe_gate_up_silu_ws": (c_int, [c_void_p, ExpertTables, ExpertTables, c_void_p, c_void_p,
+                                          c_void_p, c_void_p, c_void_p, c_u32, c_u32, c_u32, c_u32,
+                                          c_u32, c_u32, ctypes.POINTER(LaunchOpts), c_void_p,
+                                          ctypes.c_size_t, c_void_p]),
+    "nvfp4_moe_down_ws": (c_int, [c_void_p, ExpertTables, c_void_p, c_void_p, c_void_p, c_void_p,
+                                  c_u32, c_u32, c_u32, c_u32, c_u32, c_u32, ctypes.POINTER(LaunchOpts),
+                                  c_void_p, ctypes.c_size_t, c_void_p]),
+    "nvfp4_moe_workspace_bytes": (ctypes.c_size_t, [c_u32, c_u32, c_u32, c_u32]),
+    "nvfp4_moe_device_error": (c_int, [c_int]),
     "nvfp4_moe_active_cap": (c_u32, [c_u32, c_u32]),
     "nvfp4_moe_status_string": (ctypes.c_char_p, [c_int]),
 }
@@ -172,3 +181,47 @@ def transpose_u8(src, dst, stream=None) -> None:
         raise ValueError("dst must be [cols, rows]")
     _check("nvfp4_moe_transpose_u8", _lib.nvfp4_moe_transpose_u8(
         _ptr(src, torch.uint8, "src"), _ptr(dst, torch.uint8, "dst"), rows, cols, _stream(stream)))
+
+
+def workspace_bytes(num_tokens, topk, hidden, inter) -> int:
+    return int(_lib.nvfp4_moe_workspace_bytes(num_tokens, topk, hidden, inter))
+
+
+def device_error(clear: bool = True) -> int:
+    """The library's device error word (synchronises the device)."""
+    return int(_lib.nvfp4_moe_device_error(1 if clear else 0))
+
+
+def _ws(workspace):
+    if workspace.dtype != torch.uint8 or workspace.device.type != "cuda" or not workspace.is_contiguous():
+        raise ValueError("workspace: contiguous uint8 CUDA tensor")
+    return workspace.data_ptr(), workspace.numel()
+
+
+def gate_up_silu_ws(x, gate: ExpertTables, up: ExpertTables, act, expert_offsets, sorted_pair_ids,
+                    active_experts, active_count, n_inter, k_hidden, cap, num_tokens, topk,
+                    num_experts, workspace, path=0, split=0, tiles=0, depth=0, stream=None) -> None:
+    if x.dtype not in (torch.bfloat16, torch.uint16, torch.int16):
+        raise TypeError("x: expected bf16 (or its uint16 bits)")
+    wp, wn = _ws(workspace)
+    _check("nvfp4_moe_gate_up_silu_ws", _lib.nvfp4_moe_gate_up_silu_ws(
+        _ptr(x, None, "x"), gate, up, _ptr(act, torch.float32, "act"),
+        _ptr(expert_offsets, torch.int32, "expert_offsets"),
+        _ptr(sorted_pair_ids, torch.int32, "sorted_pair_ids"),
+        _ptr(active_experts, torch.int32, "active_experts"),
+        _ptr(active_count, torch.int32, "active_count"),
+        n_inter, k_hidden, cap, num_tokens, topk, num_experts,
+        _opts(path, split, tiles, depth), wp, wn, _stream(stream)))
+
+
+def down_ws(act, down_w: ExpertTables, y, expert_offsets, active_experts, active_count, n_hidden,
+            k_inter, cap, num_tokens, topk, num_experts, workspace, path=0, split=0, tiles=0, depth=0,
+            stream=None) -> None:
+    wp, wn = _ws(workspace)
+    _check("nvfp4_moe_down_ws", _lib.nvfp4_moe_down_ws(
+        _ptr(act, torch.float32, "act"), down_w, _ptr(y, torch.float32, "y"),
+        _ptr(expert_offsets, torch.int32, "expert_offsets"),
+        _ptr(active_experts, torch.int32, "active_experts"),
+        _ptr(active_count, torch.int32, "active_count"),
+        n_hidden, k_inter, cap, num_tokens, topk, num_experts,
+        _opts(path, split, tiles, depth), wp, wn, _stream(stream)))

@@ -147,6 +147,7 @@ int nvfp4_moe_gate_up_silu_ex(const uint16_t* x, nvfp4_expert_tables gate,
   a.N = n_inter;
   a.K = k_hidden;
   a.topk = topk;
+  a.num_experts = 0;
   return status_of(launch_grouped(kModeGateUp, plan, a, cap, stream));
 }
 
@@ -200,6 +201,125 @@ int nvfp4_moe_down(const float* act, nvfp4_expert_tables down, float* y,
                    uint32_t cap, uint32_t num_tokens, uint32_t topk, cudaStream_t stream) {
   return nvfp4_moe_down_ex(act, down, y, expert_offsets, active_experts, active_count, n_hidden,
                            k_inter, cap, num_tokens, topk, nullptr, stream);
+}
+
+size_t nvfp4_moe_workspace_bytes(uint32_t num_tokens, uint32_t topk, uint32_t hidden,
+                                 uint32_t inter) {
+  return tc_workspace_bytes(num_tokens, topk, hidden, inter);
+}
+
+int nvfp4_moe_device_error(int clear) {
+  int v = 0;
+  if (read_device_error(&v, clear != 0) != cudaSuccess) return -1;
+  return v;
+}
+
+namespace {
+
+// Token rows per pass of the tcgen05 kernel: 16 for decode-shaped batches (a
+// few rows per expert), 128 when experts carry many rows.
+int plan_tc_rows(uint64_t tokens, uint64_t pairs, uint32_t num_experts, const nvfp4_moe_launch_opts* o) {
+  if (o && o->tiles) return o->tiles * 8;
+  const uint64_t mean = (pairs + num_experts - 1) / num_experts;
+  return mean <= 16 ? 16 : 128;
+}
+
+// The tcgen05 kernel covers 128 (gate+up) or 256 (down) output rows per CTA.
+bool use_tc(uint32_t n, uint32_t rows_per_cta, const nvfp4_moe_launch_opts* o) {
+  const int path = o ? o->path : 0;
+  if (path == 1) return false;
+  return n % rows_per_cta == 0;
+}
+
+}  // namespace
+
+int nvfp4_moe_gate_up_silu_ws(const uint16_t* x, nvfp4_expert_tables gate, nvfp4_expert_tables up,
+                              float* act, const int32_t* expert_offsets,
+                              const int32_t* sorted_pair_ids, const int32_t* active_experts,
+                              const int32_t* active_count, uint32_t n_inter, uint32_t k_hidden,
+                              uint32_t cap, uint32_t num_tokens, uint32_t topk,
+                              uint32_t num_experts, const nvfp4_moe_launch_opts* opts,
+                              void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const int path = opts ? opts->path : 0;
+  if (path < 0 || path > 2) return NVFP4_MOE_EINVAL;
+  if (!use_tc(n_inter, 128, opts)) {
+    if (path == 2) return NVFP4_MOE_ESHAPE;
+    return nvfp4_moe_gate_up_silu_ex(x, gate, up, act, expert_offsets, sorted_pair_ids,
+                                     active_experts, active_count, n_inter, k_hidden, cap,
+                                     num_tokens, topk, opts, stream);
+  }
+  if (k_hidden == 0 || k_hidden % 256 != 0 || topk == 0 || cap > 65535 || num_experts == 0 ||
+      num_experts > kMaxExperts)
+    return NVFP4_MOE_ESHAPE;
+  const uint64_t pairs = (uint64_t)num_tokens * topk;
+  if (pairs > kMaxPairs) return NVFP4_MOE_ESHAPE;
+  if (pairs == 0 || cap == 0) return NVFP4_MOE_OK;
+  if (x == nullptr || act == nullptr || expert_offsets == nullptr || sorted_pair_ids == nullptr ||
+      active_experts == nullptr || active_count == nullptr || !tables_ok(gate) || !tables_ok(up) ||
+      workspace == nullptr)
+    return NVFP4_MOE_EINVAL;
+  if (workspace_bytes < tc_workspace_bytes(num_tokens, topk, k_hidden, n_inter)) return NVFP4_MOE_EINVAL;
+  const int nt = plan_tc_rows(num_tokens, pairs, num_experts, opts);
+  if (nt != 16 && nt != 128) return NVFP4_MOE_EINVAL;
+  GroupedArgs a{};
+  a.src = x;
+  a.packed0 = gate.packed_ptrs;
+  a.scale0 = gate.scale_ptrs;
+  a.s2_0 = gate.scale2;
+  a.packed1 = up.packed_ptrs;
+  a.scale1 = up.scale_ptrs;
+  a.s2_1 = up.scale2;
+  a.out = act;
+  a.offsets = expert_offsets;
+  a.sorted_pair_ids = sorted_pair_ids;
+  a.active_experts = active_experts;
+  a.active_count = active_count;
+  a.N = n_inter;
+  a.K = k_hidden;
+  a.topk = topk;
+  a.num_experts = num_experts;
+  return status_of(launch_tc(kModeGateUp, nt, a, workspace, num_tokens, k_hidden, n_inter, cap, stream));
+}
+
+int nvfp4_moe_down_ws(const float* act, nvfp4_expert_tables down, float* y,
+                      const int32_t* expert_offsets, const int32_t* active_experts,
+                      const int32_t* active_count, uint32_t n_hidden, uint32_t k_inter,
+                      uint32_t cap, uint32_t num_tokens, uint32_t topk, uint32_t num_experts,
+                      const nvfp4_moe_launch_opts* opts, void* workspace, size_t workspace_bytes,
+                      cudaStream_t stream) {
+  const int path = opts ? opts->path : 0;
+  if (path < 0 || path > 2) return NVFP4_MOE_EINVAL;
+  if (!use_tc(n_hidden, 256, opts)) {
+    if (path == 2) return NVFP4_MOE_ESHAPE;
+    return nvfp4_moe_down_ex(act, down, y, expert_offsets, active_experts, active_count, n_hidden,
+                             k_inter, cap, num_tokens, topk, opts, stream);
+  }
+  if (k_inter == 0 || k_inter % 256 != 0 || topk == 0 || cap > 65535 || num_experts == 0 ||
+      num_experts > kMaxExperts)
+    return NVFP4_MOE_ESHAPE;
+  const uint64_t pairs = (uint64_t)num_tokens * topk;
+  if (pairs > kMaxPairs) return NVFP4_MOE_ESHAPE;
+  if (pairs == 0 || cap == 0) return NVFP4_MOE_OK;
+  if (act == nullptr || y == nullptr || expert_offsets == nullptr || active_experts == nullptr ||
+      active_count == nullptr || !tables_ok(down) || workspace == nullptr)
+    return NVFP4_MOE_EINVAL;
+  if (workspace_bytes < tc_workspace_bytes(num_tokens, topk, n_hidden, k_inter)) return NVFP4_MOE_EINVAL;
+  const int nt = plan_tc_rows(num_tokens, pairs, num_experts, opts);
+  if (nt != 16 && nt != 128) return NVFP4_MOE_EINVAL;
+  GroupedArgs a{};
+  a.src = act;
+  a.packed0 = down.packed_ptrs;
+  a.scale0 = down.scale_ptrs;
+  a.s2_0 = down.scale2;
+  a.out = y;
+  a.offsets = expert_offsets;
+  a.active_experts = active_experts;
+  a.active_count = active_count;
+  a.N = n_hidden;
+  a.K = k_inter;
+  a.topk = topk;
+  a.num_experts = num_experts;
+  return status_of(launch_tc(kModeDown, nt, a, workspace, num_tokens, n_hidden, k_inter, cap, stream));
 }
 
 int nvfp4_moe_blend(const float* y, const float* topk_weights, const int32_t* pair_pos,

@@ -25,6 +25,7 @@ struct GroupedArgs {
   const int32_t* active_experts;
   const int32_t* active_count;
   uint32_t N, K, topk;
+  uint32_t num_experts;
 };
 
 // Launch shape of the decode path (grouped_mma.cu):
@@ -41,6 +42,13 @@ cudaError_t launch_grouped(int mode, const DecodePlan& plan, const GroupedArgs& 
                            cudaStream_t stream);
 bool grouped_plan_supported(int mode, const DecodePlan& plan);
 int grouped_rows_per_cta(int mode, int split);
+
+// tcgen05 path (grouped_tc.cu): activation packing into `workspace`, then the
+// projection kernel with NT token rows per pass (16 or 128).
+size_t tc_workspace_bytes(uint64_t tokens, uint64_t topk, uint64_t hidden, uint64_t inter);
+cudaError_t launch_tc(int mode, int nt, const GroupedArgs& a, void* workspace, uint32_t tokens,
+                      uint32_t hidden, uint32_t inter, uint32_t cap, cudaStream_t stream);
+cudaError_t read_device_error(int* value, bool clear);
 
 cudaError_t launch_route_sort(const int32_t* topk_ids, uint32_t num_pairs, uint32_t num_experts,
                               int32_t* expert_offsets, int32_t* sorted_pair_ids, int32_t* pair_pos,

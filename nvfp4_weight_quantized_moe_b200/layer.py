@@ -88,13 +88,21 @@ class NVFP4MoE:
         return MoEBuffers(num_tokens, self.topk, self.num_experts, self.hidden, self.inter,
                           self.gate.packed.device, out_bf16)
 
+    def workspace(self, num_tokens: int) -> torch.Tensor:
+        """Device workspace of the tcgen05 path for batches of up to num_tokens."""
+        n = B.workspace_bytes(num_tokens, self.topk, self.hidden, self.inter)
+        return torch.empty(max(n, 1), dtype=torch.uint8, device=self.gate.packed.device)
+
     def forward(self, x: torch.Tensor, topk_ids: torch.Tensor, topk_weights: torch.Tensor,
                 bufs: Optional[MoEBuffers] = None, path: int = 0, split: int = 0,
-                tiles: int = 0, depth: int = 0, stream=None) -> MoEBuffers:
+                tiles: int = 0, depth: int = 0, workspace: Optional[torch.Tensor] = None,
+                stream=None) -> MoEBuffers:
         """Run the four steps on ``stream``; results land in ``bufs`` (returned).
 
         path / split / tiles / depth are the launch options of the two
-        projections (0 = chosen from the shape); see nvfp4_moe_launch_opts."""
+        projections (0 = chosen from the shape); see nvfp4_moe_launch_opts.
+        With a ``workspace`` (see :meth:`workspace`) the projections may take
+        the tcgen05 path."""
         m = x.shape[0]
         if bufs is None:
             bufs = self.buffers(m)
@@ -103,12 +111,20 @@ class NVFP4MoE:
         B.route_sort(topk_ids, self.num_experts, bufs.expert_offsets, bufs.sorted_pair_ids,
                      bufs.pair_pos, bufs.active_experts, bufs.active_count, bufs.status,
                      stream=stream)
-        B.gate_up_silu(x, self.gate.tables, self.up.tables, bufs.act, bufs.expert_offsets,
-                       bufs.sorted_pair_ids, bufs.active_experts, bufs.active_count,
-                       self.inter, self.hidden, cap, m, self.topk, path=path, split=split,
-                       tiles=tiles, depth=depth, stream=stream)
-        B.down(bufs.act, self.down.tables, bufs.y, bufs.expert_offsets, bufs.active_experts,
-               bufs.active_count, self.hidden, self.inter, cap, m, self.topk, path=path,
-               split=split, tiles=tiles, depth=depth, stream=stream)
+        opts = dict(path=path, split=split, tiles=tiles, depth=depth, stream=stream)
+        if workspace is None:
+            B.gate_up_silu(x, self.gate.tables, self.up.tables, bufs.act, bufs.expert_offsets,
+                           bufs.sorted_pair_ids, bufs.active_experts, bufs.active_count,
+                           self.inter, self.hidden, cap, m, self.topk, **opts)
+            B.down(bufs.act, self.down.tables, bufs.y, bufs.expert_offsets, bufs.active_experts,
+                   bufs.active_count, self.hidden, self.inter, cap, m, self.topk, **opts)
+        else:
+            B.gate_up_silu_ws(x, self.gate.tables, self.up.tables, bufs.act, bufs.expert_offsets,
+                              bufs.sorted_pair_ids, bufs.active_experts, bufs.active_count,
+                              self.inter, self.hidden, cap, m, self.topk, self.num_experts,
+                              workspace, **opts)
+            B.down_ws(bufs.act, self.down.tables, bufs.y, bufs.expert_offsets,
+                      bufs.active_experts, bufs.active_count, self.hidden, self.inter, cap, m,
+                      self.topk, self.num_experts, workspace, **opts)
         B.blend(bufs.y, topk_weights, bufs.pair_pos, bufs.out, bufs.out_bf16, stream=stream)
         return bufs

@@ -42,16 +42,21 @@ def _fns(prob):
     return [lambda e, m=m: prob.expert_weight(m, e, cache=True) for m in (MATRIX_GATE, MATRIX_UP, MATRIX_DOWN)]
 
 
-def _gpu_forward(prob, layer=None, **opts):
+def _gpu_forward(prob, layer=None, ws=False, **opts):
     from workloads.device import upload_inputs, upload_layer
+    import nvfp4_weight_quantized_moe_b200 as nvm
     layer = layer or upload_layer(prob)
     x, ids, w = upload_inputs(prob)
     bufs = layer.buffers(prob.cfg.tokens, out_bf16=True)
     bufs.act.fill_(float("nan"))
     bufs.y.fill_(float("nan"))
     bufs.out.fill_(float("nan"))
-    layer.forward(x, ids, w, bufs, **opts)
+    workspace = layer.workspace(prob.cfg.tokens) if ws else None
+    if workspace is not None:
+        workspace.fill_(0xFF)  # NaN f16 patterns: anything read before it is written shows up
+    layer.forward(x, ids, w, bufs, workspace=workspace, **opts)
     torch.cuda.synchronize()
+    assert nvm.device_error() == 0
     return layer, bufs
 
 
@@ -221,6 +226,23 @@ def test_gate_up_four_tiles():
     _close(bufs.act.cpu().numpy()[:kept], ref["act"][:kept], "act")
 
 
+# tcgen05 path: token rows per pass 16 (tiles=2) or 128 (tiles=16); 0 = from the shape.
+@pytest.mark.parametrize("tiles", [0, 2, 16])
+@pytest.mark.parametrize("name", list(SMALL))
+def test_forward_small_tcgen05(name, tiles):
+    _need_gpu()
+    prob = make_problem(SMALL[name])
+    _, bufs = _gpu_forward(prob, ws=True, path=2, tiles=tiles)
+    _check_full(prob, bufs)
+
+
+def test_null_experts_tcgen05():
+    _need_gpu()
+    prob = make_problem(SMALL["ragged"], null_experts=[1, 3])
+    _, bufs = _gpu_forward(prob, ws=True, path=2)
+    _check_full(prob, bufs)
+
+
 def test_null_experts_write_zero_rows():
     _need_gpu()
     prob = make_problem(SMALL["ragged"], null_experts=[1, 3])
@@ -300,11 +322,12 @@ def test_large_activation_range():
 # The five workloads at full size
 # --------------------------------------------------------------------------- #
 
+@pytest.mark.parametrize("ws", [False, True], ids=["decode-path", "tcgen05"])
 @pytest.mark.parametrize("name", ["decode_m1", "decode_m32"])
-def test_forward_full_decode(name):
+def test_forward_full_decode(name, ws):
     _need_gpu()
     prob = make_problem(name)
-    _, bufs = _gpu_forward(prob)
+    _, bufs = _gpu_forward(prob, ws=ws)
     _check_full(prob, bufs)
 
 
@@ -331,12 +354,13 @@ def _check_sampled(prob, bufs, tokens):
             _close(y[pos], wd @ h, f"y[{pos}]")
 
 
+@pytest.mark.parametrize("ws", [False, True], ids=["decode-path", "tcgen05"])
 @pytest.mark.parametrize("name", ["decode_m256", "prefill_m8192"])
-def test_forward_full_size_sampled(name):
+def test_forward_full_size_sampled(name, ws):
     """Full-size launch, checked on a seeded sample of tokens (tokens are independent)."""
     _need_gpu()
     prob = make_problem(name)
-    _, bufs = _gpu_forward(prob)
+    _, bufs = _gpu_forward(prob, ws=ws)
     mid = int(np.random.default_rng(99).integers(1, prob.cfg.tokens - 1))
     tokens = [0, mid, prob.cfg.tokens - 1]
     _check_sampled(prob, bufs, tokens)
