@@ -290,7 +290,7 @@ def run_ours(args, rank, world, local):
     routed_gbs = world * routed_bytes / (ms_per_step * 1e-3) / 1e9
 
     # Dominant kernel, timed alone: gate+up SiLU, one launch per replica.
-    tc = ws is not None and args.path != 1
+    tc = ws is not None and _tc_path(args, cfg)
     prefill = tc and _uses_prefill(args, cfg)
     gu_graph = torch.cuda.CUDAGraph()
     cap = nvm.active_cap(cfg.experts, cfg.pairs)
@@ -359,7 +359,7 @@ def run_ours(args, rank, world, local):
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": (6 if ws is not None else 4) * steps,
+        "gpu_launches": (6 if tc else 4) * steps,
         "clocks": clocks,
     }
     if rank == 0:
@@ -371,6 +371,15 @@ def run_ours(args, rank, world, local):
 
 def _opts(args):
     return dict(path=args.path, split=args.split, tiles=args.tiles, depth=args.depth)
+
+
+def _tc_path(args, cfg):
+    """Whether the projections take the tcgen05 path (the library's rule for
+    the workspace calls: widths divisible by 128 / 256, and path 2, or path 0
+    with at least 4 routed rows per expert on average)."""
+    if args.path == 1 or cfg.inter % 128 or cfg.hidden % 256:
+        return False
+    return args.path == 2 or cfg.pairs >= 4 * cfg.experts
 
 
 def _uses_prefill(args, cfg):

@@ -225,10 +225,15 @@ int plan_tc_rows(uint64_t tokens, uint64_t pairs, uint32_t num_experts, const nv
 }
 
 // The tcgen05 kernel covers 128 (gate+up) or 256 (down) output rows per CTA.
-bool use_tc(uint32_t n, uint32_t rows_per_cta, const nvfp4_moe_launch_opts* o) {
+// Chosen automatically from 4 routed rows per expert on average: below that
+// the register-fed decode kernel keeps more weight bytes in flight per SM
+// (measured on B200: faster at 0.06 and 2 rows per expert, slower at 8).
+bool use_tc(uint32_t n, uint32_t rows_per_cta, uint64_t pairs, uint32_t num_experts,
+            const nvfp4_moe_launch_opts* o) {
   const int path = o ? o->path : 0;
-  if (path == 1) return false;
-  return n % rows_per_cta == 0;
+  if (path == 1 || n % rows_per_cta != 0) return false;
+  if (path == 2) return true;
+  return pairs >= 4ull * num_experts;
 }
 
 }  // namespace
@@ -242,7 +247,7 @@ int nvfp4_moe_gate_up_silu_ws(const uint16_t* x, nvfp4_expert_tables gate, nvfp4
                               void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   const int path = opts ? opts->path : 0;
   if (path < 0 || path > 2) return NVFP4_MOE_EINVAL;
-  if (!use_tc(n_inter, 128, opts)) {
+  if (!use_tc(n_inter, 128, (uint64_t)num_tokens * topk, num_experts, opts)) {
     if (path == 2) return NVFP4_MOE_ESHAPE;
     return nvfp4_moe_gate_up_silu_ex(x, gate, up, act, expert_offsets, sorted_pair_ids,
                                      active_experts, active_count, n_inter, k_hidden, cap,
@@ -289,7 +294,7 @@ int nvfp4_moe_down_ws(const float* act, nvfp4_expert_tables down, float* y,
                       cudaStream_t stream) {
   const int path = opts ? opts->path : 0;
   if (path < 0 || path > 2) return NVFP4_MOE_EINVAL;
-  if (!use_tc(n_hidden, 256, opts)) {
+  if (!use_tc(n_hidden, 256, (uint64_t)num_tokens * topk, num_experts, opts)) {
     if (path == 2) return NVFP4_MOE_ESHAPE;
     return nvfp4_moe_down_ex(act, down, y, expert_offsets, active_experts, active_count, n_hidden,
                              k_inter, cap, num_tokens, topk, opts, stream);
