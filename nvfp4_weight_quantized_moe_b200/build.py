@@ -1,6 +1,8 @@
 """Build the sm_100a shared library ``libnvfp4moe.so`` in-tree with nvcc.
 
-    python -m nvfp4_weight_quantized_moe_b200.build [--verbose-ptxas]
+    python nvfp4_weight_quantized_moe_b200/build.py [--verbose-ptxas] [--force]
+
+(run by path: importing the package first would load the library being rebuilt)
 
 The library is a plain C ABI (include/nvfp4_moe.h) with the CUDA runtime
 linked statically, so it loads with ctypes next to any PyTorch build.

@@ -21,8 +21,8 @@ def _declared():
 
 @pytest.fixture(scope="module")
 def lib():
-    from nvfp4_weight_quantized_moe_b200 import build
-    path = build.build()
+    import __graft_entry__
+    path = __graft_entry__._build_module().build()
     return ctypes.CDLL(path)
 
 
