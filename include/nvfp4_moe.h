@@ -222,6 +222,32 @@ NVFP4_MOE_API int nvfp4_moe_down_ws(
     const nvfp4_moe_launch_opts* opts, void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Allocation-free gate+up (tcgen05 path).  The pages have no counterpart to
+ * this call; it exists for callers that cannot hand the library a workspace:
+ * code whose device memory is owned by another allocator or a fixed budget,
+ * and code that must not call cudaMalloc, which can block on the whole device
+ * or fail midway.
+ *
+ * Same arguments and result as nvfp4_moe_gate_up_silu_ws with path 2 and no
+ * workspace.  The packed token rows go to a fixed scratch array inside the
+ * library: 8 MiB of device memory on every GPU that loads the library, held
+ * until the process exits.  Requests needing more than that
+ * (num_tokens * k_hidden * 2 bytes plus num_tokens * 4, each rounded up to 256)
+ * return NVFP4_MOE_ESHAPE before anything is launched; so do widths the
+ * tcgen05 path does not take (n_inter % 128, k_hidden % 256).  The call never
+ * allocates memory.  Its first call on a device looks the scratch array's
+ * device address up (cudaGetSymbolAddress) with that device current; make
+ * that first call before any stream capture.  All calls share the one array
+ * and each call leaves its packed rows there: calls whose kernels overlap on
+ * the GPU (different streams, or different host threads) race on it.
+ */
+NVFP4_MOE_API int nvfp4_moe_gate_up_silu_noalloc(
+    const uint16_t* x, nvfp4_expert_tables gate, nvfp4_expert_tables up, float* act,
+    const int32_t* expert_offsets, const int32_t* sorted_pair_ids, const int32_t* active_experts,
+    const int32_t* active_count, uint32_t n_inter, uint32_t k_hidden, uint32_t cap,
+    uint32_t num_tokens, uint32_t topk, uint32_t num_experts, cudaStream_t stream);
+
+/*
  * Device error word of the library: 0, or 1 if a tcgen05-path kernel gave up
  * waiting on one of its barriers (its outputs are then not valid).  Kernels
  * never trap; they set this word and exit.  Reading it synchronises the

@@ -68,6 +68,9 @@ _sig = {
     "nvfp4_moe_down_ws": (c_int, [c_void_p, ExpertTables, c_void_p, c_void_p, c_void_p, c_void_p,
                                   c_u32, c_u32, c_u32, c_u32, c_u32, c_u32, ctypes.POINTER(LaunchOpts),
                                   c_void_p, ctypes.c_size_t, c_void_p]),
+    "nvfp4_moe_gate_up_silu_noalloc": (c_int, [c_void_p, ExpertTables, ExpertTables, c_void_p,
+                                               c_void_p, c_void_p, c_void_p, c_void_p, c_u32,
+                                               c_u32, c_u32, c_u32, c_u32, c_u32, c_void_p]),
     "nvfp4_moe_workspace_bytes": (ctypes.c_size_t, [c_u32, c_u32, c_u32, c_u32]),
     "nvfp4_moe_device_error": (c_int, [c_int]),
     "nvfp4_moe_active_cap": (c_u32, [c_u32, c_u32]),
