@@ -50,6 +50,7 @@ DEFAULT_STEPS = {"tiny": 20000, "decode_m1": 20000, "decode_m32": 5000, "decode_
 NCU_TRAFFIC_BYTES = {
     ("decode_m1", "mma.sync"): 28355840,     # 28.36 MB read, 0 written (routed gate+up: 28.31 MB)
     ("decode_m32", "mma.sync"): 316248320,   # 311.60 MB read, 4.64 MB written
+    ("prefill_m8192", "tcgen05"): 4047628000,  # 3.658 GB read, 0.390 GB written (4 token passes)
 }
 
 
