@@ -20,6 +20,8 @@ __global__ void __launch_bounds__(kBlendThreads)
     blend_kernel(const float* __restrict__ y, const float* __restrict__ w,
                  const int32_t* __restrict__ pair_pos, float* __restrict__ out,
                  uint16_t* __restrict__ out_bf16, int k, int H) {
+  griddep_wait();  // y of the down projection is complete
+  griddep_launch_dependents();
   const int t = blockIdx.y;
   const int col = (blockIdx.x * kBlendThreads + threadIdx.x) * 4;
   if (col >= H) return;
@@ -49,9 +51,8 @@ cudaError_t launch_blend(const float* y, const float* topk_weights, const int32_
                          float* out_f32, uint16_t* out_bf16, uint32_t num_tokens, uint32_t topk,
                          uint32_t hidden, cudaStream_t stream) {
   const dim3 grid((hidden / 4 + kBlendThreads - 1) / kBlendThreads, num_tokens);
-  blend_kernel<<<grid, kBlendThreads, 0, stream>>>(y, topk_weights, pair_pos, out_f32, out_bf16,
-                                                   (int)topk, (int)hidden);
-  return cudaGetLastError();
+  return launch_pdl(blend_kernel, grid, dim3(kBlendThreads), 0, stream, y, topk_weights, pair_pos,
+                    out_f32, out_bf16, (int)topk, (int)hidden);
 }
 
 }  // namespace nvm

@@ -111,4 +111,33 @@ NVM_DEV float warp_max(float v) {
 
 NVM_DEV float silu_f32(float z) { return z / (1.0f + expf(-z)); }
 
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch and L2 prefetch
+// ---------------------------------------------------------------------------
+// Block until the grids this one depends on have completed and their memory
+// is visible (a no-op for a kernel launched without the programmatic
+// serialization attribute).
+NVM_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the dependent grid start launching (it still waits for this grid's
+// completion before it reads what this grid writes).
+NVM_DEV void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Ask L2 to fetch `bytes` (multiple of 16) starting at a 16-byte aligned global
+// address; nothing is returned to the SM.
+NVM_DEV void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Load that is never served from a stale L1 line (cached in L2 only).
+NVM_DEV int ld_cg_i32(const int32_t* p) {
+  int v;
+  asm volatile("ld.global.cg.s32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+NVM_DEV const void* ld_cg_ptr(const void* const* p) {
+  uint64_t v;
+  asm volatile("ld.global.cg.u64 %0, [%1];" : "=l"(v) : "l"(p));
+  return reinterpret_cast<const void*>(v);
+}
+
 }  // namespace nvm

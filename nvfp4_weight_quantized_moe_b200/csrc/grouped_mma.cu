@@ -112,23 +112,54 @@ __global__ void __launch_bounds__(128) grouped_mma_kernel(GroupedArgs a) {
   const int s = warp % S, q = warp / S;
   const int g = lane >> 2, c = lane & 3;
 
+  // Gate+up reads the route sort's outputs at once, so it waits for the previous
+  // kernel first.  Down starts before gate+up has finished: the route sort's
+  // outputs are complete by the time it launches (gate+up lets it launch only
+  // after its own wait), and the weights are never written, so down looks up
+  // its expert and starts fetching its weights before it waits for act.
+  if (MODE == kModeGateUp) {
+    griddep_wait();
+    griddep_launch_dependents();
+  }
   const int slot = blockIdx.y;
-  if (slot >= *a.active_count) return;
-  const int e = a.active_experts[slot];
-  const int row_lo = a.offsets[e], row_hi = a.offsets[e + 1];
+  const int count = ld_cg_i32(a.active_count);
+  const int e = slot < count ? ld_cg_i32(a.active_experts + slot) : 0;
+  const int row_lo = slot < count ? ld_cg_i32(a.offsets + e) : 0;
+  const int row_hi = slot < count ? ld_cg_i32(a.offsets + e + 1) : 0;
   const int N = (int)a.N, K = (int)a.K;
   const int n_cta = blockIdx.x * C::ROWS_PER_CTA;
   const int nw = n_cta + q * C::ROWS_PER_WARP;
   const bool warp_on = nw < N;
 
-  const uint8_t* P0 = static_cast<const uint8_t*>(a.packed0[e]);
-  const uint8_t* S0 = static_cast<const uint8_t*>(a.scale0[e]);
+  const uint8_t* P0 = nullptr;
+  const uint8_t* S0 = nullptr;
+  if (slot < count) {
+    P0 = static_cast<const uint8_t*>(ld_cg_ptr(a.packed0 + e));
+    S0 = static_cast<const uint8_t*>(ld_cg_ptr(a.scale0 + e));
+  }
   const uint8_t* P1 = P0;
   const uint8_t* S1 = S0;
-  if (MODE == kModeGateUp) {
-    P1 = static_cast<const uint8_t*>(a.packed1[e]);
-    S1 = static_cast<const uint8_t*>(a.scale1[e]);
+  if (MODE == kModeGateUp && slot < count) {
+    P1 = static_cast<const uint8_t*>(ld_cg_ptr(a.packed1 + e));
+    S1 = static_cast<const uint8_t*>(ld_cg_ptr(a.scale1 + e));
   }
+  // A CTA whose weight slice is small asks L2 for all of it at once, so the
+  // whole slice streams from HBM while the first chunks are being waited on.
+  if (slot < count && P0 != nullptr && P1 != nullptr && tid < 4) {
+    const uint32_t rows = (uint32_t)min(C::ROWS_PER_CTA, N - n_cta);
+    const uint32_t nib = rows * (uint32_t)(K >> 1), scl = rows * (uint32_t)(K >> 4);
+    if ((MODE == kModeGateUp ? 2u : 1u) * (nib + scl) <= 160u * 1024u) {
+      const uint8_t* base = (tid & 2) ? ((tid & 1) ? S1 : S0) : ((tid & 1) ? P1 : P0);
+      const uint32_t bytes = (tid & 2) ? scl : nib;
+      const size_t row_bytes = (tid & 2) ? (size_t)(K >> 4) : (size_t)(K >> 1);
+      if (MODE == kModeGateUp || (tid & 1) == 0) prefetch_l2_bulk(base + (size_t)n_cta * row_bytes, bytes);
+    }
+  }
+  if (MODE == kModeDown) {
+    griddep_wait();  // act is complete
+    griddep_launch_dependents();
+  }
+  if (slot >= count) return;
   if (P0 == nullptr || P1 == nullptr) {
     // NULL expert: its rows are zero.
     const int rows = row_hi - row_lo;
@@ -442,8 +473,7 @@ cudaError_t launch_grouped_impl(const GroupedArgs& a, uint32_t cap, cudaStream_t
   cudaError_t err = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::SMEM);
   if (err != cudaSuccess) return err;
   const dim3 grid((a.N + C::ROWS_PER_CTA - 1) / C::ROWS_PER_CTA, cap);
-  kern<<<grid, C::THREADS, C::SMEM, stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, dim3(C::THREADS), C::SMEM, stream, a);
 }
 
 cudaError_t launch_grouped(int mode, const DecodePlan& p, const GroupedArgs& a, uint32_t cap,

@@ -113,6 +113,8 @@ NVM_DEV uint32_t pack_f16x2(float a, float b) {
 // One warp per token row: xs[t] = f16(x[t] * 2^-e_t), xexp[t] = 2^e_t.
 __global__ void __launch_bounds__(256) pack_x_kernel(const uint16_t* __restrict__ x, int M, int K,
                                                      uint16_t* __restrict__ xs, float* __restrict__ xexp) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (row >= M) return;
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)row * K);
@@ -147,6 +149,8 @@ __global__ void __launch_bounds__(256) pack_act_kernel(const float* __restrict__
                                                        const int32_t* __restrict__ kept_rows,
                                                        uint16_t* __restrict__ hi, uint16_t* __restrict__ lo,
                                                        float* __restrict__ aexp) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (row >= P || row >= *kept_rows) return;
   const float4* src = reinterpret_cast<const float4*>(act + (size_t)row * K);
@@ -210,6 +214,8 @@ __global__ void __launch_bounds__(kThreads, NT <= 16 ? 2 : 1) grouped_tc_kernel(
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_ABORT);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  griddep_wait();
+  griddep_launch_dependents();
   const int slot_idx = blockIdx.y;
   if (slot_idx >= *a.active_count) return;
   const int e = a.active_experts[slot_idx];
@@ -454,8 +460,7 @@ cudaError_t launch_tc_impl(const TcArgs& a, uint32_t cap, cudaStream_t stream) {
   cudaError_t err = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::SMEM);
   if (err != cudaSuccess) return err;
   const dim3 grid(a.N / C::ROWS_PER_CTA, cap);
-  kern<<<grid, kThreads, C::SMEM, stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, dim3(kThreads), C::SMEM, stream, a);
 }
 
 size_t tc_workspace_bytes(uint64_t tokens, uint64_t topk, uint64_t hidden, uint64_t inter) {
@@ -511,9 +516,9 @@ cudaError_t launch_tc(int mode, int nt, const GroupedArgs& g, void* workspace, u
   a.topk = g.topk;
   cudaError_t err;
   if (mode == kModeGateUp) {
-    pack_x_kernel<<<(tokens + 7) / 8, 256, 0, stream>>>(static_cast<const uint16_t*>(g.src), (int)tokens,
-                                                        (int)g.K, w.xs, w.xexp);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    err = launch_pdl(pack_x_kernel, dim3((tokens + 7) / 8), dim3(256), 0, stream,
+                     static_cast<const uint16_t*>(g.src), (int)tokens, (int)g.K, w.xs, w.xexp);
+    if (err != cudaSuccess) return err;
     a.b0 = w.xs;
     a.b1 = w.xs;
     a.bexp = w.xexp;
@@ -521,10 +526,10 @@ cudaError_t launch_tc(int mode, int nt, const GroupedArgs& g, void* workspace, u
     if (nt == 128) return launch_tc_impl<kModeGateUp, 128>(a, cap, stream);
   } else {
     // Rows past offsets[E] (dropped pairs) are not packed: offsets[E] bounds the grid's work.
-    pack_act_kernel<<<(pairs + 7) / 8, 256, 0, stream>>>(static_cast<const float*>(g.src), (int)pairs,
-                                                         (int)g.K, g.offsets + g.num_experts, w.act_hi,
-                                                         w.act_lo, w.aexp);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    err = launch_pdl(pack_act_kernel, dim3((pairs + 7) / 8), dim3(256), 0, stream,
+                     static_cast<const float*>(g.src), (int)pairs, (int)g.K, g.offsets + g.num_experts,
+                     w.act_hi, w.act_lo, w.aexp);
+    if (err != cudaSuccess) return err;
     a.b0 = w.act_hi;
     a.b1 = w.act_lo;
     a.bexp = w.aexp;

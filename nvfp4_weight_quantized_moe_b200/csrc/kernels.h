@@ -65,4 +65,23 @@ cudaError_t launch_transpose_u8(const uint8_t* src, uint8_t* dst, uint32_t rows,
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device).
 cudaError_t ensure_dynamic_smem(const void* kernel, int bytes);
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel on the stream is still running; every kernel of this
+// library calls griddep_wait() before it touches data an earlier kernel writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 }  // namespace nvm

@@ -68,6 +68,8 @@ __global__ void __launch_bounds__(kSortThreads)
   __shared__ int bad;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  griddep_wait();  // the previous kernel on the stream (e.g. the last blend) is done
+  griddep_launch_dependents();
   for (int i = tid; i < E; i += kSortThreads) cnt[i] = 0;
   if (tid == 0) bad = 0;
   __syncthreads();
@@ -135,10 +137,9 @@ cudaError_t launch_route_sort(const int32_t* topk_ids, uint32_t num_pairs, uint3
   const int smem = (int)num_experts * (2 * 4 + 32 * 2);
   cudaError_t err = ensure_dynamic_smem(reinterpret_cast<const void*>(route_sort_kernel), smem);
   if (err != cudaSuccess) return err;
-  route_sort_kernel<<<1, kSortThreads, smem, stream>>>(topk_ids, (int)num_pairs, (int)num_experts,
-                                                       expert_offsets, sorted_pair_ids, pair_pos,
-                                                       active_experts, active_count, status);
-  return cudaGetLastError();
+  return launch_pdl(route_sort_kernel, dim3(1), dim3(kSortThreads), smem, stream, topk_ids,
+                    (int)num_pairs, (int)num_experts, expert_offsets, sorted_pair_ids, pair_pos,
+                    active_experts, active_count, status);
 }
 
 }  // namespace nvm
