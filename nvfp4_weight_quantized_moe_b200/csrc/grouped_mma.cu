@@ -121,9 +121,12 @@ __global__ void __launch_bounds__(128) grouped_mma_kernel(GroupedArgs a) {
     griddep_wait();
     griddep_launch_dependents();
   }
+  // The active count and this slot's expert id are read together (the list is
+  // padded with -1 past the count), then the expert's offsets and pointers.
   const int slot = blockIdx.y;
   const int count = ld_cg_i32(a.active_count);
-  const int e = slot < count ? ld_cg_i32(a.active_experts + slot) : 0;
+  const int e_raw = ld_cg_i32(a.active_experts + slot);
+  const int e = (slot < count && e_raw >= 0) ? e_raw : 0;
   const int row_lo = slot < count ? ld_cg_i32(a.offsets + e) : 0;
   const int row_hi = slot < count ? ld_cg_i32(a.offsets + e + 1) : 0;
   const int N = (int)a.N, K = (int)a.K;
@@ -211,6 +214,14 @@ __global__ void __launch_bounds__(128) grouped_mma_kernel(GroupedArgs a) {
   for (int g0 = row_lo; g0 < row_hi; g0 += C::GROUP) {
     const int nrows = min(C::GROUP, row_hi - g0);
     const int ntiles = (nrows + 7) >> 3;
+    // Split-K CTAs (short K slices) put their first DEPTH weight chunks in
+    // flight before the token rows are looked up; full-K CTAs do it after, which
+    // keeps those registers free during the look-up.
+    if (S > 1 && warp_on) {
+#pragma unroll
+      for (int d = 0; d < DEPTH; ++d)
+        if (d < my_nch) load_chunk(d, wbuf[d], sbuf[d]);
+    }
     __syncthreads();  // the previous group is done with shared memory
     if (tid < C::GROUP) {
       int src = -1;
@@ -298,10 +309,10 @@ __global__ void __launch_bounds__(128) grouped_mma_kernel(GroupedArgs a) {
       }
     };
 
-    // ---- prologue: raw chunks 0 and 1 in flight, weights 0..DEPTH-1 in flight ----
+    // ---- prologue: raw chunks 0 and 1 and weights 0..DEPTH-1 in flight ----
     copy_raw(0, 0);
     cp_async_commit();
-    if (warp_on) {
+    if (S == 1 && warp_on) {
 #pragma unroll
       for (int d = 0; d < DEPTH; ++d)
         if (d < my_nch) load_chunk(d, wbuf[d], sbuf[d]);
