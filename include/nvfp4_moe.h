@@ -196,14 +196,17 @@ NVFP4_MOE_API size_t nvfp4_moe_workspace_bytes(uint32_t num_tokens, uint32_t top
  * path 0 when the output width is a multiple of 128 for gate+up, 256 for
  * down, and there are at least 4 routed rows per expert on average; path 2
  * with another width returns NVFP4_MOE_ESHAPE): activations are packed
- * once into f16 (x per token; act per sorted row as an f16 hi + lo pair, each
- * row scaled by a power of two into the f16 range), and the projection kernel
- * decodes each weight row straight into tensor memory for tcgen05.mma with
- * FP32 accumulators in tensor memory.  Arguments as for the calls without
+ * once into f16 rows by sorted position (x gathered from its token; act as an
+ * f16 hi + lo pair; each row scaled by a power of two into the f16 range),
+ * per-expert TMA tensor maps of the weights are built on the device from the
+ * tables, and the projection kernel loads weight and activation tiles with
+ * TMA, decodes the weights into tensor memory and runs tcgen05.mma with FP32
+ * accumulators in tensor memory.  Arguments as for the calls without
  * _ws, plus num_experts (the length of the expert tables; it bounds the
  * offsets read) and `workspace`: device memory of at least
  * nvfp4_moe_workspace_bytes(num_tokens, topk, hidden, inter) bytes, 256-byte
- * aligned, owned by the caller, overwritten by the call.  For the tcgen05
+ * aligned (NVFP4_MOE_EINVAL otherwise), owned by the caller, overwritten by
+ * the call.  For the tcgen05
  * path opts->tiles selects the token rows per pass (2 -> 16, 16 -> 128; 0 =
  * from the shape).  Results equal the other path's within FP32 rounding.
  * Calls on one stream may share the workspace; concurrent calls may not.
@@ -231,9 +234,9 @@ NVFP4_MOE_API int nvfp4_moe_down_ws(
  * Same arguments and result as nvfp4_moe_gate_up_silu_ws with path 2 and no
  * workspace.  The packed token rows go to a fixed scratch array inside the
  * library: 8 MiB of device memory on every GPU that loads the library, held
- * until the process exits.  Requests needing more than that
- * (num_tokens * k_hidden * 2 bytes plus num_tokens * 4, each rounded up to 256)
- * return NVFP4_MOE_ESHAPE before anything is launched; so do widths the
+ * until the process exits.  Requests needing more than that (P * k_hidden * 2
+ * bytes plus P * 4, each rounded up to 256, plus 512 KiB of tensor maps,
+ * P = num_tokens * topk) return NVFP4_MOE_ESHAPE before anything is launched; so do widths the
  * tcgen05 path does not take (n_inter % 128, k_hidden % 256).  The call never
  * allocates memory.  Its first call on a device looks the scratch array's
  * device address up (cudaGetSymbolAddress) with that device current; make

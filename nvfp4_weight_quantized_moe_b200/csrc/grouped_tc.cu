@@ -7,31 +7,45 @@
 // rows are sorted positions).
 //
 // Design.  A CTA owns 128 weight rows of one expert (for gate+up: 128 gate rows
-// and the same 128 up rows) and a group of up to NT of the expert's token rows.
-//   * Producer warps 0..7: one weight row per thread.  Each thread streams its
-//     row's packed nibbles and block scales with 16-byte loads, DEPTH stages of
-//     64 k ahead in registers, decodes them exactly to f16 (hardware
-//     E2M1 -> f16x2 and E4M3 -> f16x2 conversions, one f16 multiply), and
-//     writes them to its own TMEM lane with tcgen05.st: TMEM is the MMA's A
-//     operand, so decoded weights never pass through shared memory.  The same
-//     threads gather the group's activation rows (f16, prepared once per call
-//     by the pack kernels below) into a K-major shared-memory ring with
-//     cp.async.
-//   * Warp 8: one thread issues tcgen05.mma.kind::f16 (A = 128 x 16 from TMEM,
-//     B = NT x 16 from shared memory, D = FP32 accumulators in TMEM) and
-//     tcgen05.commit to the ring's "empty" mbarriers.
-//   * Epilogue (warps 0..7): tcgen05.ld of the accumulators; weight_scale_2 and
-//     the activation row's power-of-two scale applied in FP32; SiLU(gate)*up in
-//     FP32 for gate+up; coalesced FP32 stores by sorted position.
-// Every mbarrier wait is bounded: on timeout the kernel sets the device error
-// word, skips its remaining work and still frees its TMEM.
+// and the same 128 up rows; for down: 256 rows as two halves) and walks the
+// expert's sorted token rows in groups of NT.  Every operand moves by TMA:
+//   * Warp 9 (one thread) loads weight tiles: per 256 k, for each of the two
+//     128-row matrices, 128 rows x 128 bytes of packed nibbles (128-byte
+//     swizzle) and 128 rows x 16 scale bytes, into a ring of WS slots.  The
+//     tensor maps of each expert's matrices are built on the device from the
+//     pointer tables (build_weight_maps_kernel).
+//   * Warp 10 (one thread) loads token tiles: per 64 k, NT rows x 128 bytes of
+//     f16 activations (128-byte swizzle, the canonical K-major layout of the
+//     MMA's B operand), into a ring of SB slots.
+//   * Warps 0..7 decode: thread (warp w, lane l) owns weight row
+//     32 (w % 4) + l of matrix w / 4.  Per 64 k it reads its row's 32 nibble
+//     bytes and 4 scale bytes from shared memory (conflict-free: the swizzle
+//     spreads eight consecutive rows over all banks), converts them exactly
+//     to f16 (hardware E2M1 -> f16x2 and E4M3 -> f16x2 conversions, one f16
+//     multiply) and writes them to its own TMEM lane with tcgen05.st: TMEM is
+//     the MMA's A operand, in a ring of SA stages.
+//   * Warp 8 (one thread) issues tcgen05.mma.kind::f16 (A = 128 x 16 from
+//     TMEM, B = NT x 16 from shared memory, D = FP32 accumulators in TMEM) and
+//     tcgen05.commit to the rings' "empty" mbarriers.
+//   * Epilogue (warps 0..7, per group): tcgen05.ld of the accumulators;
+//     weight_scale_2 and the activation row's power-of-two scale applied in
+//     FP32; SiLU(gate)*up in FP32 for gate+up; coalesced FP32 stores by sorted
+//     position.  The loaders run ahead into the next group meanwhile.
+// The roles synchronise through mbarriers only.  Every wait is bounded: on
+// timeout the kernel sets the device error word, skips its remaining waits,
+// lets its TMA loads in flight land and still frees its TMEM.
 //
-// Activations.  x is BF16 and act FP32; the MMA takes f16.  pack_x_kernel turns
-// each token row into f16 after scaling it by 2^-e (e from the row's max |x|,
-// so the row fits the f16 range; the epilogue multiplies by 2^e).
-// pack_act_kernel turns each FP32 act row into an f16 hi + lo pair with the same
-// row scaling, and down runs two MMAs (hi, lo) into one accumulator, keeping
-// about 22 bits of the FP32 product.
+// Activations.  x is BF16 and act FP32; the MMA takes f16.  The pack kernels
+// write one f16 row per sorted position (gate+up gathers the token rows, so a
+// group's B rows are contiguous for TMA), each scaled by 2^-e (e from the row's
+// max |value|, so the row fits the f16 range; the epilogue multiplies by 2^e).
+// act becomes an f16 hi + lo pair with the same row scaling, and down runs two
+// MMAs (hi, lo) into one accumulator, keeping about 22 bits of the FP32 value.
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -41,11 +55,25 @@ namespace nvm {
 
 namespace {
 
-constexpr int kStageK = 64;     // k per pipeline stage (4 MMAs of K = 16)
-constexpr int kStages = 3;      // ring depth in shared memory / TMEM
+constexpr int kStageK = 64;                     // k per MMA stage (4 MMAs of K = 16)
+constexpr int kTileK = 256;                     // k per weight tile load (4 stages)
 constexpr int kProdWarps = 8;
-constexpr int kProdThreads = 32 * kProdWarps;
-constexpr int kThreads = kProdThreads + 32;  // + MMA warp
+constexpr int kMmaWarp = kProdWarps;            // warp 8
+constexpr int kWLoadWarp = kProdWarps + 1;      // warp 9
+constexpr int kBLoadWarp = kProdWarps + 2;      // warp 10
+constexpr int kThreads = 32 * (kProdWarps + 3);
+constexpr int kMaxExperts = 1024;
+constexpr int kMapsPerExpert = 4;               // packed0, scale0, packed1, scale1
+constexpr size_t kMapBytes = (size_t)kMaxExperts * kMapsPerExpert * sizeof(CUtensorMap);
+
+// One weight tile: two matrices x (128 rows x 128 nibble bytes + 128 rows x 16
+// scale bytes), every part 1024-byte aligned.
+constexpr int kWNibBytes = 128 * 128;
+constexpr int kWScaleBytes = 128 * 16;
+constexpr int kWSlotBytes = 2 * kWNibBytes + 2 * kWScaleBytes;
+
+constexpr int kSmemPerSM = 228 * 1024;  // shared memory of one SM
+constexpr int kSmemReservedPerCta = 1024;
 
 constexpr uint32_t pow2_at_least(uint32_t v) {
   uint32_t p = 32;
@@ -53,9 +81,9 @@ constexpr uint32_t pow2_at_least(uint32_t v) {
   return p;
 }
 
-// Two A matrices per CTA, 128 rows each, always 64 k (32 TMEM columns) per
-// stage: gate+up = (gate rows, up rows) of the same 128 outputs; down = the
-// two 128-row halves of 256 outputs, which then share every token tile.
+// Rings: weight tiles WS slots (shared memory), token tiles SB slots (shared
+// memory), decoded weights SA stages (TMEM).  D takes 2 NT TMEM columns (gate
+// and up, or the two row halves of down).
 template <int MODE, int NT>
 struct TcCfg {
   static constexpr int PLANES = MODE == kModeGateUp ? 1 : 2;  // down: f16 hi + lo
@@ -64,40 +92,25 @@ struct TcCfg {
   static constexpr int B_SLOT_BYTES = PLANES * B_PLANE_BYTES;
   static constexpr int A_COLS = 64;                             // TMEM columns per stage
   static constexpr int D_COLS = 2 * NT;
-  static constexpr uint32_t TMEM_COLS = pow2_at_least(D_COLS + kStages * A_COLS);
-  static constexpr int DEPTH = 4;                               // weight stages in flight
-  static constexpr int OFF_BAR = kStages * B_SLOT_BYTES;        // full[3], empty[3], done
-  static constexpr int OFF_TMEM = OFF_BAR + 8 * (2 * kStages + 1);
-  static constexpr int OFF_ROWSRC = OFF_TMEM + 16;
-  static constexpr int OFF_ABORT = OFF_ROWSRC + NT * 4;
-  static constexpr int SMEM_USED = OFF_ABORT + 16;
-  // A CTA that takes all 512 TMEM columns also asks for more than half of the
-  // SM's shared memory, so a second one is never resident waiting in alloc.
-  static constexpr int SMEM = TMEM_COLS == 512 && SMEM_USED < 120 * 1024 ? 120 * 1024 : SMEM_USED;
+  static constexpr int SA = NT <= 16 ? 3 : 4;
+  static constexpr int WS = (NT <= 16 || MODE == kModeDown) ? 2 : 3;
+  static constexpr int SB = (MODE == kModeDown && NT > 16) ? 4 : 6;
+  static constexpr uint32_t TMEM_COLS = pow2_at_least(D_COLS + SA * A_COLS);
+  static constexpr int OFF_W = 0;
+  static constexpr int OFF_B = WS * kWSlotBytes;
+  static constexpr int OFF_BAR = OFF_B + SB * B_SLOT_BYTES;
+  // full_w[WS], empty_w[WS], full_b[SB], empty_b[SB], full_a[SA], empty_a[SA], done, d_free
+  static constexpr int NBAR = 2 * WS + 2 * SB + 2 * SA + 2;
+  static constexpr int OFF_TMEM = OFF_BAR + 8 * NBAR;
+  static constexpr int OFF_ABORT = OFF_TMEM + 16;
+  static constexpr int SMEM = OFF_ABORT + 16 + 1024;  // + room to align the base to 1024 B
+  static constexpr int CTAS_PER_SM = kSmemPerSM / (SMEM + kSmemReservedPerCta);
+  static_assert(B_PLANE_BYTES % 1024 == 0 && kWSlotBytes % 1024 == 0, "TMA tiles stay 1024-byte aligned");
   static_assert(TMEM_COLS <= 512, "TMEM budget");
+  // Every CTA that shared memory lets share an SM must find its TMEM columns
+  // free, or a CTA would wait in tcgen05.alloc.
+  static_assert(CTAS_PER_SM >= 1 && CTAS_PER_SM * TMEM_COLS <= 512, "TMEM per SM");
 };
-
-// Shared-memory layout of one B plane of a stage: no-swizzle K-major core
-// matrices (8 rows x 16 B).  Per MMA k-step s (16 k) a [NT/8][2][8][16 B]
-// block: LBO (between the two 8-k halves) = 128 B, SBO (between 8-row groups)
-// = 256 B.  Unit u (16 bytes, u = 0 .. NT*8-1, in shared-memory order) holds
-// k = 16 s + 8 h .. +7 of token row t; consecutive threads take consecutive
-// units, so the 16-byte stores hit consecutive banks.
-template <int NT>
-NVM_DEV void b_unit(int u, int& t, int& piece) {
-  const int s = u / (NT * 2);        // NT*32 bytes per k-step = NT*2 units
-  const int rem = u % (NT * 2);
-  const int grp = rem >> 4, h = (rem >> 3) & 1, r = rem & 7;
-  t = grp * 8 + r;
-  piece = 2 * s + h;
-}
-
-NVM_DEV void cp_async_16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-NVM_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-NVM_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-NVM_DEV void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 NVM_DEV uint32_t pack_f16x2(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
@@ -110,14 +123,18 @@ NVM_DEV uint32_t pack_f16x2(float a, float b) {
 // Activation packing (once per call)
 // ---------------------------------------------------------------------------
 
-// One warp per token row: xs[t] = f16(x[t] * 2^-e_t), xexp[t] = 2^e_t.
-__global__ void __launch_bounds__(256) pack_x_kernel(const uint16_t* __restrict__ x, int M, int K,
-                                                     uint16_t* __restrict__ xs, float* __restrict__ xexp) {
+// One warp per sorted row r < offsets[E]: xs[r] = f16(x[t] * 2^-e), t the
+// row's token, xexp[r] = 2^e.
+__global__ void __launch_bounds__(256)
+    pack_x_sorted_kernel(const uint16_t* __restrict__ x, int P, int K, int topk,
+                         const int32_t* __restrict__ sorted_pair_ids, const int32_t* __restrict__ kept_rows,
+                         uint16_t* __restrict__ xs, float* __restrict__ xexp) {
   griddep_wait();
   griddep_launch_dependents();
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (row >= M) return;
-  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)row * K);
+  if (row >= P || row >= *kept_rows) return;
+  const int t = sorted_pair_ids[row] / topk;
+  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * K);
   float m = 0.0f;
   for (int i = lane; i < K / 8; i += 32) {
     const uint4 v = src[i];
@@ -179,38 +196,80 @@ __global__ void __launch_bounds__(256) pack_act_kernel(const float* __restrict__
 }
 
 // ---------------------------------------------------------------------------
+// Per-expert weight tensor maps (once per call)
+// ---------------------------------------------------------------------------
+
+// Block e, warp j < nmaps: out[4 e + j] = the template map (nibbles for even
+// j, scales for odd j) with its global address replaced by expert e's matrix
+// j / 2 (packed0/scale0, packed1/scale1).  A NULL expert gets no maps: the
+// projection kernel never reads them.  The map is edited in shared memory and
+// copied out with a release fence of the tensor-map proxy; the projection
+// kernel acquires it before its first TMA load.
+__global__ void __launch_bounds__(128)
+    build_weight_maps_kernel(const __grid_constant__ CUtensorMap tmpl_nib,
+                             const __grid_constant__ CUtensorMap tmpl_scale,
+                             const void* const* __restrict__ p0, const void* const* __restrict__ s0,
+                             const void* const* __restrict__ p1, const void* const* __restrict__ s1,
+                             int nmaps, CUtensorMap* __restrict__ out) {
+  __shared__ alignas(128) CUtensorMap tmp[kMapsPerExpert];
+  griddep_wait();  // the kernel that last read `out` has completed
+  griddep_launch_dependents();
+  const int e = blockIdx.x, w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (w >= nmaps) return;
+  if (p0[e] == nullptr || (nmaps == 4 && p1[e] == nullptr)) return;
+  const void* src = w == 0 ? p0[e] : w == 1 ? s0[e] : w == 2 ? p1[e] : s1[e];
+  const CUtensorMap* t = (w & 1) ? &tmpl_scale : &tmpl_nib;
+  if (lane < (int)(sizeof(CUtensorMap) / 16))
+    reinterpret_cast<uint4*>(&tmp[w])[lane] = reinterpret_cast<const uint4*>(t)[lane];
+  __syncwarp();
+  if (lane == 0)
+    asm volatile("tensormap.replace.tile.global_address.shared::cta.b1024.b64 [%0], %1;" ::"r"(smem_u32(&tmp[w])),
+                 "l"(src)
+                 : "memory");
+  __syncwarp();
+  asm volatile(
+      "tensormap.cp_fenceproxy.global.shared::cta.tensormap::generic.release.gpu.sync.aligned [%0], [%1], 128;" ::"l"(
+          out + (size_t)e * kMapsPerExpert + w),
+      "r"(smem_u32(&tmp[w]))
+      : "memory");
+}
+
+// ---------------------------------------------------------------------------
 // The projection kernel
 // ---------------------------------------------------------------------------
 
 struct TcArgs {
-  const uint16_t* b0;      // gate+up: packed x [M, K]; down: act hi plane [P, K]
-  const uint16_t* b1;      // down: act lo plane [P, K]
-  const float* bexp;       // gate+up: per token 2^e; down: per sorted row 2^e
-  const void* const* packed0;
-  const void* const* scale0;
-  const float* s2_0;
+  const float* bexp;          // per sorted row: 2^e of its packed activation row
+  const CUtensorMap* wmaps;   // [E][4] weight tensor maps
+  const void* const* packed0; // NULL-expert test only
   const void* const* packed1;
-  const void* const* scale1;
+  const float* s2_0;
   const float* s2_1;
   float* out;
   const int32_t* offsets;
-  const int32_t* sorted_pair_ids;
   const int32_t* active_experts;
   const int32_t* active_count;
-  uint32_t N, K, topk;
+  uint32_t N, K;
 };
 
 template <int MODE, int NT>
-__global__ void __launch_bounds__(kThreads, NT <= 16 ? 2 : 1) grouped_tc_kernel(TcArgs a) {
+__global__ void __launch_bounds__(kThreads, NT <= 16 ? 2 : 1)
+    grouped_tc_kernel(const TcArgs a, const __grid_constant__ CUtensorMap tm_b0,
+                      const __grid_constant__ CUtensorMap tm_b1) {
   using C = TcCfg<MODE, NT>;
-  constexpr int DEPTH = C::DEPTH;
-  extern __shared__ __align__(1024) uint8_t smem[];
-  const uint32_t s_base = smem_u32(smem);
-  const uint32_t bar_full = s_base + C::OFF_BAR;                 // + 8 * slot
-  const uint32_t bar_empty = bar_full + 8 * kStages;             // + 8 * slot
-  const uint32_t bar_done = bar_empty + 8 * kStages;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t s_base = (raw_base + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (s_base - raw_base);
+  const uint32_t full_w = s_base + C::OFF_BAR;     // TMA weight tile landed (+ 8 * slot)
+  const uint32_t empty_w = full_w + 8 * C::WS;     // decoders done with the tile
+  const uint32_t full_b = empty_w + 8 * C::WS;     // TMA token tile landed
+  const uint32_t empty_b = full_b + 8 * C::SB;     // MMAs done with the tile
+  const uint32_t full_a = empty_b + 8 * C::SB;     // decoded A stage in TMEM
+  const uint32_t empty_a = full_a + 8 * C::SA;     // MMAs done with the A stage
+  const uint32_t bar_done = empty_a + 8 * C::SA;   // a group's accumulators are final
+  const uint32_t bar_dfree = bar_done + 8;         // the epilogue has read them
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
-  int* rowsrc = reinterpret_cast<int*>(smem + C::OFF_ROWSRC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_ABORT);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -222,34 +281,37 @@ __global__ void __launch_bounds__(kThreads, NT <= 16 ? 2 : 1) grouped_tc_kernel(
   const int row_lo = a.offsets[e], row_hi = a.offsets[e + 1];
   const int N = (int)a.N, K = (int)a.K;
   const int n0 = blockIdx.x * C::ROWS_PER_CTA;
-
-  const uint8_t* P0 = static_cast<const uint8_t*>(a.packed0[e]);
-  const uint8_t* S0 = static_cast<const uint8_t*>(a.scale0[e]);
-  const uint8_t* P1 = P0;
-  const uint8_t* S1 = S0;
-  if (MODE == kModeGateUp) {
-    P1 = static_cast<const uint8_t*>(a.packed1[e]);
-    S1 = static_cast<const uint8_t*>(a.scale1[e]);
-  }
-  if (P0 == nullptr || P1 == nullptr) {  // NULL expert: its rows are zero
+  if (a.packed0[e] == nullptr || (MODE == kModeGateUp && a.packed1[e] == nullptr)) {
+    // NULL expert: its rows are zero
     for (int i = tid; i < (row_hi - row_lo) * C::ROWS_PER_CTA; i += kThreads)
       a.out[(size_t)(row_lo + i / C::ROWS_PER_CTA) * N + n0 + i % C::ROWS_PER_CTA] = 0.0f;
     return;
   }
-  const float s2a = a.s2_0[e];
-  const float s2b = MODE == kModeGateUp ? a.s2_1[e] : s2a;
+  const int ngroups = (row_hi - row_lo + NT - 1) / NT;
+  if (ngroups <= 0) return;
+  const int nst = K / kStageK;   // MMA stages per group
+  const int ntile = K / kTileK;  // weight tiles per group
 
   // ---- set-up: barriers and TMEM ----
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar_full + 8 * s, kProdWarps);
-      mbar_init(bar_empty + 8 * s, 1);
+    for (int s = 0; s < C::WS; ++s) {
+      mbar_init(full_w + 8 * s, 1);
+      mbar_init(empty_w + 8 * s, kProdWarps);
+    }
+    for (int s = 0; s < C::SB; ++s) {
+      mbar_init(full_b + 8 * s, 1);
+      mbar_init(empty_b + 8 * s, 1);
+    }
+    for (int s = 0; s < C::SA; ++s) {
+      mbar_init(full_a + 8 * s, kProdWarps);
+      mbar_init(empty_a + 8 * s, 1);
     }
     mbar_init(bar_done, 1);
+    mbar_init(bar_dfree, kProdWarps);
     *abort_flag = 0;
     mbar_init_fence();
   }
-  if (warp == kProdWarps) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -257,174 +319,192 @@ __global__ void __launch_bounds__(kThreads, NT <= 16 ? 2 : 1) grouped_tc_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t tmem_d = tmem;                  // D: two NT-column regions
-  const uint32_t tmem_a = tmem + C::D_COLS;      // A ring after D
+  const uint32_t tmem_d = tmem;              // D: two NT-column regions
+  const uint32_t tmem_a = tmem + C::D_COLS;  // A ring after D
 
-  const int nst = K / kStageK;
-  // Producer identity: one weight row per thread.  Warps 0-3 hold matrix 0
-  // (gate / rows n0 .. n0+127), warps 4-7 matrix 1 (up / rows n0+128 ..).
-  const int prow = (warp & 3) * 32 + lane;   // row within the 128 of its matrix (= TMEM lane)
-  const int pmat = warp >> 2;
-  const uint8_t* wrow = nullptr;
-  const uint8_t* srow = nullptr;
-  if (warp < kProdWarps) {
-    const uint8_t* pb = (MODE == kModeGateUp && pmat == 1) ? P1 : P0;
-    const uint8_t* sb = (MODE == kModeGateUp && pmat == 1) ? S1 : S0;
-    const int wn = n0 + (MODE == kModeDown ? 128 * pmat : 0) + prow;
-    wrow = pb + (size_t)wn * (K >> 1);
-    srow = sb + (size_t)wn * (K >> 4);
-  }
-  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+  // A wait that gives up (and flags the CTA) once any role has timed out.
+  auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+    if (*abort_flag) return false;
+    if (mbar_wait(bar, parity)) return true;
+    *abort_flag = 1;
+    return false;
+  };
 
-  uint32_t it = 0;      // ring iteration, continues across groups
-  uint32_t groups = 0;  // groups done (parity of the done barrier)
-  for (int g0 = row_lo; g0 < row_hi; g0 += NT) {
-    const int nrows = min(NT, row_hi - g0);
-    if (tid < NT) {
-      int src = -1;
-      if (tid < nrows) src = MODE == kModeGateUp ? a.sorted_pair_ids[g0 + tid] / (int)a.topk : g0 + tid;
-      rowsrc[tid] = src;
-    }
-    __syncthreads();
-
-    if (warp < kProdWarps) {
-      // ================= producers =================
-      uint4 wb[DEPTH][2];
-      uint32_t sb[DEPTH];
-      // 32 bytes of nibbles (64 k) and 4 scale bytes of the row per stage.
-      // L1-allocating loads: the two 16-byte halves share one 32-byte sector and
-      // one scale sector serves eight stages.
-      auto load = [&](int st, uint4 (&w)[2], uint32_t& sc) {
-        const uint8_t* p = wrow + (size_t)st * 32;
-        w[0] = __ldg(reinterpret_cast<const uint4*>(p));
-        w[1] = __ldg(reinterpret_cast<const uint4*>(p + 16));
-        sc = __ldg(reinterpret_cast<const uint32_t*>(srow + (size_t)st * 4));
-      };
-#pragma unroll
-      for (int d = 0; d < DEPTH; ++d)
-        if (d < nst) load(d, wb[d], sb[d]);
-
-      // B (this group's token rows, 64 k of stage st) into ring slot `slot`,
-      // after the MMAs that last read the slot have completed.
-      auto issue_b = [&](int st) {
-        const uint32_t slot = (it + st) % kStages;
-        const uint32_t round = (it + st) / kStages;
-        if (round > 0 && !*abort_flag) {
-          if (!mbar_wait(bar_empty + 8 * slot, (round - 1) & 1)) *abort_flag = 1;
-        }
-        const uint32_t bslot = s_base + slot * C::B_SLOT_BYTES;
-        for (int u = tid; u < NT * 8; u += kProdThreads) {
-          int t, piece;
-          b_unit<NT>(u, t, piece);
-          const int off = u * 16;
-          if (t < nrows) {
-            const size_t eoff = (size_t)rowsrc[t] * K + (size_t)st * kStageK + piece * 8;
-            cp_async_16(bslot + off, a.b0 + eoff);
-            if constexpr (MODE == kModeDown) cp_async_16(bslot + C::B_PLANE_BYTES + off, a.b1 + eoff);
-          } else {
-            *reinterpret_cast<uint4*>(smem + slot * C::B_SLOT_BYTES + off) = make_uint4(0, 0, 0, 0);
-            if constexpr (MODE == kModeDown)
-              *reinterpret_cast<uint4*>(smem + slot * C::B_SLOT_BYTES + C::B_PLANE_BYTES + off) =
-                  make_uint4(0, 0, 0, 0);
-          }
-        }
-      };
-      issue_b(0);
-      cp_async_commit();
-
-      for (int base = 0; base < nst; base += DEPTH) {
-#pragma unroll
-        for (int d = 0; d < DEPTH; ++d) {
-          const int st = base + d;
-          if (st < nst) {
-            const uint32_t slot = (it + st) % kStages;
-            // The next stage's B goes in flight before this stage is decoded;
-            // its slot's "empty" wait also frees that slot's A columns.
-            if (st + 1 < nst) issue_b(st + 1);
-            cp_async_commit();
-            // A: decode this thread's row for the stage and write it to TMEM.
-            uint32_t sc0, sc1;  // f16x2 (blk0, blk1), (blk2, blk3)
-            e4m3x4_to_f16x2x2(sb[d], sc0, sc1);
-            uint32_t v[32];
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              const uint32_t wv[4] = {wb[d][q].x, wb[d][q].y, wb[d][q].z, wb[d][q].w};
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const int blk = q * 2 + (i >> 1);  // 8 bytes (16 k) per block
-                const uint32_t scl = blk == 0 ? bcast_lo(sc0) : blk == 1 ? bcast_hi(sc0)
-                                     : blk == 2 ? bcast_lo(sc1) : bcast_hi(sc1);
-                uint32_t dec[4];
-                e2m1x8_to_f16x2x4(wv[i], dec);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) v[q * 16 + i * 4 + j] = hmul2_u32(dec[j], scl);
-              }
-            }
-            tmem_st32(tmem_a + lane_off + slot * C::A_COLS + pmat * 32, v);
-            // Refill this register slot DEPTH stages ahead.
-            if (st + DEPTH < nst) load(st + DEPTH, wb[d], sb[d]);
-            cp_async_wait_one();  // this stage's B has landed (the next one may be in flight)
-            fence_proxy_async_smem();
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_full + 8 * slot);
-          }
+  if (warp == kWLoadWarp) {
+    // ================= weight tile loader =================
+    if (lane == 0) {
+      const CUtensorMap* m = a.wmaps + (size_t)e * kMapsPerExpert;
+      const CUtensorMap* nib0 = m;
+      const CUtensorMap* sc0 = m + 1;
+      const CUtensorMap* nib1 = MODE == kModeGateUp ? m + 2 : m;
+      const CUtensorMap* sc1 = MODE == kModeGateUp ? m + 3 : m + 1;
+      tmap_acquire(nib0);
+      tmap_acquire(sc0);
+      if (MODE == kModeGateUp) {
+        tmap_acquire(nib1);
+        tmap_acquire(sc1);
+      }
+      const int y1 = MODE == kModeGateUp ? n0 : n0 + 128;
+      uint32_t issued = 0;
+      for (int g = 0; g < ngroups && !*abort_flag; ++g) {
+        for (int kt = 0; kt < ntile; ++kt) {
+          const uint32_t slot = issued % C::WS, round = issued / C::WS;
+          if (round > 0 && !wait(empty_w + 8 * slot, (round - 1) & 1)) break;
+          const uint32_t dst = s_base + C::OFF_W + slot * kWSlotBytes;
+          const uint32_t bar = full_w + 8 * slot;
+          mbar_arrive_expect_tx(bar, kWSlotBytes);
+          tma_load_2d(dst, nib0, kt * (kTileK / 2), n0, bar);
+          tma_load_2d(dst + kWNibBytes, nib1, kt * (kTileK / 2), y1, bar);
+          tma_load_2d(dst + 2 * kWNibBytes, sc0, kt * (kTileK / 16), n0, bar);
+          tma_load_2d(dst + 2 * kWNibBytes + kWScaleBytes, sc1, kt * (kTileK / 16), y1, bar);
+          ++issued;
         }
       }
-      cp_async_wait_all();
-    } else if (lane == 0) {
-      // ================= MMA issuer =================
+      // Let the last tiles land before the CTA can exit (they already have,
+      // unless a wait timed out).
+      for (uint32_t i = issued > (uint32_t)C::WS ? issued - C::WS : 0; i < issued; ++i)
+        mbar_wait(full_w + 8 * (i % C::WS), (i / C::WS) & 1);
+    }
+  } else if (warp == kBLoadWarp) {
+    // ================= token tile loader =================
+    if (lane == 0) {
+      uint32_t issued = 0;
+      for (int g = 0; g < ngroups && !*abort_flag; ++g) {
+        const int g0 = row_lo + g * NT;
+        for (int st = 0; st < nst; ++st) {
+          const uint32_t slot = issued % C::SB, round = issued / C::SB;
+          if (round > 0 && !wait(empty_b + 8 * slot, (round - 1) & 1)) break;
+          const uint32_t dst = s_base + C::OFF_B + slot * C::B_SLOT_BYTES;
+          const uint32_t bar = full_b + 8 * slot;
+          mbar_arrive_expect_tx(bar, C::B_SLOT_BYTES);
+          tma_load_2d(dst, &tm_b0, st * kStageK, g0, bar);
+          if constexpr (MODE == kModeDown) tma_load_2d(dst + C::B_PLANE_BYTES, &tm_b1, st * kStageK, g0, bar);
+          ++issued;
+        }
+      }
+      for (uint32_t i = issued > (uint32_t)C::SB ? issued - C::SB : 0; i < issued; ++i)
+        mbar_wait(full_b + 8 * (i % C::SB), (i / C::SB) & 1);
+    }
+  } else if (warp == kMmaWarp) {
+    // ================= MMA issuer =================
+    if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16_f32(128, NT);
-      for (int st = 0; st < nst && !*abort_flag; ++st) {
-        const uint32_t slot = (it + st) % kStages;
-        const uint32_t round = (it + st) / kStages;
-        if (!mbar_wait(bar_full + 8 * slot, round & 1)) {
-          *abort_flag = 1;
-          break;
+      for (int g = 0; g < ngroups; ++g) {
+        if (g > 0) {
+          wait(bar_dfree, (g - 1) & 1);  // the epilogue has read the previous group's D
+          tc_fence_after();
         }
-        tc_fence_after();
-        const uint32_t bslot = s_base + slot * C::B_SLOT_BYTES;
-        const uint32_t aslot = tmem_a + slot * C::A_COLS;
+        for (int st = 0; st < nst; ++st) {
+          const uint32_t ga = (uint32_t)(g * nst + st);
+          const uint32_t aslot = ga % C::SA, bslot = ga % C::SB;
+          if (!wait(full_a + 8 * aslot, (ga / C::SA) & 1)) break;
+          if (!wait(full_b + 8 * bslot, (ga / C::SB) & 1)) break;
+          tc_fence_after();
+          const uint32_t bbase = s_base + C::OFF_B + bslot * C::B_SLOT_BYTES;
+          const uint32_t abase = tmem_a + aslot * C::A_COLS;
 #pragma unroll
-        for (int s = 0; s < 4; ++s) {
-          const uint32_t acc = (st > 0 || s > 0) ? 1u : 0u;
-          const uint64_t bdesc = smem_desc_noswizzle(bslot + s * NT * 32, 128, 256);
-          tc_mma_f16_ts(tmem_d, aslot + s * 8, bdesc, idesc, acc);
-          tc_mma_f16_ts(tmem_d + NT, aslot + 32 + s * 8, bdesc, idesc, acc);
-          if constexpr (MODE == kModeDown) {
-            const uint64_t bdesc_lo = smem_desc_noswizzle(bslot + C::B_PLANE_BYTES + s * NT * 32, 128, 256);
-            tc_mma_f16_ts(tmem_d, aslot + s * 8, bdesc_lo, idesc, 1u);
-            tc_mma_f16_ts(tmem_d + NT, aslot + 32 + s * 8, bdesc_lo, idesc, 1u);
+          for (int s = 0; s < 4; ++s) {
+            const uint32_t acc = (st > 0 || s > 0) ? 1u : 0u;
+            const uint64_t bdesc = smem_desc_sw128(bbase + s * 32);
+            tc_mma_f16_ts(tmem_d, abase + s * 8, bdesc, idesc, acc);
+            tc_mma_f16_ts(tmem_d + NT, abase + 32 + s * 8, bdesc, idesc, acc);
+            if constexpr (MODE == kModeDown) {
+              const uint64_t bdesc_lo = smem_desc_sw128(bbase + C::B_PLANE_BYTES + s * 32);
+              tc_mma_f16_ts(tmem_d, abase + s * 8, bdesc_lo, idesc, 1u);
+              tc_mma_f16_ts(tmem_d + NT, abase + 32 + s * 8, bdesc_lo, idesc, 1u);
+            }
           }
+          tc_commit(empty_a + 8 * aslot);
+          tc_commit(empty_b + 8 * bslot);
         }
-        tc_commit(bar_empty + 8 * slot);
+        tc_commit(bar_done);  // also after a timeout, so nothing waits on MMAs in flight
       }
-      tc_commit(bar_done);
+      // No MMA may still run when TMEM is freed.
+      mbar_wait(bar_done, (ngroups - 1) & 1);
     }
-    it += nst;
+  } else {
+    // ================= decoders (warps 0..7) =================
+    const int prow = (warp & 3) * 32 + lane;   // row within the 128 of its matrix (= TMEM lane)
+    const int pmat = warp >> 2;                // gate / up, or the two halves of down
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const int swz = prow & 7;
+    const float s2a = a.s2_0[e];
+    const float s2b = a.s2_1[e];
+    for (int g = 0; g < ngroups; ++g) {
+      const int g0 = row_lo + g * NT;
+      const int nrows = min(NT, row_hi - g0);
+      for (int kt = 0; kt < ntile; ++kt) {
+        const uint32_t gw = (uint32_t)(g * ntile + kt);
+        const uint32_t wslot = gw % C::WS;
+        wait(full_w + 8 * wslot, (gw / C::WS) & 1);
+        const uint8_t* wtile = smem + C::OFF_W + wslot * kWSlotBytes;
+        const uint8_t* nrow = wtile + pmat * kWNibBytes + prow * 128;
+        const uint4 sc4 = *reinterpret_cast<const uint4*>(wtile + 2 * kWNibBytes + pmat * kWScaleBytes + prow * 16);
+        const uint32_t scw[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t ga = gw * 4 + j;
+          const uint32_t aslot = ga % C::SA, around = ga / C::SA;
+          // 32 nibble bytes (64 k) of this row: 16-byte chunks 2j, 2j+1, swizzled.
+          const uint4 q0 = *reinterpret_cast<const uint4*>(nrow + (((2 * j) ^ swz) << 4));
+          const uint4 q1 = *reinterpret_cast<const uint4*>(nrow + (((2 * j + 1) ^ swz) << 4));
+          uint32_t sc0, sc1;  // f16x2 (blk0, blk1), (blk2, blk3)
+          e4m3x4_to_f16x2x2(scw[j], sc0, sc1);
+          uint32_t v[32];
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const uint4 qq = q == 0 ? q0 : q1;
+            const uint32_t wv[4] = {qq.x, qq.y, qq.z, qq.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int blk = q * 2 + (i >> 1);  // 8 bytes (16 k) per block
+              const uint32_t scl = blk == 0 ? bcast_lo(sc0) : blk == 1 ? bcast_hi(sc0)
+                                   : blk == 2 ? bcast_lo(sc1) : bcast_hi(sc1);
+              uint32_t dec[4];
+              e2m1x8_to_f16x2x4(wv[i], dec);
+#pragma unroll
+              for (int jj = 0; jj < 4; ++jj) v[q * 16 + i * 4 + jj] = hmul2_u32(dec[jj], scl);
+            }
+          }
+          if (j == 3) {  // the weight tile is consumed: hand the slot back to the loader
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty_w + 8 * wslot);
+          }
+          // The A stage is free once the MMAs of stage ga - SA are done.
+          if (around > 0) wait(empty_a + 8 * aslot, (around - 1) & 1);
+          tc_fence_after();
+          tmem_st32(tmem_a + lane_off + aslot * C::A_COLS + pmat * 32, v);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(full_a + 8 * aslot);
+        }
+      }
 
-    // ================= epilogue =================
-    if (warp < kProdWarps) {
-      bool ok = !*abort_flag && mbar_wait(bar_done, groups & 1);
-      if (!ok) *abort_flag = 1;
+      // ---- epilogue: warps 0-3 take tokens [0, NT/2), warps 4-7 [NT/2, NT) ----
+      constexpr int HALF = NT / 2;
+      constexpr int CHUNK = HALF < 32 ? HALF : 32;  // tokens per scale load
+      const int tbase = pmat * HALF;
+      bool ok = wait(bar_done, g & 1);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
-      // Warps 0-3 take tokens [0, NT/2), warps 4-7 [NT/2, NT), each lane its row.
       const int n = n0 + prow;
-      constexpr int HALF = NT / 2;
 #pragma unroll 1
-      for (int t0 = pmat * HALF; t0 < (pmat + 1) * HALF; t0 += 8) {
-        uint32_t d0[8], d1[8];
-        tmem_ld8(tmem_d + lane_off + t0, d0);
-        tmem_ld8(tmem_d + lane_off + NT + t0, d1);
-        tmem_wait_ld();
-        if (ok) {
+      for (int c0 = 0; c0 < HALF; c0 += CHUNK) {
+        // lane l holds the scale of token tbase + c0 + l
+        const int tl = tbase + c0 + lane;
+        const float xm_l = (lane < CHUNK && tl < nrows) ? a.bexp[g0 + tl] : 0.0f;
+#pragma unroll 1
+        for (int t8 = 0; t8 < CHUNK; t8 += 8) {
+          uint32_t d0[8], d1[8];
+          tmem_ld8(tmem_d + lane_off + tbase + c0 + t8, d0);
+          tmem_ld8(tmem_d + lane_off + NT + tbase + c0 + t8, d1);
+          tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const int t = t0 + j;
-            if (t < nrows) {
-              const float xm = a.bexp[MODE == kModeGateUp ? rowsrc[t] : g0 + t];
+            const int t = tbase + c0 + t8 + j;
+            const float xm = __shfl_sync(0xffffffffu, xm_l, t8 + j);
+            if (ok && t < nrows) {
               float* dst = a.out + (size_t)(g0 + t) * N + n;
               if (MODE == kModeGateUp) {
                 const float gv = __uint_as_float(d0[j]) * xm * s2a;
@@ -439,104 +519,175 @@ __global__ void __launch_bounds__(kThreads, NT <= 16 ? 2 : 1) grouped_tc_kernel(
         }
       }
       tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_dfree);
     }
-    ++groups;
-    __syncthreads();  // accumulators and rowsrc are free for the next group
-    tc_fence_after();
   }
 
   __syncthreads();
-  if (warp == kProdWarps) tmem_dealloc(tmem, C::TMEM_COLS);
+  if (warp == kMmaWarp) {
+    __syncwarp();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
 }
 
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 
+namespace {
+
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime.
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Row-major 2-D tensor [rows, cols] of `elem`-byte elements at `base`; box
+// [box_rows, box_cols]; out-of-range rows read as zero.
+cudaError_t make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType type, uint32_t elem,
+                        uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols,
+                        CUtensorMapSwizzle swizzle) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * elem};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estride[2] = {1, 1};
+  const CUresult r = fn(map, type, 2, const_cast<void*>(base), dims, strides, box, estride,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <int MODE, int NT>
-cudaError_t launch_tc_impl(const TcArgs& a, uint32_t cap, cudaStream_t stream) {
+cudaError_t launch_tc_impl(const TcArgs& a, const CUtensorMap& b0, const CUtensorMap& b1, uint32_t cap,
+                           cudaStream_t stream) {
   using C = TcCfg<MODE, NT>;
   auto kern = grouped_tc_kernel<MODE, NT>;
   cudaError_t err = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::SMEM);
   if (err != cudaSuccess) return err;
   const dim3 grid(a.N / C::ROWS_PER_CTA, cap);
-  return launch_pdl(kern, grid, dim3(kThreads), C::SMEM, stream, a);
+  return launch_pdl(kern, grid, dim3(kThreads), C::SMEM, stream, a, b0, b1);
+}
+
+uint64_t al256(uint64_t v) { return (v + 255) & ~uint64_t(255); }
+
+// Workspace regions, in this order: gate+up [xs | xexp | weight maps], then
+// down [act hi | act lo | aexp | weight maps].
+struct WsLayout {
+  uint16_t* xs;
+  float* xexp;
+  CUtensorMap* maps_gu;
+  uint16_t* act_hi;
+  uint16_t* act_lo;
+  float* aexp;
+  CUtensorMap* maps_down;
+};
+WsLayout ws_layout(void* ws, uint64_t pairs, uint64_t hidden, uint64_t inter) {
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  WsLayout l;
+  l.xs = reinterpret_cast<uint16_t*>(p);
+  p += al256(pairs * hidden * 2);
+  l.xexp = reinterpret_cast<float*>(p);
+  p += al256(pairs * 4);
+  l.maps_gu = reinterpret_cast<CUtensorMap*>(p);
+  p += kMapBytes;
+  l.act_hi = reinterpret_cast<uint16_t*>(p);
+  p += al256(pairs * inter * 2);
+  l.act_lo = reinterpret_cast<uint16_t*>(p);
+  p += al256(pairs * inter * 2);
+  l.aexp = reinterpret_cast<float*>(p);
+  p += al256(pairs * 4);
+  l.maps_down = reinterpret_cast<CUtensorMap*>(p);
+  return l;
+}
+
+}  // namespace
+
+size_t tc_gate_up_workspace_bytes(uint64_t pairs, uint64_t hidden) {
+  return al256(pairs * hidden * 2) + al256(pairs * 4) + kMapBytes;
 }
 
 size_t tc_workspace_bytes(uint64_t tokens, uint64_t topk, uint64_t hidden, uint64_t inter) {
   const uint64_t pairs = tokens * topk;
-  auto al = [](uint64_t v) { return (v + 255) & ~uint64_t(255); };
-  return al(tokens * hidden * 2) + al(tokens * 4) + 2 * al(pairs * inter * 2) + al(pairs * 4);
+  return tc_gate_up_workspace_bytes(pairs, hidden) + 2 * al256(pairs * inter * 2) + al256(pairs * 4) +
+         kMapBytes;
 }
-
-namespace {
-struct WsLayout {
-  uint16_t* xs;
-  float* xexp;
-  uint16_t* act_hi;
-  uint16_t* act_lo;
-  float* aexp;
-};
-WsLayout ws_layout(void* ws, uint64_t tokens, uint64_t topk, uint64_t hidden, uint64_t inter) {
-  const uint64_t pairs = tokens * topk;
-  auto al = [](uint64_t v) { return (v + 255) & ~uint64_t(255); };
-  uint8_t* p = static_cast<uint8_t*>(ws);
-  WsLayout l;
-  l.xs = reinterpret_cast<uint16_t*>(p);
-  p += al(tokens * hidden * 2);
-  l.xexp = reinterpret_cast<float*>(p);
-  p += al(tokens * 4);
-  l.act_hi = reinterpret_cast<uint16_t*>(p);
-  p += al(pairs * inter * 2);
-  l.act_lo = reinterpret_cast<uint16_t*>(p);
-  p += al(pairs * inter * 2);
-  l.aexp = reinterpret_cast<float*>(p);
-  return l;
-}
-}  // namespace
 
 cudaError_t launch_tc(int mode, int nt, const GroupedArgs& g, void* workspace, uint32_t tokens,
                       uint32_t hidden, uint32_t inter, uint32_t cap, cudaStream_t stream) {
-  const WsLayout w = ws_layout(workspace, tokens, g.topk, hidden, inter);
-  const uint32_t pairs = tokens * g.topk;
+  const uint64_t pairs = (uint64_t)tokens * g.topk;
+  const WsLayout w = ws_layout(workspace, pairs, hidden, inter);
+  if (g.num_experts == 0 || g.num_experts > (uint32_t)kMaxExperts || (nt != 16 && nt != 128))
+    return cudaErrorInvalidValue;
   TcArgs a{};
   a.packed0 = g.packed0;
-  a.scale0 = g.scale0;
+  a.packed1 = g.packed1 != nullptr ? g.packed1 : g.packed0;
   a.s2_0 = g.s2_0;
-  a.packed1 = g.packed1;
-  a.scale1 = g.scale1;
-  a.s2_1 = g.s2_1;
+  a.s2_1 = g.s2_1 != nullptr ? g.s2_1 : g.s2_0;
   a.out = g.out;
   a.offsets = g.offsets;
-  a.sorted_pair_ids = g.sorted_pair_ids;
   a.active_experts = g.active_experts;
   a.active_count = g.active_count;
   a.N = g.N;
   a.K = g.K;
-  a.topk = g.topk;
-  cudaError_t err;
+
+  // Templates of the weight maps (address replaced per expert on the device):
+  // nibbles [N, K/2] u8 in 128 x 128-byte boxes with 128-byte swizzle, scales
+  // [N, K/16] u8 in 128 x 16-byte boxes.
+  CUtensorMap t_nib, t_scale, b0, b1;
+  cudaError_t err = make_map_2d(&t_nib, workspace, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.N, g.K / 2, 128,
+                                kTileK / 2, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (err != cudaSuccess) return err;
+  err = make_map_2d(&t_scale, workspace, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.N, g.K / 16, 128, kTileK / 16,
+                    CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (err != cudaSuccess) return err;
+  const uint32_t box_rows = (uint32_t)nt;
+
   if (mode == kModeGateUp) {
-    err = launch_pdl(pack_x_kernel, dim3((tokens + 7) / 8), dim3(256), 0, stream,
-                     static_cast<const uint16_t*>(g.src), (int)tokens, (int)g.K, w.xs, w.xexp);
+    err = launch_pdl(pack_x_sorted_kernel, dim3((unsigned)((pairs + 7) / 8)), dim3(256), 0, stream,
+                     static_cast<const uint16_t*>(g.src), (int)pairs, (int)g.K, (int)g.topk, g.sorted_pair_ids,
+                     g.offsets + g.num_experts, w.xs, w.xexp);
     if (err != cudaSuccess) return err;
-    a.b0 = w.xs;
-    a.b1 = w.xs;
+    err = launch_pdl(build_weight_maps_kernel, dim3(g.num_experts), dim3(128), 0, stream, t_nib, t_scale,
+                     g.packed0, g.scale0, g.packed1, g.scale1, 4, w.maps_gu);
+    if (err != cudaSuccess) return err;
+    err = make_map_2d(&b0, w.xs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, pairs, g.K, box_rows, kStageK,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+    if (err != cudaSuccess) return err;
+    b1 = b0;
     a.bexp = w.xexp;
-    if (nt == 16) return launch_tc_impl<kModeGateUp, 16>(a, cap, stream);
-    if (nt == 128) return launch_tc_impl<kModeGateUp, 128>(a, cap, stream);
-  } else {
-    // Rows past offsets[E] (dropped pairs) are not packed: offsets[E] bounds the grid's work.
-    err = launch_pdl(pack_act_kernel, dim3((pairs + 7) / 8), dim3(256), 0, stream,
-                     static_cast<const float*>(g.src), (int)pairs, (int)g.K, g.offsets + g.num_experts,
-                     w.act_hi, w.act_lo, w.aexp);
-    if (err != cudaSuccess) return err;
-    a.b0 = w.act_hi;
-    a.b1 = w.act_lo;
-    a.bexp = w.aexp;
-    if (nt == 16) return launch_tc_impl<kModeDown, 16>(a, cap, stream);
-    if (nt == 128) return launch_tc_impl<kModeDown, 128>(a, cap, stream);
+    a.wmaps = w.maps_gu;
+    if (nt == 16) return launch_tc_impl<kModeGateUp, 16>(a, b0, b1, cap, stream);
+    return launch_tc_impl<kModeGateUp, 128>(a, b0, b1, cap, stream);
   }
-  return cudaErrorInvalidValue;
+  // Rows past offsets[E] (dropped pairs) are not packed: offsets[E] bounds the grid's work.
+  err = launch_pdl(pack_act_kernel, dim3((unsigned)((pairs + 7) / 8)), dim3(256), 0, stream,
+                   static_cast<const float*>(g.src), (int)pairs, (int)g.K, g.offsets + g.num_experts, w.act_hi,
+                   w.act_lo, w.aexp);
+  if (err != cudaSuccess) return err;
+  err = launch_pdl(build_weight_maps_kernel, dim3(g.num_experts), dim3(128), 0, stream, t_nib, t_scale,
+                   g.packed0, g.scale0, g.packed0, g.scale0, 2, w.maps_down);
+  if (err != cudaSuccess) return err;
+  err = make_map_2d(&b0, w.act_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, pairs, g.K, box_rows, kStageK,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
+  if (err != cudaSuccess) return err;
+  err = make_map_2d(&b1, w.act_lo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, pairs, g.K, box_rows, kStageK,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
+  if (err != cudaSuccess) return err;
+  a.bexp = w.aexp;
+  a.wmaps = w.maps_down;
+  if (nt == 16) return launch_tc_impl<kModeDown, 16>(a, b0, b1, cap, stream);
+  return launch_tc_impl<kModeDown, 128>(a, b0, b1, cap, stream);
 }
 
 cudaError_t read_device_error(int* value, bool clear) {

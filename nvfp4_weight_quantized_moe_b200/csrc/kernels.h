@@ -43,9 +43,13 @@ cudaError_t launch_grouped(int mode, const DecodePlan& plan, const GroupedArgs& 
 bool grouped_plan_supported(int mode, const DecodePlan& plan);
 int grouped_rows_per_cta(int mode, int split);
 
-// tcgen05 path (grouped_tc.cu): activation packing into `workspace`, then the
-// projection kernel with NT token rows per pass (16 or 128).
+// tcgen05 path (grouped_tc.cu): activation packing and per-expert weight
+// tensor maps into `workspace` (256-byte aligned), then the projection kernel
+// with NT token rows per pass (16 or 128).
 size_t tc_workspace_bytes(uint64_t tokens, uint64_t topk, uint64_t hidden, uint64_t inter);
+// Leading part of that workspace the gate+up step uses (sorted f16 rows, their
+// scales and the per-expert weight tensor maps).
+size_t tc_gate_up_workspace_bytes(uint64_t pairs, uint64_t hidden);
 cudaError_t launch_tc(int mode, int nt, const GroupedArgs& a, void* workspace, uint32_t tokens,
                       uint32_t hidden, uint32_t inter, uint32_t cap, cudaStream_t stream);
 cudaError_t read_device_error(int* value, bool clear);

@@ -48,13 +48,10 @@ cudaError_t static_scratch_address(void** out) {
   return cudaSuccess;
 }
 
-// Bytes of scratch the gate+up call reads and writes: the packed rows
-// [num_tokens, k_hidden] f16, then one f32 scale per token (each 256-aligned),
-// the first two regions of the workspace layout of the _ws calls.
-size_t gate_up_scratch_bytes(uint64_t tokens, uint64_t hidden) {
-  auto al = [](uint64_t v) { return (v + 255) & ~uint64_t(255); };
-  return al(tokens * hidden * 2) + al(tokens * 4);
-}
+// Bytes of scratch the gate+up call reads and writes: the leading gate+up part
+// of the workspace layout of the _ws calls (packed rows by sorted position
+// [P, k_hidden] f16, one f32 scale per row, the per-expert weight tensor maps).
+size_t gate_up_scratch_bytes(uint64_t pairs, uint64_t hidden) { return tc_gate_up_workspace_bytes(pairs, hidden); }
 
 }  // namespace
 }  // namespace nvm
@@ -72,7 +69,7 @@ extern "C" int nvfp4_moe_gate_up_silu_noalloc(
   const uint64_t pairs = (uint64_t)num_tokens * topk;
   if (pairs > (1ull << 24)) return NVFP4_MOE_ESHAPE;
   // Requests whose packed rows do not fit the fixed scratch are refused.
-  if (gate_up_scratch_bytes(num_tokens, k_hidden) > kStaticScratchBytes) return NVFP4_MOE_ESHAPE;
+  if (gate_up_scratch_bytes(pairs, k_hidden) > kStaticScratchBytes) return NVFP4_MOE_ESHAPE;
   if (pairs == 0 || cap == 0) return NVFP4_MOE_OK;
   if (x == nullptr || act == nullptr || expert_offsets == nullptr || sorted_pair_ids == nullptr ||
       active_experts == nullptr || active_count == nullptr || gate.packed_ptrs == nullptr ||

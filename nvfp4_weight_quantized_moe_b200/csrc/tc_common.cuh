@@ -144,4 +144,43 @@ NVM_DEV void tc_commit(uint32_t bar) {
                : "memory");
 }
 
+// Shared-memory matrix descriptor, 128-byte swizzle, K-major: rows of 128 bytes
+// (64 f16 of K) in 1024-byte atoms of 8 rows, 16-byte chunk c of row r stored
+// at chunk c ^ (r % 8) (the layout a TMA tile load with 128-byte swizzle
+// writes).  SBO = 1024 bytes between 8-row groups; the leading offset is not
+// used by this layout.  The k-th 16-element step of a 64-element row starts
+// 32 k bytes after the atom base; the atom base must be 1024-byte aligned.
+NVM_DEV uint64_t smem_desc_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1 << 16;                   // leading byte offset (unused): 16 B
+  d |= (uint64_t)(1024 >> 4) << 32;         // stride byte offset
+  d |= (uint64_t)1 << 46;                   // descriptor version of sm_100
+  d |= (uint64_t)2 << 61;                   // layout type: 128-byte swizzle
+  return d;
+}
+
+// ---------------------------------------------------------------------------
+// TMA (cp.async.bulk.tensor) and tensor maps
+// ---------------------------------------------------------------------------
+// Arrive on `bar` and add `bytes` to the transaction count of its phase.
+NVM_DEV void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+// 2-D tiled load of the box at (x, y) (x innermost, in elements) of the tensor
+// map into shared memory at `dst`; completion is signalled on `bar` as bytes.
+// No multicast.
+NVM_DEV void tma_load_2d(uint32_t dst, const void* tmap, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(dst),
+      "l"(tmap), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+// Order this thread's later TMA reads of the tensor map at `tmap` (global
+// memory, written by an earlier kernel) after that kernel's release.
+NVM_DEV void tmap_acquire(const void* tmap) {
+  asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(tmap) : "memory");
+}
+
 }  // namespace nvm

@@ -78,7 +78,7 @@ def test_no_alloc_refuses_requests_beyond_its_scratch():
     from nvfp4_weight_quantized_moe_b200 import _binding as B
     t = B.ExpertTables(8, 8, 8)
     p = ctypes.c_void_p(8)
-    # 8192 tokens x 1024 hidden x 2 bytes = 16 MiB of packed rows: over the limit.
+    # 8192 tokens x 4 pairs x 1024 hidden x 2 bytes = 64 MiB of packed rows: over the limit.
     status = B._lib.nvfp4_moe_gate_up_silu_noalloc(p, t, t, p, p, p, p, p, 512, 1024, 16, 8192, 4,
                                                    16, None)
     assert status == 2
