@@ -50,7 +50,6 @@ DEFAULT_STEPS = {"tiny": 20000, "decode_m1": 20000, "decode_m32": 5000, "decode_
 NCU_TRAFFIC_BYTES = {
     ("decode_m1", "mma.sync"): 28355840,     # 28.36 MB read, 0 written (routed gate+up: 28.31 MB)
     ("decode_m32", "mma.sync"): 316248320,   # 311.60 MB read, 4.64 MB written
-    ("prefill_m8192", "tcgen05"): 4047628000,  # 3.658 GB read, 0.390 GB written (4 token passes)
 }
 
 
@@ -360,7 +359,8 @@ def run_ours(args, rank, world, local):
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": (6 if tc else 4) * steps,
+        # route_sort, [pack, tensor maps,] gate+up, [pack, tensor maps,] down, blend
+        "gpu_launches": (8 if tc else 4) * steps,
         "clocks": clocks,
     }
     if rank == 0:
@@ -377,10 +377,10 @@ def _opts(args):
 def _tc_path(args, cfg):
     """Whether the projections take the tcgen05 path (the library's rule for
     the workspace calls: widths divisible by 128 / 256, and path 2, or path 0
-    with at least 4 routed rows per expert on average)."""
+    with at least 2 routed rows per expert on average)."""
     if args.path == 1 or cfg.inter % 128 or cfg.hidden % 256:
         return False
-    return args.path == 2 or cfg.pairs >= 4 * cfg.experts
+    return args.path == 2 or cfg.pairs >= 2 * cfg.experts
 
 
 def _uses_prefill(args, cfg):

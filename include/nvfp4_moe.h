@@ -194,7 +194,7 @@ NVFP4_MOE_API size_t nvfp4_moe_workspace_bytes(uint32_t num_tokens, uint32_t top
 /*
  * Steps 2 and 3 with a workspace, which opens the tcgen05 path (path 2, or
  * path 0 when the output width is a multiple of 128 for gate+up, 256 for
- * down, and there are at least 4 routed rows per expert on average; path 2
+ * down, and there are at least 2 routed rows per expert on average; path 2
  * with another width returns NVFP4_MOE_ESHAPE): activations are packed
  * once into f16 rows by sorted position (x gathered from its token; act as an
  * f16 hi + lo pair; each row scaled by a power of two into the f16 range),

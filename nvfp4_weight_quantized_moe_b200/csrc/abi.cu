@@ -225,15 +225,16 @@ int plan_tc_rows(uint64_t tokens, uint64_t pairs, uint32_t num_experts, const nv
 }
 
 // The tcgen05 kernel covers 128 (gate+up) or 256 (down) output rows per CTA.
-// Chosen automatically from 4 routed rows per expert on average: below that
-// the register-fed decode kernel keeps more weight bytes in flight per SM
-// (measured on B200: faster at 0.06 and 2 rows per expert, slower at 8).
+// Chosen automatically from 2 routed rows per expert on average: below that
+// the register-fed decode kernel, which splits K over more CTAs, keeps more
+// weight bytes in flight (measured on B200: decode kernel 2x faster at 0.06
+// rows per expert; tcgen05 7% faster at 2 and 28% at 8).
 bool use_tc(uint32_t n, uint32_t rows_per_cta, uint64_t pairs, uint32_t num_experts,
             const nvfp4_moe_launch_opts* o) {
   const int path = o ? o->path : 0;
   if (path == 1 || n % rows_per_cta != 0) return false;
   if (path == 2) return true;
-  return pairs >= 4ull * num_experts;
+  return pairs >= 2ull * num_experts;
 }
 
 }  // namespace

@@ -109,7 +109,12 @@ NVM_DEV float warp_max(float v) {
   return v;
 }
 
-NVM_DEV float silu_f32(float z) { return z / (1.0f + expf(-z)); }
+// SiLU(z) = z / (1 + exp(-z)) in FP32 with the hardware exponential and the
+// fast divide (relative error ~1e-5 over the range; the IEEE-rounded divide or
+// reciprocal takes a slow path whenever exp(-z) overflows, which is common for
+// large negative gate values).  For z < -87 the denominator is >= 2^126 and the
+// fast divide returns 0, the limit of SiLU there.
+NVM_DEV float silu_f32(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 // ---------------------------------------------------------------------------
 // Programmatic dependent launch and L2 prefetch

@@ -93,20 +93,26 @@ struct TcCfg {
   static constexpr int A_COLS = 64;                             // TMEM columns per stage
   static constexpr int D_COLS = 2 * NT;
   static constexpr int SA = NT <= 16 ? 3 : 4;
-  static constexpr int WS = (NT <= 16 || MODE == kModeDown) ? 2 : 3;
-  static constexpr int SB = (MODE == kModeDown && NT > 16) ? 4 : 6;
+  static constexpr int WS = 2;
+  static constexpr int SB = (MODE == kModeDown && NT > 16) ? 4 : 8;
   static constexpr uint32_t TMEM_COLS = pow2_at_least(D_COLS + SA * A_COLS);
   static constexpr int OFF_W = 0;
   static constexpr int OFF_B = WS * kWSlotBytes;
   static constexpr int OFF_BAR = OFF_B + SB * B_SLOT_BYTES;
-  // full_w[WS], empty_w[WS], full_b[SB], empty_b[SB], full_a[SA], empty_a[SA], done, d_free
-  static constexpr int NBAR = 2 * WS + 2 * SB + 2 * SA + 2;
+  // MMA completion is committed once per CG stages (a commit costs
+  // tensor-pipe time); mma_done has SB / CG entries.
+  static constexpr int CG = 2;
+  static constexpr int NMD = SB / CG;
+  // full_w[WS], empty_w[WS], full_b[SB], mma_done[NMD], full_a[SA], done, d_free
+  static constexpr int NBAR = 2 * WS + SB + NMD + SA + 2;
   static constexpr int OFF_TMEM = OFF_BAR + 8 * NBAR;
   static constexpr int OFF_ABORT = OFF_TMEM + 16;
   static constexpr int SMEM = OFF_ABORT + 16 + 1024;  // + room to align the base to 1024 B
   static constexpr int CTAS_PER_SM = kSmemPerSM / (SMEM + kSmemReservedPerCta);
   static_assert(B_PLANE_BYTES % 1024 == 0 && kWSlotBytes % 1024 == 0, "TMA tiles stay 1024-byte aligned");
   static_assert(TMEM_COLS <= 512, "TMEM budget");
+  static_assert(SB % CG == 0 && (kTileK / kStageK) % CG == 0, "commit groups tile the stages");
+  static_assert(SB >= SA, "mma_done also tracks the A ring");
   // Every CTA that shared memory lets share an SM must find its TMEM columns
   // free, or a CTA would wait in tcgen05.alloc.
   static_assert(CTAS_PER_SM >= 1 && CTAS_PER_SM * TMEM_COLS <= 512, "TMEM per SM");
@@ -252,8 +258,11 @@ struct TcArgs {
   uint32_t N, K;
 };
 
+// Registers: 128-token tiles run one CTA per SM, 16-token tiles two.  The
+// register file is handed out to warps in groups of four, so the 11 warps
+// count as 12: at most 168 registers per thread for one CTA, 80 for two.
 template <int MODE, int NT>
-__global__ void __launch_bounds__(kThreads, NT <= 16 ? 2 : 1)
+__global__ void __launch_bounds__(kThreads) __maxnreg__(NT <= 16 ? 80 : 168)
     grouped_tc_kernel(const TcArgs a, const __grid_constant__ CUtensorMap tm_b0,
                       const __grid_constant__ CUtensorMap tm_b1) {
   using C = TcCfg<MODE, NT>;
@@ -264,10 +273,11 @@ __global__ void __launch_bounds__(kThreads, NT <= 16 ? 2 : 1)
   const uint32_t full_w = s_base + C::OFF_BAR;     // TMA weight tile landed (+ 8 * slot)
   const uint32_t empty_w = full_w + 8 * C::WS;     // decoders done with the tile
   const uint32_t full_b = empty_w + 8 * C::WS;     // TMA token tile landed
-  const uint32_t empty_b = full_b + 8 * C::SB;     // MMAs done with the tile
-  const uint32_t full_a = empty_b + 8 * C::SB;     // decoded A stage in TMEM
-  const uint32_t empty_a = full_a + 8 * C::SA;     // MMAs done with the A stage
-  const uint32_t bar_done = empty_a + 8 * C::SA;   // a group's accumulators are final
+  // mma_done[(ga / CG) % NMD]: the MMAs of stages up to CG (ga / CG) + CG - 1
+  // have completed.  It frees B slot ga % SB and A slot ga % SA.
+  const uint32_t mma_done = full_b + 8 * C::SB;
+  const uint32_t full_a = mma_done + 8 * C::NMD;   // decoded A stage in TMEM
+  const uint32_t bar_done = full_a + 8 * C::SA;    // a group's accumulators are final
   const uint32_t bar_dfree = bar_done + 8;         // the epilogue has read them
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_ABORT);
@@ -298,14 +308,9 @@ __global__ void __launch_bounds__(kThreads, NT <= 16 ? 2 : 1)
       mbar_init(full_w + 8 * s, 1);
       mbar_init(empty_w + 8 * s, kProdWarps);
     }
-    for (int s = 0; s < C::SB; ++s) {
-      mbar_init(full_b + 8 * s, 1);
-      mbar_init(empty_b + 8 * s, 1);
-    }
-    for (int s = 0; s < C::SA; ++s) {
-      mbar_init(full_a + 8 * s, kProdWarps);
-      mbar_init(empty_a + 8 * s, 1);
-    }
+    for (int s = 0; s < C::SB; ++s) mbar_init(full_b + 8 * s, 1);
+    for (int s = 0; s < C::NMD; ++s) mbar_init(mma_done + 8 * s, 1);
+    for (int s = 0; s < C::SA; ++s) mbar_init(full_a + 8 * s, kProdWarps);
     mbar_init(bar_done, 1);
     mbar_init(bar_dfree, kProdWarps);
     *abort_flag = 0;
@@ -328,6 +333,11 @@ __global__ void __launch_bounds__(kThreads, NT <= 16 ? 2 : 1)
     if (mbar_wait(bar, parity)) return true;
     *abort_flag = 1;
     return false;
+  };
+  // Wait until the MMAs of stage x (and the rest of its commit group) are done.
+  auto wait_mma = [&](uint32_t x) -> bool {
+    const uint32_t grp = x / C::CG;
+    return wait(mma_done + 8 * (grp % C::NMD), (grp / C::NMD) & 1);
   };
 
   if (warp == kWLoadWarp) {
@@ -373,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, NT <= 16 ? 2 : 1)
         const int g0 = row_lo + g * NT;
         for (int st = 0; st < nst; ++st) {
           const uint32_t slot = issued % C::SB, round = issued / C::SB;
-          if (round > 0 && !wait(empty_b + 8 * slot, (round - 1) & 1)) break;
+          if (round > 0 && !wait_mma(issued - C::SB)) break;
           const uint32_t dst = s_base + C::OFF_B + slot * C::B_SLOT_BYTES;
           const uint32_t bar = full_b + 8 * slot;
           mbar_arrive_expect_tx(bar, C::B_SLOT_BYTES);
@@ -414,8 +424,7 @@ __global__ void __launch_bounds__(kThreads, NT <= 16 ? 2 : 1)
               tc_mma_f16_ts(tmem_d + NT, abase + 32 + s * 8, bdesc_lo, idesc, 1u);
             }
           }
-          tc_commit(empty_a + 8 * aslot);
-          tc_commit(empty_b + 8 * bslot);
+          if (ga % C::CG == C::CG - 1) tc_commit(mma_done + 8 * ((ga / C::CG) % C::NMD));
         }
         tc_commit(bar_done);  // also after a timeout, so nothing waits on MMAs in flight
       }
@@ -430,9 +439,109 @@ __global__ void __launch_bounds__(kThreads, NT <= 16 ? 2 : 1)
     const int swz = prow & 7;
     const float s2a = a.s2_0[e];
     const float s2b = a.s2_1[e];
-    for (int g = 0; g < ngroups; ++g) {
+
+    // Epilogue.  Warps 0-3 take tokens [0, NT/2), warps 4-7 [NT/2, NT), each
+    // lane its output row n0 + prow.
+    constexpr int HALF = NT / 2;
+    constexpr int CHUNK = HALF < 32 ? HALF : 32;  // tokens per scale load
+    constexpr int TL = HALF < 16 ? HALF : 16;     // tokens per TMEM load
+    const int tbase = pmat * HALF;
+    const int n = n0 + prow;
+
+    // Down: read D and store it directly, then hand D back to the MMA.
+    auto epilogue_down = [&](int g) {
       const int g0 = row_lo + g * NT;
       const int nrows = min(NT, row_hi - g0);
+      bool ok = wait(bar_done, g & 1);
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+#pragma unroll 1
+      for (int c0 = 0; c0 < HALF; c0 += CHUNK) {
+        // lane l holds the scale of token tbase + c0 + l
+        const int tl = tbase + c0 + lane;
+        const float xm_l = (lane < CHUNK && tl < nrows) ? a.bexp[g0 + tl] : 0.0f;
+#pragma unroll 1
+        for (int tt = 0; tt < CHUNK; tt += TL) {
+          uint32_t d0[TL], d1[TL];
+#pragma unroll
+          for (int h = 0; h < TL; h += 8) {
+            tmem_ld8(tmem_d + lane_off + tbase + c0 + tt + h, *reinterpret_cast<uint32_t(*)[8]>(d0 + h));
+            tmem_ld8(tmem_d + lane_off + NT + tbase + c0 + tt + h, *reinterpret_cast<uint32_t(*)[8]>(d1 + h));
+          }
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < TL; ++j) {
+            const int t = tbase + c0 + tt + j;
+            const float xm = __shfl_sync(0xffffffffu, xm_l, tt + j);
+            if (ok && t < nrows) {
+              float* dst = a.out + (size_t)(g0 + t) * N + n;
+              dst[0] = __uint_as_float(d0[j]) * xm * s2a;
+              dst[128] = __uint_as_float(d1[j]) * xm * s2a;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_dfree);
+    };
+
+    // Gate+up: SiLU(gate) * up of every token of this thread goes to registers
+    // first and D is handed back at once; the stores follow while the MMA
+    // already runs the next group's first stages.
+    float res[MODE == kModeGateUp ? HALF : 1];
+    int res_g0 = 0, res_nrows = 0;
+    bool res_ok = false;
+    // Row scales of the group being decoded (xm_cur) and of the one before
+    // (xm_prev), loaded when a group starts: lane l holds token tbase + 32 c + l.
+    constexpr int NXC = HALF / CHUNK;
+    float xm_cur[NXC], xm_prev[NXC];
+    auto load_scales = [&](int g) {
+      const int g0 = row_lo + g * NT;
+      const int nrows = min(NT, row_hi - g0);
+#pragma unroll
+      for (int c = 0; c < NXC; ++c) {
+        xm_prev[c] = xm_cur[c];
+        const int tl = tbase + c * CHUNK + lane;
+        xm_cur[c] = (lane < CHUNK && tl < nrows) ? a.bexp[g0 + tl] : 0.0f;
+      }
+    };
+    auto epilogue_gate_up = [&](int g, const float (&xm_g)[NXC]) {
+      res_g0 = row_lo + g * NT;
+      res_nrows = min(NT, row_hi - res_g0);
+      bool ok = wait(bar_done, g & 1);
+      res_ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+#pragma unroll
+      for (int c0 = 0; c0 < HALF; c0 += CHUNK) {
+        const float xm_l = xm_g[c0 / CHUNK];
+#pragma unroll
+        for (int tt = 0; tt < CHUNK; tt += 8) {
+          uint32_t d0[8], d1[8];
+          tmem_ld8(tmem_d + lane_off + tbase + c0 + tt, d0);
+          tmem_ld8(tmem_d + lane_off + NT + tbase + c0 + tt, d1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float xm = __shfl_sync(0xffffffffu, xm_l, tt + j);
+            const float gv = __uint_as_float(d0[j]) * xm * s2a;
+            const float uv = __uint_as_float(d1[j]) * xm * s2b;
+            res[c0 + tt + j] = silu_f32(gv) * uv;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_dfree);
+#pragma unroll
+      for (int j = 0; j < HALF; ++j) {
+        const int t = tbase + j;
+        if (res_ok && t < res_nrows) a.out[(size_t)(res_g0 + t) * N + n] = res[j];
+      }
+    };
+
+    for (int g = 0; g < ngroups; ++g) {
+      if constexpr (MODE == kModeGateUp) load_scales(g);
       for (int kt = 0; kt < ntile; ++kt) {
         const uint32_t gw = (uint32_t)(g * ntile + kt);
         const uint32_t wslot = gw % C::WS;
@@ -450,9 +559,9 @@ __global__ void __launch_bounds__(kThreads, NT <= 16 ? 2 : 1)
           const uint4 q1 = *reinterpret_cast<const uint4*>(nrow + (((2 * j + 1) ^ swz) << 4));
           uint32_t sc0, sc1;  // f16x2 (blk0, blk1), (blk2, blk3)
           e4m3x4_to_f16x2x2(scw[j], sc0, sc1);
-          uint32_t v[32];
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
+          // 32 k per half (16 TMEM columns).  The first half is decoded before
+          // waiting for the A slot, so a freed slot mostly waits for stores.
+          auto decode_half = [&](int q, uint32_t (&v)[16]) {
             const uint4 qq = q == 0 ? q0 : q1;
             const uint32_t wv[4] = {qq.x, qq.y, qq.z, qq.w};
 #pragma unroll
@@ -463,64 +572,39 @@ __global__ void __launch_bounds__(kThreads, NT <= 16 ? 2 : 1)
               uint32_t dec[4];
               e2m1x8_to_f16x2x4(wv[i], dec);
 #pragma unroll
-              for (int jj = 0; jj < 4; ++jj) v[q * 16 + i * 4 + jj] = hmul2_u32(dec[jj], scl);
+              for (int jj = 0; jj < 4; ++jj) v[i * 4 + jj] = hmul2_u32(dec[jj], scl);
             }
-          }
+          };
+          uint32_t v[16];
+          decode_half(0, v);
           if (j == 3) {  // the weight tile is consumed: hand the slot back to the loader
             __syncwarp();
             if (lane == 0) mbar_arrive(empty_w + 8 * wslot);
           }
           // The A stage is free once the MMAs of stage ga - SA are done.
-          if (around > 0) wait(empty_a + 8 * aslot, (around - 1) & 1);
+          if (around > 0) wait_mma(ga - C::SA);
           tc_fence_after();
-          tmem_st32(tmem_a + lane_off + aslot * C::A_COLS + pmat * 32, v);
+          tmem_st16(tmem_a + lane_off + aslot * C::A_COLS + pmat * 32, v);
+          decode_half(1, v);
+          tmem_st16(tmem_a + lane_off + aslot * C::A_COLS + pmat * 32 + 16, v);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(full_a + 8 * aslot);
-        }
-      }
-
-      // ---- epilogue: warps 0-3 take tokens [0, NT/2), warps 4-7 [NT/2, NT) ----
-      constexpr int HALF = NT / 2;
-      constexpr int CHUNK = HALF < 32 ? HALF : 32;  // tokens per scale load
-      const int tbase = pmat * HALF;
-      bool ok = wait(bar_done, g & 1);
-      ok = __all_sync(0xffffffffu, ok);
-      tc_fence_after();
-      const int n = n0 + prow;
-#pragma unroll 1
-      for (int c0 = 0; c0 < HALF; c0 += CHUNK) {
-        // lane l holds the scale of token tbase + c0 + l
-        const int tl = tbase + c0 + lane;
-        const float xm_l = (lane < CHUNK && tl < nrows) ? a.bexp[g0 + tl] : 0.0f;
-#pragma unroll 1
-        for (int t8 = 0; t8 < CHUNK; t8 += 8) {
-          uint32_t d0[8], d1[8];
-          tmem_ld8(tmem_d + lane_off + tbase + c0 + t8, d0);
-          tmem_ld8(tmem_d + lane_off + NT + tbase + c0 + t8, d1);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int t = tbase + c0 + t8 + j;
-            const float xm = __shfl_sync(0xffffffffu, xm_l, t8 + j);
-            if (ok && t < nrows) {
-              float* dst = a.out + (size_t)(g0 + t) * N + n;
-              if (MODE == kModeGateUp) {
-                const float gv = __uint_as_float(d0[j]) * xm * s2a;
-                const float uv = __uint_as_float(d1[j]) * xm * s2b;
-                *dst = silu_f32(gv) * uv;
-              } else {
-                dst[0] = __uint_as_float(d0[j]) * xm * s2a;
-                dst[128] = __uint_as_float(d1[j]) * xm * s2a;
-              }
-            }
+          // Once the first SA stages of this group are in TMEM (all the A ring
+          // holds before the MMA may start on them), drain the previous group,
+          // so the MMA finds its next stages ready the moment D is free.
+          if (g > 0 && kt * 4 + j == C::SA - 1) {
+            if constexpr (MODE == kModeGateUp) epilogue_gate_up(g - 1, xm_prev);
+            else epilogue_down(g - 1);
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_dfree);
+    }
+    if constexpr (MODE == kModeGateUp) {
+      epilogue_gate_up(ngroups - 1, xm_cur);
+    } else {
+      epilogue_down(ngroups - 1);
     }
   }
 
