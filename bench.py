@@ -45,11 +45,12 @@ DEFAULT_STEPS = {"tiny": 20000, "decode_m1": 20000, "decode_m32": 5000, "decode_
 
 # DRAM bytes (read + write) of one launch of the dominant kernel (gate+up
 # SiLU) from an ncu capture of the same kernel build and launch shape; see the
-# grouped_mma_*_ncu_full summaries.  Absent for workloads not captured, and
-# cleared whenever that kernel changes.
+# summaries under profiles/.  Absent for workloads not captured, and cleared
+# whenever that kernel changes.
 NCU_TRAFFIC_BYTES = {
-    ("decode_m1", "mma.sync"): 28355840,     # 28.36 MB read, 0 written (routed gate+up: 28.31 MB)
-    ("decode_m32", "mma.sync"): 316248320,   # 311.60 MB read, 4.64 MB written
+    ("decode_m1", "mma.sync"): 28357888,      # 28.36 MB read, 0 written (routed gate+up: 28.31 MB)
+    ("decode_m32", "tcgen05"): 334938368,     # 330.22 MB read, 4.72 MB written
+    ("prefill_m8192", "tcgen05"): 4236745000,  # 3.826 GB read, 0.411 GB written (4 token passes)
 }
 
 
