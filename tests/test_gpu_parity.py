@@ -155,6 +155,28 @@ def test_route_sort_out_of_range_ids_and_max_experts():
         assert int(bufs.status.item()) == 1
 
 
+def test_route_sort_small_batches_bit_exact():
+    # Up to 32 pairs take the single-warp sort: cover every P in 1..33 (the
+    # boundary on both sides), out-of-range ids, one expert, and 1024 experts.
+    _need_gpu()
+    import nvfp4_weight_quantized_moe_b200 as nvm
+    rng = np.random.default_rng(11)
+    for p in range(1, 34):
+        for e in (1, 7, 128, 1024):
+            k = int(rng.integers(1, min(e, 8) + 1))
+            m = max(1, p // k)
+            ids = rng.integers(-1, e + 1, (m, k)).astype(np.int32)
+            bufs = nvm.MoEBuffers(m, k, e, 4, 4, "cuda")
+            nvm.route_sort(torch.from_numpy(ids).cuda(), e, bufs.expert_offsets, bufs.sorted_pair_ids,
+                           bufs.pair_pos, bufs.active_experts, bufs.active_count, bufs.status)
+            torch.cuda.synchronize()
+            rs = orc.route_sort(ids, e)
+            _check_sort(bufs, rs, e, m * k)
+            kept = int(rs.expert_offsets[-1])
+            assert np.all(bufs.sorted_pair_ids.cpu().numpy()[kept:m * k] == -1)
+            assert int(bufs.status.item()) == (1 if rs.dropped > 0 else 0)
+
+
 # --------------------------------------------------------------------------- #
 # transpose_u8: bit-exact
 # --------------------------------------------------------------------------- #
