@@ -9,10 +9,11 @@
 //      "count > 0" flags, the ascending list of active experts;
 //   3. the pairs are placed in passes of 1024 in pair order.  Inside a warp,
 //      __match_any_sync finds the lanes with the same expert and the rank of a
-//      lane among them; per-warp counts per expert, scanned over the 32 warps in
-//      warp order, give each warp's base, so a pair's position is
-//      cursor[e] + warp base + lane rank: ascending pair id within an expert,
-//      the same result on every run.
+//      lane among them; per-warp counts per expert (stored [expert][warp], so
+//      one warp scans an expert's 32 counts with shuffles) give each warp's
+//      base, so a pair's position is cursor[e] + warp base + lane rank:
+//      ascending pair id within an expert, the same result on every run.  The
+//      next pass's ids are loaded while the current pass is placed.
 // Out-of-range ids are dropped (pair_pos = -1) and flagged in `status`.
 //
 // Up to 32 pairs (decode batches of a few tokens) take route_sort_small_kernel
@@ -72,7 +73,7 @@ __global__ void __launch_bounds__(kSortThreads)
   extern __shared__ int sm[];
   int* cnt = sm;                                            // [E]
   int* cursor = sm + E;                                     // [E]
-  uint16_t* wc = reinterpret_cast<uint16_t*>(sm + 2 * E);   // [32][E]
+  uint16_t* wc = reinterpret_cast<uint16_t*>(sm + 2 * E);   // [E][32]
   __shared__ int tmp[33];
   __shared__ int bad;
 
@@ -80,6 +81,7 @@ __global__ void __launch_bounds__(kSortThreads)
   griddep_wait();  // the previous kernel on the stream (e.g. the last blend) is done
   griddep_launch_dependents();
   for (int i = tid; i < E; i += kSortThreads) cnt[i] = 0;
+  for (int i = tid; i < 32 * E; i += kSortThreads) wc[i] = 0;
   if (tid == 0) bad = 0;
   __syncthreads();
   for (int p = tid; p < P; p += kSortThreads) {
@@ -106,35 +108,42 @@ __global__ void __launch_bounds__(kSortThreads)
   for (int i = nactive + tid; i < E; i += kSortThreads) active[i] = -1;
   for (int i = kept + tid; i < P; i += kSortThreads) sorted[i] = -1;
 
+  int v_next = tid < P ? ids[tid] : -1;
   for (int base = 0; base < P; base += kSortThreads) {
-    for (int i = tid; i < 32 * E; i += kSortThreads) wc[i] = 0;
     const int p = base + tid;
-    const int v = p < P ? ids[p] : -1;
+    const int v = p < P ? v_next : -1;
+    if (base + kSortThreads + tid < P) v_next = ids[base + kSortThreads + tid];
     const bool valid = (unsigned)v < (unsigned)E;
     const unsigned peers = __match_any_sync(0xffffffffu, valid ? v : -1);
     const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (valid && rank == 0) wc[v * 32 + warp] = (uint16_t)__popc(peers);
     __syncthreads();
-    if (valid && rank == 0) wc[warp * E + v] = (uint16_t)__popc(peers);
-    __syncthreads();
-    if (tid < E) {
-      int run = 0;
-      for (int w = 0; w < 32; ++w) {
-        const int t = wc[w * E + tid];
-        wc[w * E + tid] = (uint16_t)run;
-        run += t;
+    // Exclusive scan of each expert's 32 per-warp counts, one warp per expert.
+    for (int e = warp; e < E; e += 32) {
+      const int c = wc[e * 32 + lane];
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
       }
-      cnt[tid] = run;
+      wc[e * 32 + lane] = (uint16_t)(incl - c);
+      if (lane == 31) cnt[e] = incl;
     }
     __syncthreads();
     if (valid) {
-      const int pos = cursor[v] + wc[warp * E + v] + rank;
+      const int pos = cursor[v] + wc[v * 32 + warp] + rank;
       sorted[pos] = p;
       pair_pos[p] = pos;
     } else if (p < P) {
       pair_pos[p] = -1;
     }
     __syncthreads();
-    if (tid < E) cursor[tid] += cnt[tid];
+    // The same warp clears its experts' counts and advances their cursors.
+    for (int e = warp; e < E; e += 32) {
+      wc[e * 32 + lane] = 0;
+      if (lane == 0) cursor[e] += cnt[e];
+    }
     __syncthreads();
   }
 }
