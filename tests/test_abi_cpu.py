@@ -90,3 +90,35 @@ def test_active_cap_and_status_strings(lib):
     L = m._binding._lib
     for s in range(4):
         assert L.nvfp4_moe_status_string(s)
+
+
+def test_workspace_calls_check_size_and_alignment_on_the_host(lib):
+    # The tcgen05 path (path 2) needs nvfp4_moe_workspace_bytes of 256-byte aligned
+    # workspace; a short or misaligned one is refused before anything is launched.
+    import nvfp4_weight_quantized_moe_b200._binding as B
+    L = B._lib
+    t = B.ExpertTables(8, 8, 8)
+    p8 = ctypes.c_void_p(8)
+    tokens, topk, hidden, inter, experts = 16, 4, 512, 256, 8
+    need = L.nvfp4_moe_workspace_bytes(tokens, topk, hidden, inter)
+    pairs = tokens * topk
+    # sorted f16 rows, their scales, 512 KiB of tensor maps, act hi + lo, their scales, maps
+    assert need >= pairs * hidden * 2 + pairs * inter * 4 + 2 * (512 << 10)
+    opts = B.LaunchOpts(2, 0, 0, 0)
+    cap = min(experts, pairs)
+
+    def gate_up(ws, nbytes):
+        return L.nvfp4_moe_gate_up_silu_ws(p8, t, t, p8, p8, p8, p8, p8, inter, hidden, cap, tokens, topk,
+                                           experts, ctypes.byref(opts), ws, nbytes, None)
+
+    def down(ws, nbytes):
+        return L.nvfp4_moe_down_ws(p8, t, p8, p8, p8, p8, hidden, inter, cap, tokens, topk, experts,
+                                   ctypes.byref(opts), ws, nbytes, None)
+
+    for call in (gate_up, down):
+        assert call(None, need) == 1
+        assert call(ctypes.c_void_p(1 << 20), need - 1) == 1
+        assert call(ctypes.c_void_p((1 << 20) + 128), need) == 1
+    # path 2 with a width the tcgen05 kernels do not take
+    assert L.nvfp4_moe_down_ws(p8, t, p8, p8, p8, p8, 128, inter, cap, tokens, topk, experts,
+                               ctypes.byref(opts), ctypes.c_void_p(1 << 20), need, None) == 2
