@@ -9,12 +9,19 @@
 //      "count > 0" flags, the ascending list of active experts;
 //   3. the pairs are placed in passes of 1024 in pair order.  Inside a warp,
 //      __match_any_sync finds the lanes with the same expert and the rank of a
-//      lane among them; per-warp counts per expert (stored [expert][warp], so
-//      one warp scans an expert's 32 counts with shuffles) give each warp's
-//      base, so a pair's position is cursor[e] + warp base + lane rank:
-//      ascending pair id within an expert, the same result on every run.  The
-//      next pass's ids are loaded while the current pass is placed.
+//      lane among them; per-warp counts per expert, scanned over the 32 warps in
+//      warp order, give each warp's base, so a pair's position is
+//      cursor[e] + warp base + lane rank: ascending pair id within an expert,
+//      the same result on every run.
 // Out-of-range ids are dropped (pair_pos = -1) and flagged in `status`.
+//
+// Large batches (more than 4096 pairs, prefill) take route_sort_cluster_kernel:
+// a cluster of 8 CTAs, CTA r owning the r-th contiguous eighth of the pairs.
+// Each CTA counts its slice; after a cluster barrier every CTA reads the 8
+// count arrays through distributed shared memory, so it knows the expert
+// offsets and, per expert, how many pairs of the lower slices precede its own;
+// then it places its slice with the same passes as above.  Slices are in pair
+// order, so the result is the same stable order, bit for bit.
 //
 // Up to 32 pairs (decode batches of a few tokens) take route_sort_small_kernel
 // instead: one warp sorts the keys (expert, pair id) in registers with a
@@ -24,6 +31,8 @@
 // for bit, in about a third of the barrier steps.
 
 #include <climits>
+
+#include <cooperative_groups.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -63,6 +72,46 @@ NVM_DEV int block_exclusive_scan(int v, int* warp_tmp, int& total) {
   return ex;
 }
 
+// Place pairs [lo, hi) in passes of 1024 in pair order: a pair's position is
+// cursor[e] + (pairs of expert e in earlier warps of the pass) + (its rank among
+// its warp's lanes with expert e); cursor advances by the pass's count.  cnt
+// and wc are scratch; the caller has set cursor and synchronised.
+NVM_DEV void place_pairs(const int32_t* __restrict__ ids, int lo, int hi, int E, int* cnt, int* cursor,
+                         uint16_t* wc, int32_t* __restrict__ sorted, int32_t* __restrict__ pair_pos) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int base = lo; base < hi; base += kSortThreads) {
+    for (int i = tid; i < 32 * E; i += kSortThreads) wc[i] = 0;
+    const int p = base + tid;
+    const int v = p < hi ? ids[p] : -1;
+    const bool valid = (unsigned)v < (unsigned)E;
+    const unsigned peers = __match_any_sync(0xffffffffu, valid ? v : -1);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    __syncthreads();
+    if (valid && rank == 0) wc[warp * E + v] = (uint16_t)__popc(peers);
+    __syncthreads();
+    if (tid < E) {
+      int run = 0;
+      for (int w = 0; w < 32; ++w) {
+        const int t = wc[w * E + tid];
+        wc[w * E + tid] = (uint16_t)run;
+        run += t;
+      }
+      cnt[tid] = run;
+    }
+    __syncthreads();
+    if (valid) {
+      const int pos = cursor[v] + wc[warp * E + v] + rank;
+      sorted[pos] = p;
+      pair_pos[p] = pos;
+    } else if (p < hi) {
+      pair_pos[p] = -1;
+    }
+    __syncthreads();
+    if (tid < E) cursor[tid] += cnt[tid];
+    __syncthreads();
+  }
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(kSortThreads)
@@ -73,15 +122,14 @@ __global__ void __launch_bounds__(kSortThreads)
   extern __shared__ int sm[];
   int* cnt = sm;                                            // [E]
   int* cursor = sm + E;                                     // [E]
-  uint16_t* wc = reinterpret_cast<uint16_t*>(sm + 2 * E);   // [E][32]
+  uint16_t* wc = reinterpret_cast<uint16_t*>(sm + 2 * E);   // [32][E]
   __shared__ int tmp[33];
   __shared__ int bad;
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   griddep_wait();  // the previous kernel on the stream (e.g. the last blend) is done
   griddep_launch_dependents();
   for (int i = tid; i < E; i += kSortThreads) cnt[i] = 0;
-  for (int i = tid; i < 32 * E; i += kSortThreads) wc[i] = 0;
   if (tid == 0) bad = 0;
   __syncthreads();
   for (int p = tid; p < P; p += kSortThreads) {
@@ -108,44 +156,76 @@ __global__ void __launch_bounds__(kSortThreads)
   for (int i = nactive + tid; i < E; i += kSortThreads) active[i] = -1;
   for (int i = kept + tid; i < P; i += kSortThreads) sorted[i] = -1;
 
-  int v_next = tid < P ? ids[tid] : -1;
-  for (int base = 0; base < P; base += kSortThreads) {
-    const int p = base + tid;
-    const int v = p < P ? v_next : -1;
-    if (base + kSortThreads + tid < P) v_next = ids[base + kSortThreads + tid];
-    const bool valid = (unsigned)v < (unsigned)E;
-    const unsigned peers = __match_any_sync(0xffffffffu, valid ? v : -1);
-    const int rank = __popc(peers & ((1u << lane) - 1u));
-    if (valid && rank == 0) wc[v * 32 + warp] = (uint16_t)__popc(peers);
-    __syncthreads();
-    // Exclusive scan of each expert's 32 per-warp counts, one warp per expert.
-    for (int e = warp; e < E; e += 32) {
-      const int c = wc[e * 32 + lane];
-      int incl = c;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
-      }
-      wc[e * 32 + lane] = (uint16_t)(incl - c);
-      if (lane == 31) cnt[e] = incl;
-    }
-    __syncthreads();
-    if (valid) {
-      const int pos = cursor[v] + wc[v * 32 + warp] + rank;
-      sorted[pos] = p;
-      pair_pos[p] = pos;
-    } else if (p < P) {
-      pair_pos[p] = -1;
-    }
-    __syncthreads();
-    // The same warp clears its experts' counts and advances their cursors.
-    for (int e = warp; e < E; e += 32) {
-      wc[e * 32 + lane] = 0;
-      if (lane == 0) cursor[e] += cnt[e];
-    }
-    __syncthreads();
+  place_pairs(ids, 0, P, E, cnt, cursor, wc, sorted, pair_pos);
+}
+
+namespace {
+constexpr int kClusterCtas = 8;
+constexpr uint32_t kClusterMinPairs = 4097;
+}  // namespace
+
+__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kSortThreads)
+    route_sort_cluster_kernel(const int32_t* __restrict__ ids, int P, int E, int32_t* __restrict__ offsets,
+                              int32_t* __restrict__ sorted, int32_t* __restrict__ pair_pos,
+                              int32_t* __restrict__ active, int32_t* __restrict__ active_count,
+                              int32_t* __restrict__ status) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  extern __shared__ int sm[];
+  int* cnt = sm;                                            // [E] this slice's counts, then scratch
+  int* cursor = sm + E;                                     // [E]
+  uint16_t* wc = reinterpret_cast<uint16_t*>(sm + 2 * E);   // [32][E]
+  __shared__ int tmp[33];
+  __shared__ int bad;
+
+  const int tid = threadIdx.x;
+  const int r = (int)cluster.block_rank();
+  const int lo = (int)((int64_t)P * r / kClusterCtas), hi = (int)((int64_t)P * (r + 1) / kClusterCtas);
+  griddep_wait();
+  griddep_launch_dependents();
+  for (int i = tid; i < E; i += kSortThreads) cnt[i] = 0;
+  if (tid == 0) bad = 0;
+  __syncthreads();
+  for (int p = lo + tid; p < hi; p += kSortThreads) {
+    const int v = ids[p];
+    if ((unsigned)v < (unsigned)E) atomicAdd(&cnt[v], 1);
+    else bad = 1;
   }
+  cluster.sync();  // every slice's counts are complete
+
+  // Expert e: pairs in all slices (total) and in the slices before this one.
+  int total = 0, before = 0, any_bad = 0;
+  if (tid < E) {
+    for (int q = 0; q < kClusterCtas; ++q) {
+      const int c = *cluster.map_shared_rank(cnt + tid, q);
+      total += c;
+      if (q < r) before += c;
+    }
+  }
+  if (tid == 0)
+    for (int q = 0; q < kClusterCtas; ++q) any_bad |= *cluster.map_shared_rank(&bad, q);
+  cluster.sync();  // no CTA reuses cnt or bad before all have read them
+
+  int kept = 0, nactive = 0;
+  const int off = block_exclusive_scan(total, tmp, kept);
+  const int arank = block_exclusive_scan(total > 0 ? 1 : 0, tmp, nactive);
+  if (tid < E) cursor[tid] = off + before;
+  if (r == 0) {
+    if (tid < E) {
+      offsets[tid] = off;
+      if (total > 0) active[arank] = tid;
+    }
+    if (tid == 0) {
+      offsets[E] = kept;
+      *active_count = nactive;
+      if (status != nullptr) *status = any_bad;
+    }
+    for (int i = nactive + tid; i < E; i += kSortThreads) active[i] = -1;
+  }
+  // Positions past the kept pairs hold -1 (split over the CTAs).
+  for (int i = kept + (int)(r * kSortThreads) + tid; i < P; i += kClusterCtas * kSortThreads) sorted[i] = -1;
+  __syncthreads();
+  place_pairs(ids, lo, hi, E, cnt, cursor, wc, sorted, pair_pos);
 }
 
 namespace {
@@ -233,6 +313,13 @@ cudaError_t launch_route_sort(const int32_t* topk_ids, uint32_t num_pairs, uint3
                       (int)num_pairs, (int)num_experts, expert_offsets, sorted_pair_ids, pair_pos,
                       active_experts, active_count, status);
   const int smem = (int)num_experts * (2 * 4 + 32 * 2);
+  if (num_pairs >= kClusterMinPairs) {
+    cudaError_t err = ensure_dynamic_smem(reinterpret_cast<const void*>(route_sort_cluster_kernel), smem);
+    if (err != cudaSuccess) return err;
+    return launch_pdl(route_sort_cluster_kernel, dim3(kClusterCtas), dim3(kSortThreads), smem, stream,
+                      topk_ids, (int)num_pairs, (int)num_experts, expert_offsets, sorted_pair_ids, pair_pos,
+                      active_experts, active_count, status);
+  }
   cudaError_t err = ensure_dynamic_smem(reinterpret_cast<const void*>(route_sort_kernel), smem);
   if (err != cudaSuccess) return err;
   return launch_pdl(route_sort_kernel, dim3(1), dim3(kSortThreads), smem, stream, topk_ids,
