@@ -11,6 +11,13 @@
  *
  * plus the load-time twin builder nvfp4_moe_transpose_u8.
  *
+ * Launch order.  The kernels use programmatic dependent launch: each may start
+ * while the previous kernel on the stream is still running and waits for it
+ * before reading what it writes.  Step 3 reads step 1's outputs before that
+ * wait (to start fetching its weights early), which is safe because step 2
+ * runs in between: run the four steps in this order, with no step left out,
+ * on one stream (other kernels may be interleaved).
+ *
  * Sources.  The operations and layouts are those of the rustdoc source pages of
  * the "metrale" project:
  *   - metrale_model_layers/layers/ops/nvfp4_moe_grouped.rs: module doc (rows

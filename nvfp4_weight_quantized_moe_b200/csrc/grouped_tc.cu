@@ -167,6 +167,50 @@ __global__ void __launch_bounds__(256)
   if (lane == 0) xexp[row] = exp2i(e);
 }
 
+// Single-pass form of pack_act for rows that fit in registers (NV 16-byte
+// pieces per lane): the row is read once, its max taken, then converted from
+// registers.  (For x the register form needs so many registers at K = 4096
+// that it runs one CTA per SM and is slower than the two-pass kernel.)
+template <int NV>
+__global__ void __launch_bounds__(256)
+    pack_act_reg_kernel(const float* __restrict__ act, int P, int K, const int32_t* __restrict__ kept_rows,
+                        uint16_t* __restrict__ hi, uint16_t* __restrict__ lo, float* __restrict__ aexp) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= P || row >= *kept_rows) return;
+  const float4* src = reinterpret_cast<const float4*>(act + (size_t)row * K);
+  const int n16 = K / 4;
+  float4 r[NV];
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int idx = lane + 32 * i;
+    r[i] = idx < n16 ? src[idx] : make_float4(0.f, 0.f, 0.f, 0.f);
+    m = fmaxf(fmaxf(fmaxf(m, fabsf(r[i].x)), fabsf(r[i].y)), fmaxf(fabsf(r[i].z), fabsf(r[i].w)));
+  }
+  const int e = f16_range_exponent(warp_max(m));
+  const float mul = exp2i(-e);
+  uint2* dh = reinterpret_cast<uint2*>(hi + (size_t)row * K);
+  uint2* dl = reinterpret_cast<uint2*>(lo + (size_t)row * K);
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int idx = lane + 32 * i;
+    if (idx < n16) {
+      const float sv[4] = {r[i].x * mul, r[i].y * mul, r[i].z * mul, r[i].w * mul};
+      float h[4], l[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        h[j] = __half2float(__float2half_rn(sv[j]));
+        l[j] = sv[j] - h[j];
+      }
+      dh[idx] = make_uint2(pack_f16x2(h[0], h[1]), pack_f16x2(h[2], h[3]));
+      dl[idx] = make_uint2(pack_f16x2(l[0], l[1]), pack_f16x2(l[2], l[3]));
+    }
+  }
+  if (lane == 0) aexp[row] = exp2i(e);
+}
+
 // One warp per sorted row r < offsets[E]: hi/lo f16 planes of act[r] * 2^-e_r.
 __global__ void __launch_bounds__(256) pack_act_kernel(const float* __restrict__ act, int P, int K,
                                                        const int32_t* __restrict__ kept_rows,
@@ -755,9 +799,15 @@ cudaError_t launch_tc(int mode, int nt, const GroupedArgs& g, void* workspace, u
     return launch_tc_impl<kModeGateUp, 128>(a, b0, b1, cap, stream);
   }
   // Rows past offsets[E] (dropped pairs) are not packed: offsets[E] bounds the grid's work.
-  err = launch_pdl(pack_act_kernel, dim3((unsigned)((pairs + 7) / 8)), dim3(256), 0, stream,
-                   static_cast<const float*>(g.src), (int)pairs, (int)g.K, g.offsets + g.num_experts, w.act_hi,
-                   w.act_lo, w.aexp);
+  {
+    // Rows of up to 2048 floats go through registers in one pass.
+    const uint32_t pieces = (g.K / 4 + 31) / 32;
+    auto kern = pieces <= 8 ? pack_act_reg_kernel<8>
+                : pieces <= 16 ? pack_act_reg_kernel<16> : pack_act_kernel;
+    err = launch_pdl(kern, dim3((unsigned)((pairs + 7) / 8)), dim3(256), 0, stream,
+                     static_cast<const float*>(g.src), (int)pairs, (int)g.K, g.offsets + g.num_experts,
+                     w.act_hi, w.act_lo, w.aexp);
+  }
   if (err != cudaSuccess) return err;
   err = launch_pdl(build_weight_maps_kernel, dim3(g.num_experts), dim3(128), 0, stream, t_nib, t_scale,
                    g.packed0, g.scale0, g.packed0, g.scale0, 2, w.maps_down);
