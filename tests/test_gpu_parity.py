@@ -208,6 +208,10 @@ SMALL = {
     # skewed, more experts than pairs
     "zipf": MoEConfig("zipf", hidden=1024, inter=512, experts=64, topk=4, tokens=6,
                       router="zipf", seed=23),
+    # long K: a 2-way K split runs 5 chunks per warp (past the pre-converted
+    # activation buffers), a 4-way split 3 (within them)
+    "longk": MoEConfig("longk", hidden=2560, inter=2560, experts=6, topk=2, tokens=3,
+                       router="uniform", seed=24),
 }
 
 
