@@ -284,6 +284,44 @@ NVFP4_MOE_API int nvfp4_moe_blend(const float* y, const float* topk_weights, con
                     uint32_t hidden, cudaStream_t stream);
 
 /*
+ * The four steps of one layer in one call: nvfp4_moe_route_sort,
+ * nvfp4_moe_gate_up_silu(_ws), nvfp4_moe_down(_ws) and nvfp4_moe_blend, launched
+ * in that order on `stream` with cap = nvfp4_moe_active_cap(num_experts, P).
+ * The results are those of the four calls (bit for bit); one call saves the
+ * host three trips through the ABI.  Buffers (all DEVICE, caller-owned):
+ *
+ *   expert_offsets i32 [num_experts + 1]    sorted_pair_ids i32 [P]
+ *   pair_pos       i32 [P]                  active_experts  i32 [num_experts]
+ *   active_count   i32 [1]                  status          i32 [1] or NULL
+ *   act            f32 [P, inter]           y               f32 [P, hidden]
+ *   out_f32        f32 [num_tokens, hidden] out_bf16        bf16 bits [num_tokens, hidden] or NULL
+ *
+ * workspace / workspace_bytes as for the _ws calls, or NULL / 0 for the decode
+ * path only.  Returns the first non-zero status of the four steps (the later
+ * steps are then not launched).
+ */
+typedef struct {
+  int32_t* expert_offsets;
+  int32_t* sorted_pair_ids;
+  int32_t* pair_pos;
+  int32_t* active_experts;
+  int32_t* active_count;
+  int32_t* status;
+  float* act;
+  float* y;
+  float* out_f32;
+  uint16_t* out_bf16;
+} nvfp4_moe_buffers;
+
+NVFP4_MOE_API int nvfp4_moe_forward(const uint16_t* x, const int32_t* topk_ids,
+                                    const float* topk_weights, nvfp4_expert_tables gate,
+                                    nvfp4_expert_tables up, nvfp4_expert_tables down,
+                                    const nvfp4_moe_buffers* buffers, uint32_t num_tokens,
+                                    uint32_t topk, uint32_t num_experts, uint32_t hidden,
+                                    uint32_t inter, const nvfp4_moe_launch_opts* opts,
+                                    void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Load-time twin builder: byte transpose [rows, cols] -> [cols, rows]
  * (transpose_u8, used by transpose_for_gemm_gs in transpose.rs, whose host
  * fallback loop t[j*rows + i] = b[i*cols + j] defines it).  src and dst must

@@ -42,6 +42,13 @@ class LaunchOpts(ctypes.Structure):
                 ("depth", ctypes.c_int32)]
 
 
+class Buffers(ctypes.Structure):
+    """nvfp4_moe_buffers: the device outputs and intermediates of one forward."""
+    _fields_ = [("expert_offsets", c_void_p), ("sorted_pair_ids", c_void_p), ("pair_pos", c_void_p),
+                ("active_experts", c_void_p), ("active_count", c_void_p), ("status", c_void_p),
+                ("act", c_void_p), ("y", c_void_p), ("out_f32", c_void_p), ("out_bf16", c_void_p)]
+
+
 PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
 
 _sig = {
@@ -71,6 +78,10 @@ _sig = {
     "nvfp4_moe_gate_up_silu_noalloc": (c_int, [c_void_p, ExpertTables, ExpertTables, c_void_p,
                                                c_void_p, c_void_p, c_void_p, c_void_p, c_u32,
                                                c_u32, c_u32, c_u32, c_u32, c_u32, c_void_p]),
+    "nvfp4_moe_forward": (c_int, [c_void_p, c_void_p, c_void_p, ExpertTables, ExpertTables,
+                                  ExpertTables, ctypes.POINTER(Buffers), c_u32, c_u32, c_u32, c_u32,
+                                  c_u32, ctypes.POINTER(LaunchOpts), c_void_p, ctypes.c_size_t,
+                                  c_void_p]),
     "nvfp4_moe_workspace_bytes": (ctypes.c_size_t, [c_u32, c_u32, c_u32, c_u32]),
     "nvfp4_moe_device_error": (c_int, [c_int]),
     "nvfp4_moe_active_cap": (c_u32, [c_u32, c_u32]),
@@ -228,3 +239,18 @@ def down_ws(act, down_w: ExpertTables, y, expert_offsets, active_experts, active
         _ptr(active_count, torch.int32, "active_count"),
         n_hidden, k_inter, cap, num_tokens, topk, num_experts,
         _opts(path, split, tiles, depth), wp, wn, _stream(stream)))
+
+
+def forward(x, topk_ids, topk_weights, gate: ExpertTables, up: ExpertTables, down: ExpertTables,
+            buffers: Buffers, num_experts, hidden, inter, workspace=None, path=0, split=0, tiles=0,
+            depth=0, stream=None) -> None:
+    """nvfp4_moe_forward: the four steps of one layer in one library call.
+    ``buffers`` is a :class:`Buffers` of device pointers (see ``MoEBuffers.c_buffers``)."""
+    if x.dtype not in (torch.bfloat16, torch.uint16, torch.int16):
+        raise TypeError("x: expected bf16 (or its uint16 bits)")
+    m, k = topk_ids.shape
+    wp, wn = (None, 0) if workspace is None else _ws(workspace)
+    _check("nvfp4_moe_forward", _lib.nvfp4_moe_forward(
+        _ptr(x, None, "x"), _ptr(topk_ids, torch.int32, "topk_ids"),
+        _ptr(topk_weights, torch.float32, "topk_weights"), gate, up, down, ctypes.byref(buffers),
+        m, k, num_experts, hidden, inter, _opts(path, split, tiles, depth), wp, wn, _stream(stream)))

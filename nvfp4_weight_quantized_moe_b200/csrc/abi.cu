@@ -344,6 +344,41 @@ int nvfp4_moe_blend(const float* y, const float* topk_weights, const int32_t* pa
                                 hidden, stream));
 }
 
+int nvfp4_moe_forward(const uint16_t* x, const int32_t* topk_ids, const float* topk_weights,
+                      nvfp4_expert_tables gate, nvfp4_expert_tables up, nvfp4_expert_tables down,
+                      const nvfp4_moe_buffers* b, uint32_t num_tokens, uint32_t topk,
+                      uint32_t num_experts, uint32_t hidden, uint32_t inter,
+                      const nvfp4_moe_launch_opts* opts, void* workspace, size_t workspace_bytes,
+                      cudaStream_t stream) {
+  if (b == nullptr) return NVFP4_MOE_EINVAL;
+  const uint64_t pairs = (uint64_t)num_tokens * topk;
+  if (pairs > kMaxPairs) return NVFP4_MOE_ESHAPE;
+  const uint32_t cap = nvfp4_moe_active_cap(num_experts, (uint32_t)pairs);
+  int st = nvfp4_moe_route_sort(topk_ids, num_tokens, topk, num_experts, b->expert_offsets,
+                                b->sorted_pair_ids, b->pair_pos, b->active_experts, b->active_count,
+                                b->status, stream);
+  if (st != NVFP4_MOE_OK) return st;
+  if (workspace != nullptr) {
+    st = nvfp4_moe_gate_up_silu_ws(x, gate, up, b->act, b->expert_offsets, b->sorted_pair_ids,
+                                   b->active_experts, b->active_count, inter, hidden, cap, num_tokens,
+                                   topk, num_experts, opts, workspace, workspace_bytes, stream);
+    if (st != NVFP4_MOE_OK) return st;
+    st = nvfp4_moe_down_ws(b->act, down, b->y, b->expert_offsets, b->active_experts, b->active_count,
+                           hidden, inter, cap, num_tokens, topk, num_experts, opts, workspace,
+                           workspace_bytes, stream);
+  } else {
+    st = nvfp4_moe_gate_up_silu_ex(x, gate, up, b->act, b->expert_offsets, b->sorted_pair_ids,
+                                   b->active_experts, b->active_count, inter, hidden, cap, num_tokens,
+                                   topk, opts, stream);
+    if (st != NVFP4_MOE_OK) return st;
+    st = nvfp4_moe_down_ex(b->act, down, b->y, b->expert_offsets, b->active_experts, b->active_count,
+                           hidden, inter, cap, num_tokens, topk, opts, stream);
+  }
+  if (st != NVFP4_MOE_OK) return st;
+  return nvfp4_moe_blend(b->y, topk_weights, b->pair_pos, b->out_f32, b->out_bf16, num_tokens, topk,
+                         hidden, stream);
+}
+
 int nvfp4_moe_transpose_u8(const uint8_t* src, uint8_t* dst, uint32_t rows, uint32_t cols,
                            cudaStream_t stream) {
   if (rows == 0 || cols == 0) return NVFP4_MOE_OK;

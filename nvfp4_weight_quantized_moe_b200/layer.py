@@ -69,6 +69,12 @@ class MoEBuffers:
         self.out = torch.empty(max(num_tokens, 1), hidden, **f32)
         self.out_bf16 = (torch.empty(max(num_tokens, 1), hidden, dtype=torch.bfloat16, device=device)
                          if out_bf16 else None)
+        # The same pointers as one nvfp4_moe_buffers, for the one-call forward.
+        self.c_buffers = B.Buffers(
+            self.expert_offsets.data_ptr(), self.sorted_pair_ids.data_ptr(), self.pair_pos.data_ptr(),
+            self.active_experts.data_ptr(), self.active_count.data_ptr(), self.status.data_ptr(),
+            self.act.data_ptr(), self.y.data_ptr(), self.out.data_ptr(),
+            self.out_bf16.data_ptr() if self.out_bf16 is not None else None)
 
 
 class NVFP4MoE:
@@ -96,8 +102,10 @@ class NVFP4MoE:
     def forward(self, x: torch.Tensor, topk_ids: torch.Tensor, topk_weights: torch.Tensor,
                 bufs: Optional[MoEBuffers] = None, path: int = 0, split: int = 0,
                 tiles: int = 0, depth: int = 0, workspace: Optional[torch.Tensor] = None,
-                stream=None) -> MoEBuffers:
+                stream=None, steps: bool = False) -> MoEBuffers:
         """Run the four steps on ``stream``; results land in ``bufs`` (returned).
+        One library call (nvfp4_moe_forward) by default; ``steps=True`` makes the
+        four single-step calls instead (same kernels, same results).
 
         path / split / tiles / depth are the launch options of the two
         projections (0 = chosen from the shape); see nvfp4_moe_launch_opts.
@@ -106,6 +114,13 @@ class NVFP4MoE:
         m = x.shape[0]
         if bufs is None:
             bufs = self.buffers(m)
+        if m > bufs.num_tokens:
+            raise ValueError("buffers were sized for fewer tokens")
+        if not steps:
+            B.forward(x, topk_ids, topk_weights, self.gate.tables, self.up.tables, self.down.tables,
+                      bufs.c_buffers, self.num_experts, self.hidden, self.inter, workspace=workspace,
+                      path=path, split=split, tiles=tiles, depth=depth, stream=stream)
+            return bufs
         p = m * self.topk
         cap = B.active_cap(self.num_experts, p)
         B.route_sort(topk_ids, self.num_experts, bufs.expert_offsets, bufs.sorted_pair_ids,

@@ -155,6 +155,24 @@ def test_route_sort_out_of_range_ids_and_max_experts():
         assert int(bufs.status.item()) == 1
 
 
+@pytest.mark.parametrize("name,ws", [("tiny", False), ("zipf", False), ("zipf", True), ("hot", True)])
+def test_one_call_forward_equals_the_four_steps(name, ws):
+    # nvfp4_moe_forward launches the same kernels as the four single-step calls:
+    # every output is bit-identical.
+    _need_gpu()
+    prob = make_problem(SMALL[name])
+    layer, one = _gpu_forward(prob, ws=ws)
+    _, four = _gpu_forward(prob, layer=layer, ws=ws, steps=True)
+    def bits(t):  # bit patterns, so that NaN rows left untouched compare equal too
+        return t.view(torch.int16) if t.dtype == torch.bfloat16 else (
+            t.view(torch.int32) if t.dtype == torch.float32 else t)
+
+    for f in ("expert_offsets", "sorted_pair_ids", "pair_pos", "active_experts", "active_count", "act",
+              "y", "out", "out_bf16"):
+        assert torch.equal(bits(getattr(one, f)), bits(getattr(four, f))), f
+    _check_full(prob, one)
+
+
 def test_route_sort_small_batches_bit_exact():
     # Up to 32 pairs take the single-warp sort: cover every P in 1..33 (the
     # boundary on both sides), out-of-range ids, one expert, and 1024 experts.
