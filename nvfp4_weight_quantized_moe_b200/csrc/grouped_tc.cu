@@ -99,12 +99,12 @@ struct TcCfg {
   static constexpr int OFF_W = 0;
   static constexpr int OFF_B = WS * kWSlotBytes;
   static constexpr int OFF_BAR = OFF_B + SB * B_SLOT_BYTES;
-  // MMA completion is committed once per CG stages: a commit costs
-  // tensor-pipe time, so 128-token tiles commit every other stage; 16-token
-  // tiles, whose stages are short, commit every stage to free ring slots
-  // sooner (measured 3% faster than every other stage).  mma_done has SB / CG
-  // entries.
-  static constexpr int CG = NT <= 16 ? 1 : 2;
+  // MMA completion is committed once per CG stages.  Any tcgen05.commit in the
+  // MMA stream costs tensor-pipe time (measured: 64 -> 77 cycles per
+  // 128x128x16 MMA), but that cost does not grow with the commit rate, and a
+  // commit per stage frees ring slots sooner: measured 2-3 % faster than one
+  // per two stages at both tile sizes.  mma_done has SB / CG entries.
+  static constexpr int CG = 1;
   static constexpr int NMD = SB / CG;
   // full_w[WS], empty_w[WS], full_b[SB], mma_done[NMD], full_a[SA], done, d_free
   static constexpr int NBAR = 2 * WS + SB + NMD + SA + 2;
