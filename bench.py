@@ -49,8 +49,8 @@ DEFAULT_STEPS = {"tiny": 20000, "decode_m1": 20000, "decode_m32": 5000, "decode_
 # whenever that kernel changes.
 NCU_TRAFFIC_BYTES = {
     ("decode_m1", "mma.sync"): 28357888,      # 28.36 MB read, 0 written (routed gate+up: 28.31 MB)
-    ("decode_m32", "tcgen05"): 334348288,     # 330.17 MB read, 4.18 MB written
-    ("prefill_m8192", "tcgen05"): 4236745000,  # 3.826 GB read, 0.411 GB written (4 token passes)
+    ("decode_m32", "tcgen05"): 335457536,     # 329.50 MB read, 5.96 MB written
+    ("prefill_m8192", "tcgen05"): 4249585000,  # 3.838 GB read, 0.411 GB written (4 token passes)
 }
 
 
