@@ -10,6 +10,7 @@ from ._binding import (  # noqa: F401
     PATH_AUTO,
     PATH_DECODE,
     PATH_PREFILL,
+    Buffers,
     ExpertTables,
     LaunchOpts,
     NVFP4MoEError,
@@ -19,6 +20,7 @@ from ._binding import (  # noqa: F401
     down,
     down_ws,
     exported_symbols,
+    forward,
     gate_up_silu,
     gate_up_silu_ws,
     route_sort,
