@@ -155,6 +155,23 @@ def test_route_sort_out_of_range_ids_and_max_experts():
         assert int(bufs.status.item()) == 1
 
 
+def test_route_sort_large_batch_bit_exact():
+    # 2^22 routed pairs over 1024 experts (the cluster sort: 512 Ki pairs per CTA),
+    # with out-of-range ids, against the oracle's stable sort.
+    _need_gpu()
+    import nvfp4_weight_quantized_moe_b200 as nvm
+    rng = np.random.default_rng(12)
+    m, k, e = 1 << 19, 8, 1024
+    ids = rng.integers(-1, e + 1, (m, k)).astype(np.int32)
+    bufs = nvm.MoEBuffers(m, k, e, 4, 4, "cuda")
+    nvm.route_sort(torch.from_numpy(ids).cuda(), e, bufs.expert_offsets, bufs.sorted_pair_ids,
+                   bufs.pair_pos, bufs.active_experts, bufs.active_count, bufs.status)
+    torch.cuda.synchronize()
+    rs = orc.route_sort(ids, e)
+    _check_sort(bufs, rs, e, m * k)
+    assert int(bufs.status.item()) == 1
+
+
 @pytest.mark.parametrize("name,ws", [("tiny", False), ("zipf", False), ("zipf", True), ("hot", True)])
 def test_one_call_forward_equals_the_four_steps(name, ws):
     # nvfp4_moe_forward launches the same kernels as the four single-step calls:
