@@ -26,11 +26,14 @@
 //     the MMA's A operand, in a ring of SA stages.
 //   * Warp 8 (one thread) issues tcgen05.mma.kind::f16 (A = 128 x 16 from
 //     TMEM, B = NT x 16 from shared memory, D = FP32 accumulators in TMEM) and
-//     tcgen05.commit to the rings' "empty" mbarriers.
-//   * Epilogue (warps 0..7, per group): tcgen05.ld of the accumulators;
-//     weight_scale_2 and the activation row's power-of-two scale applied in
-//     FP32; SiLU(gate)*up in FP32 for gate+up; coalesced FP32 stores by sorted
-//     position.  The loaders run ahead into the next group meanwhile.
+//     one tcgen05.commit per stage to a completion ring that frees both the
+//     stage's token slot and its A slot.
+//   * Epilogue (warps 0..7, per group): once the next group's first A stages
+//     are in TMEM, tcgen05.ld of the accumulators; weight_scale_2 and the
+//     activation row's power-of-two scale applied in FP32; for gate+up,
+//     SiLU(gate)*up in FP32 into registers and the accumulators handed back to
+//     the MMA before the stores; coalesced FP32 stores by sorted position.  The
+//     loaders run ahead into the next group meanwhile.
 // The roles synchronise through mbarriers only.  Every wait is bounded: on
 // timeout the kernel sets the device error word, skips its remaining waits,
 // lets its TMA loads in flight land and still frees its TMEM.
