@@ -28,6 +28,10 @@ Sources (rustdoc source pages of the "metrale" project; cited by page and item):
   the E4M3 variant as the finite "FN" one (max 448, no infinities).
 * metrale_model_layers/weight_map/expert.rs, ``ExpertWeight::null``: a NULL
   expert is skipped by the MoE kernels.
+* nvfp4_moe_grouped.rs, docs of the two projection launchers: the shared
+  expert runs in the same gate+up and down launches as the routed experts,
+  over every token, one row per token, with its own weights; its SiLU product
+  and down output (``sh_act``, ``sh_down_out``) are laid out by token.
 
 Readings where the pages are silent (each also listed in the design notes):
 
@@ -41,7 +45,10 @@ Readings where the pages are silent (each also listed in the design notes):
 * sort ties are broken by pair id (pair p = token * k + slot), so the sort is
   stable and unique; ``active_experts`` is ascending and padded with -1;
   an expert id outside [0, E) drops its pair (pair_pos = -1, contributes 0);
-* a NULL expert's rows of ``act`` and ``y`` are zero.
+* a NULL expert's rows of ``act`` and ``y`` are zero;
+* the shared expert has the routed experts' shapes (the fused launches take
+  one width pair for both) and its down output joins the token's sum with a
+  per-token weight, 1 unless the caller gives one.
 
 Parity pins for every function live in ``tests/test_oracle_pins.py``.
 """
@@ -69,6 +76,9 @@ __all__ = [
     "moe_forward",
     "moe_forward_tokens",
     "transpose_u8",
+    "shared_expert",
+    "moe_forward_shared",
+    "append_shared_routing",
     "RouteSort",
 ]
 
@@ -349,6 +359,71 @@ def moe_forward_tokens(x_bf16, topk_ids, topk_weights, num_experts, gate_fn, up_
             h = silu(wg @ x[t]) * (wu @ x[t])
             out[i] += w[t, s] * (wd @ h)
     return out
+
+
+# --------------------------------------------------------------------------- #
+# Shared expert
+# --------------------------------------------------------------------------- #
+
+Weight = Tuple[np.ndarray, np.ndarray, float]
+
+
+def shared_expert(x_bf16, gate: Weight, up: Weight, down: Weight) -> Tuple[np.ndarray, np.ndarray]:
+    """(sh_act [M, I], sh_out [M, H]) of the shared expert, float64, rows by token.
+
+    The launcher docs of nvfp4_moe_grouped.rs give the shared expert one row per
+    token in both projections: sh_act[t] = SiLU(Wg x_t) * (Wu x_t) and
+    sh_out[t] = Wd sh_act[t].
+    """
+    x = bf16_bits_to_f64(x_bf16)
+    wg, wu, wd = (dequantize_nvfp4(*w) for w in (gate, up, down))
+    h = silu(x @ wg.T) * (x @ wu.T)
+    return h, h @ wd.T
+
+
+def moe_forward_shared(x_bf16, topk_ids, topk_weights, num_experts, gate_fn, up_fn, down_fn,
+                       hidden: int, inter: int, shared: Tuple[Weight, Weight, Weight],
+                       shared_weights: Optional[np.ndarray] = None) -> Dict[str, object]:
+    """The routed forward plus the shared expert: out[t] += c_t * sh_out[t].
+
+    c_t is ``shared_weights[t]``, or 1 for every token when it is None.
+    """
+    res = moe_forward(x_bf16, topk_ids, topk_weights, num_experts, gate_fn, up_fn, down_fn,
+                      hidden, inter)
+    sh_act, sh_out = shared_expert(x_bf16, *shared)
+    m = sh_out.shape[0]
+    c = (np.ones(m) if shared_weights is None
+         else np.asarray(shared_weights, dtype=np.float64).reshape(m))
+    res["sh_act"] = sh_act
+    res["sh_out"] = sh_out
+    res["out"] = res["out"] + c[:, None] * sh_out
+    return res
+
+
+def append_shared_routing(topk_ids, topk_weights, num_experts: int, shared_rows: int,
+                          shared_weights: Optional[np.ndarray] = None
+                          ) -> Tuple[np.ndarray, np.ndarray]:
+    """Routing [M, k+1] that sends every token to the shared expert as one more slot.
+
+    Slot k of token t names expert num_experts + t // shared_rows: the shared
+    expert is listed once per block of ``shared_rows`` tokens, each listing a
+    table entry that holds the shared weights, so the grouped launches give it
+    as many row groups as it has token blocks.  Its weight is
+    ``shared_weights[t]`` (1 when None).  Slots 0..k-1 are copied unchanged.
+    """
+    ids = np.asarray(topk_ids, dtype=np.int32)
+    w = np.asarray(topk_weights, dtype=np.float32)
+    m, k = ids.shape
+    if shared_rows < 1:
+        raise ValueError("shared_rows must be >= 1")
+    ids_out = np.empty((m, k + 1), dtype=np.int32)
+    w_out = np.empty((m, k + 1), dtype=np.float32)
+    for t in range(m):
+        ids_out[t, :k] = ids[t]
+        w_out[t, :k] = w[t]
+        ids_out[t, k] = num_experts + t // shared_rows
+        w_out[t, k] = 1.0 if shared_weights is None else np.float32(shared_weights[t])
+    return ids_out, w_out
 
 
 # --------------------------------------------------------------------------- #

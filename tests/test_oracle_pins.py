@@ -338,6 +338,114 @@ def test_down_is_linear_in_scale2():
 
 
 # --------------------------------------------------------------------------- #
+# Shared expert
+# --------------------------------------------------------------------------- #
+
+def _shared(prob):
+    return tuple(prob.shared_weight(m) for m in (MATRIX_GATE, MATRIX_UP, MATRIX_DOWN))
+
+
+def test_shared_expert_all_ones_closed_form():
+    # Every weight 1.0 (E2M1 code 2 in both nibbles, E4M3 scale 0x38 = 1,
+    # s2 = 1): g = u = S = sum_k x_k, every act entry is SiLU(S) * S and every
+    # output entry I * SiLU(S) * S.
+    h, i = 64, 32
+    ones = lambda n, k: (np.full((n, k // 2), 0x22, np.uint8), np.full((n, k // 16), 0x38, np.uint8),
+                         np.float32(1.0))
+    x = np.array([[0x3F80] * h, [0xBF00] * h, [0x3E80] * (h // 2) + [0xC000] * (h // 2)],
+                 dtype=np.uint16)  # 1, -0.5, (0.25 | -2)
+    sums = np.array([h * 1.0, h * -0.5, h // 2 * 0.25 + h // 2 * -2.0])
+    sh_act, sh_out = orc.shared_expert(x, ones(i, h), ones(i, h), ones(h, i))
+    expect_h = sums / (1.0 + np.exp(-sums)) * sums
+    np.testing.assert_allclose(sh_act, np.repeat(expect_h[:, None], i, axis=1), rtol=1e-15)
+    np.testing.assert_allclose(sh_out, np.repeat(i * expect_h[:, None], h, axis=1), rtol=1e-14)
+
+
+def test_shared_expert_equals_a_routed_expert_with_its_weights():
+    # Give routed expert 2 the shared weights and route every token to it alone
+    # with weight 1: the per-token routed forward must reproduce the shared
+    # expert's output (a gate/up swap or a transposed operand breaks this).
+    prob = make_problem(_tiny_cfg(tokens=7, experts=4, topk=1, hidden=64, inter=48, seed=21))
+    cfg = prob.cfg
+    shared = _shared(prob)
+    fns = [lambda e, m=m: shared[m] if e == 2 else prob.expert_weight(m, e)
+           for m in (MATRIX_GATE, MATRIX_UP, MATRIX_DOWN)]
+    ids = np.full((cfg.tokens, 1), 2, dtype=np.int32)
+    w = np.ones((cfg.tokens, 1), dtype=np.float32)
+    routed = orc.moe_forward_tokens(prob.x_bf16, ids, w, cfg.experts, *fns,
+                                    tokens=range(cfg.tokens), hidden=cfg.hidden)
+    _, sh_out = orc.shared_expert(prob.x_bf16, *shared)
+    np.testing.assert_allclose(sh_out, routed, rtol=1e-12, atol=1e-12)
+
+
+def test_forward_with_shared_adds_the_weighted_shared_output():
+    prob = make_problem(_tiny_cfg(tokens=6, experts=4, topk=2, hidden=64, inter=32, seed=22))
+    cfg = prob.cfg
+    fns = [lambda e, m=m: prob.expert_weight(m, e) for m in (MATRIX_GATE, MATRIX_UP, MATRIX_DOWN)]
+    c = np.random.default_rng(4).random(cfg.tokens)
+    base = orc.moe_forward_tokens(prob.x_bf16, prob.topk_ids, prob.topk_weights, cfg.experts,
+                                  *fns, tokens=range(cfg.tokens), hidden=cfg.hidden)
+    res1 = orc.moe_forward_shared(prob.x_bf16, prob.topk_ids, prob.topk_weights, cfg.experts,
+                                  *fns, hidden=cfg.hidden, inter=cfg.inter, shared=_shared(prob))
+    res_c = orc.moe_forward_shared(prob.x_bf16, prob.topk_ids, prob.topk_weights, cfg.experts,
+                                   *fns, hidden=cfg.hidden, inter=cfg.inter, shared=_shared(prob),
+                                   shared_weights=c)
+    sh = res1["out"] - base
+    np.testing.assert_allclose(res_c["out"], base + c[:, None] * sh, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(sh, res1["sh_out"], rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("m,k,e,rows", [(1, 2, 8, 1), (7, 3, 5, 2), (33, 8, 128, 16), (40, 1, 3, 64)])
+def test_append_shared_routing_layout(m, k, e, rows):
+    rng = np.random.default_rng(m + k + e)
+    ids = rng.integers(0, e, (m, k)).astype(np.int32)
+    w = rng.random((m, k)).astype(np.float32)
+    sw = rng.random(m).astype(np.float32)
+    ids2, w2 = orc.append_shared_routing(ids, w, e, rows, sw)
+    assert ids2.shape == (m, k + 1) and w2.shape == (m, k + 1)
+    np.testing.assert_array_equal(ids2[:, :k], ids)
+    np.testing.assert_array_equal(w2[:, :k], w)
+    np.testing.assert_array_equal(w2[:, k], sw)
+    slots = -(-m // rows)
+    for t in range(m):
+        assert ids2[t, k] == e + t // rows
+    assert ids2[:, k].max() == e + slots - 1
+    _, w1 = orc.append_shared_routing(ids, w, e, rows)
+    assert np.all(w1[:, k] == 1.0)
+    # Grouped by expert, the shared rows come last, contiguous and in token order.
+    rs = orc.route_sort(ids2, e + slots)
+    lo = int(rs.expert_offsets[e])
+    assert int(rs.expert_offsets[e + slots]) == lo + m == m * (k + 1)
+    np.testing.assert_array_equal(rs.sorted_pair_ids[lo:lo + m] // (k + 1), np.arange(m))
+    np.testing.assert_array_equal(rs.sorted_pair_ids[lo:lo + m] % (k + 1), np.full(m, k))
+
+
+def test_shared_expert_as_extra_slots_equals_the_plain_definition():
+    # The grouped forward over the appended routing, whose extra table entries
+    # all hold the shared weights, reaches the plain definition, and its shared
+    # rows are sh_act / sh_out in token order.
+    prob = make_problem(_tiny_cfg(tokens=9, experts=5, topk=2, hidden=64, inter=48, seed=23))
+    cfg = prob.cfg
+    shared = _shared(prob)
+    sw = np.random.default_rng(5).random(cfg.tokens).astype(np.float32)
+    rows = 4
+    slots = -(-cfg.tokens // rows)
+    ids2, w2 = orc.append_shared_routing(prob.topk_ids, prob.topk_weights, cfg.experts, rows, sw)
+    fns = [lambda e, m=m: shared[m] if e >= cfg.experts else prob.expert_weight(m, e)
+           for m in (MATRIX_GATE, MATRIX_UP, MATRIX_DOWN)]
+    grouped = orc.moe_forward(prob.x_bf16, ids2, w2, cfg.experts + slots, *fns,
+                              hidden=cfg.hidden, inter=cfg.inter)
+    plain = orc.moe_forward_shared(prob.x_bf16, prob.topk_ids, prob.topk_weights, cfg.experts,
+                                   *fns, hidden=cfg.hidden, inter=cfg.inter, shared=shared,
+                                   shared_weights=sw)
+    np.testing.assert_allclose(grouped["out"], plain["out"], rtol=1e-12, atol=1e-12)
+    lo = int(grouped["sort"].expert_offsets[cfg.experts])
+    np.testing.assert_allclose(grouped["act"][lo:lo + cfg.tokens], plain["sh_act"], rtol=1e-13)
+    np.testing.assert_allclose(grouped["y"][lo:lo + cfg.tokens], plain["sh_out"], rtol=1e-12,
+                               atol=1e-13)
+
+
+# --------------------------------------------------------------------------- #
 # transpose_u8
 # --------------------------------------------------------------------------- #
 
@@ -391,6 +499,17 @@ def test_pins_catch_a_transposed_operand(monkeypatch):
         expect = orc.silu(wg[:, j[t]]) * wu[:, j[t]]
         bad += int(not np.array_equal(res["act"][rs.pair_pos[t]], expect))
     assert bad > 0
+
+
+def test_pins_catch_swapped_gate_and_up_in_the_shared_expert(monkeypatch):
+    real = orc.shared_expert
+
+    def swapped(x, gate, up, down):
+        return real(x, up, gate, down)
+
+    monkeypatch.setattr(orc, "shared_expert", swapped)
+    with pytest.raises(AssertionError):
+        test_shared_expert_equals_a_routed_expert_with_its_weights()
 
 
 def test_pins_catch_an_unstable_sort(monkeypatch):

@@ -97,6 +97,24 @@ def draw_expert_weight(cfg: MoEConfig, matrix: int, expert: int) -> Tuple[np.nda
     return packed, scale
 
 
+def draw_shared_weight(cfg: MoEConfig, matrix: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Packed bytes and scale codes of the shared expert's projection ``matrix``.
+
+    Same recipe and shapes as a routed expert, from a stream of its own.
+    """
+    n, k = matrix_shape(cfg, matrix)
+    rng = np.random.default_rng([cfg.seed, 4 + matrix, 0])
+    packed = rng.integers(0, 256, size=(n, k // 2), dtype=np.uint8)
+    scale = rng.integers(SCALE_CODE_LO, SCALE_CODE_HI + 1, size=(n, k // 16), dtype=np.uint8)
+    return packed, scale
+
+
+def draw_shared_gate(cfg: MoEConfig) -> np.ndarray:
+    """Per-token weight of the shared expert, f32 [M]: the sigmoid of an N(0, 1) logit."""
+    z = np.random.default_rng([cfg.seed, 0, 3]).standard_normal(cfg.tokens)
+    return (1.0 / (1.0 + np.exp(-z))).astype(np.float32)
+
+
 def draw_routing(cfg: MoEConfig) -> Tuple[np.ndarray, np.ndarray]:
     """topk_ids int32 [M, k] and topk_weights f32 [M, k]."""
     m, e, k = cfg.tokens, cfg.experts, cfg.topk
@@ -157,6 +175,11 @@ class MoEProblem:
             if cache:
                 self._cache[key] = (packed, scale)
         return packed, scale, self.scale2[matrix, expert]
+
+    def shared_weight(self, matrix: int) -> Tuple[np.ndarray, np.ndarray, np.float32]:
+        """(packed, scale, weight_scale_2) of the shared expert's projection."""
+        packed, scale = draw_shared_weight(self.cfg, matrix)
+        return packed, scale, np.float32(1.0 / 448.0)
 
     def stacked_weight(self, matrix: int) -> Tuple[np.ndarray, np.ndarray]:
         """All experts' bytes stacked: packed [E, N, K/2], scale [E, N, K/16].
