@@ -1,11 +1,13 @@
 #!/usr/bin/env python3
 """Throughput of the grouped NVFP4 MoE expert forward on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--shared]
+                    [--impl ours|reference]
 
 One step = one layer forward: route sort, gate+up SiLU, down, blend (the four
 C-ABI calls) over one batch of the workload's synthetic tokens, weights and
-inputs resident in HBM.  The weights rotate over R device replicas (R x the
+inputs resident in HBM.  ``--shared`` adds the workload's shared expert,
+run by every token inside the same launches (one more routing slot).  The weights rotate over R device replicas (R x the
 routed bytes of a step >= 4 x L2), so every step streams its expert weights
 from HBM.  Steps are replayed from CUDA graphs and timed with CUDA events on
 the launching stream; under torchrun (N > 1) each rank runs an independent
@@ -61,6 +63,11 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--op", choices=["layer", "check_scales"], default="layer",
+                    help="layer: the forward; check_scales: the load-time scale check over the "
+                         "workload's three projections")
+    ap.add_argument("--shared", action="store_true",
+                    help="add a shared expert (every token, same launches as the routed experts)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--path", type=int, default=0, help="0 auto, 1 decode, 2 prefill")
@@ -189,12 +196,15 @@ class ClockSampler:
 def _replicate(layer, copies):
     """`copies` extra device copies of a layer's weights (distinct memory, same values)."""
     import nvfp4_weight_quantized_moe_b200 as nvm
+
+    def clone(p):
+        return nvm.NVFP4Projection(p.packed.clone(), p.scale.clone(), p.scale2.clone())
+
     out = [layer]
     for _ in range(copies):
-        projs = []
-        for p in (layer.gate, layer.up, layer.down):
-            projs.append(nvm.NVFP4Projection(p.packed.clone(), p.scale.clone(), p.scale2.clone()))
-        out.append(nvm.NVFP4MoE(*projs, layer.topk))
+        projs = [clone(p) for p in (layer.gate, layer.up, layer.down)]
+        shared = tuple(clone(p) for p in layer.shared) if layer.shared is not None else None
+        out.append(nvm.NVFP4MoE(*projs, layer.topk, shared=shared, shared_rows=layer.shared_rows))
     return out
 
 
@@ -216,7 +226,7 @@ def run_ours(args, rank, world, local):
     dev = torch.device("cuda", local)
     stream = torch.cuda.Stream(device=dev)
 
-    base = upload_layer(prob, dev)
+    base = upload_layer(prob, dev, shared=args.shared)
     x, ids, w = upload_inputs(prob, dev)
     bufs = base.buffers(cfg.tokens)
     ws = None if args.no_workspace else base.workspace(cfg.tokens)
@@ -226,9 +236,19 @@ def run_ours(args, rank, world, local):
     stream.synchronize()
     if nvm.device_error() != 0:
         raise RuntimeError("device error word set by the forward")
-    active = int(bufs.active_count.item())
+    # With a shared expert, the forward runs topk + 1 slots over num_experts +
+    # slots table entries; the shared expert's weights count once in the bytes.
+    slots = 0
+    topk_run, experts_run, pairs_run = cfg.topk, cfg.experts, cfg.pairs
+    if args.shared:
+        rows = base.rows_per_shared_slot(cfg.tokens)
+        slots = nvm.shared_slots(cfg.tokens, rows)
+        topk_run, experts_run = cfg.topk + 1, cfg.experts + slots
+        pairs_run = cfg.tokens * topk_run
+    active_all = int(bufs.active_count.item())
+    active = active_all - slots
     per_expert = base.gate.nbytes_per_expert
-    routed_bytes = 3 * active * per_expert
+    routed_bytes = 3 * (active + (1 if args.shared else 0)) * per_expert
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     replicas = max(1, math.ceil(4 * l2 / max(routed_bytes, 1)))
     free = torch.cuda.mem_get_info(dev)[0]
@@ -291,20 +311,23 @@ def run_ours(args, rank, world, local):
     routed_gbs = world * routed_bytes / (ms_per_step * 1e-3) / 1e9
 
     # Dominant kernel, timed alone: gate+up SiLU, one launch per replica.
-    tc = ws is not None and _tc_path(args, cfg)
-    prefill = tc and _uses_prefill(args, cfg)
+    tc = ws is not None and _tc_path(args, cfg, pairs_run, experts_run)
+    prefill = tc and _uses_prefill(args, pairs_run, experts_run)
     gu_graph = torch.cuda.CUDAGraph()
-    cap = nvm.active_cap(cfg.experts, cfg.pairs)
+    cap = nvm.active_cap(experts_run, pairs_run)
 
     def gate_up(lay):
+        g, u = lay.gate.tables, lay.up.tables
+        if args.shared:
+            g, u = (t.tables for t in lay._ext_tables(slots)[:2])
         if ws is None:
-            nvm.gate_up_silu(x, lay.gate.tables, lay.up.tables, bufs.act, bufs.expert_offsets,
+            nvm.gate_up_silu(x, g, u, bufs.act, bufs.expert_offsets,
                              bufs.sorted_pair_ids, bufs.active_experts, bufs.active_count,
-                             cfg.inter, cfg.hidden, cap, cfg.tokens, cfg.topk, **_opts(args))
+                             cfg.inter, cfg.hidden, cap, cfg.tokens, topk_run, **_opts(args))
         else:
-            nvm.gate_up_silu_ws(x, lay.gate.tables, lay.up.tables, bufs.act, bufs.expert_offsets,
+            nvm.gate_up_silu_ws(x, g, u, bufs.act, bufs.expert_offsets,
                                 bufs.sorted_pair_ids, bufs.active_experts, bufs.active_count,
-                                cfg.inter, cfg.hidden, cap, cfg.tokens, cfg.topk, cfg.experts, ws,
+                                cfg.inter, cfg.hidden, cap, cfg.tokens, topk_run, experts_run, ws,
                                 **_opts(args))
     with torch.cuda.graph(gu_graph, stream=stream):
         for lay in layers:
@@ -318,8 +341,8 @@ def run_ours(args, rank, world, local):
         ev1.record(stream)
     torch.cuda.synchronize(dev)
     gu_ms = ev0.elapsed_time(ev1) / (reps * len(layers))
-    gu_bytes = 2 * active * per_expert
-    gu_flops = 2.0 * 2 * cfg.pairs * cfg.hidden * cfg.inter
+    gu_bytes = 2 * (active + (1 if args.shared else 0)) * per_expert
+    gu_flops = 2.0 * 2 * pairs_run * cfg.hidden * cfg.inter
     if prefill:
         achieved = gu_flops / (gu_ms * 1e-3) / 1e12
         roofline = {"kernel": "nvfp4_moe_gate_up_silu_ws (tcgen05, 128-row passes)", "bound": "tensor",
@@ -340,15 +363,17 @@ def run_ours(args, rank, world, local):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(prob)
+        cpu = cpu_baseline(prob, shared=args.shared)
 
     line = {
         "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
         "steps": steps, "warmup": warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16-mma/f32-acc", "data": "synthetic",
-        "config": {"workload": cfg.name, "hidden": cfg.hidden, "inter": cfg.inter,
+        "config": {"workload": cfg.name + ("+shared" if args.shared else ""), "hidden": cfg.hidden, "inter": cfg.inter,
                    "experts": cfg.experts, "topk": cfg.topk, "tokens": cfg.tokens,
                    "router": cfg.router, "active_experts": active,
+                   "shared_expert": ({"rows_per_table_entry": base.rows_per_shared_slot(cfg.tokens),
+                                      "table_entries": slots} if args.shared else None),
                    "path": ("tcgen05-nt128" if prefill else "tcgen05-nt16") if tc else "mma.sync",
                    "weight_replicas": len(layers),
                    "l2": f"weights rotate over {len(layers)} device replicas; "
@@ -360,8 +385,9 @@ def run_ours(args, rank, world, local):
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        # route_sort, [pack, tensor maps,] gate+up, [pack, tensor maps,] down, blend
-        "gpu_launches": (8 if tc else 4) * steps,
+        # [append_shared,] route_sort, [pack, tensor maps,] gate+up, [pack, tensor maps,]
+        # down, blend
+        "gpu_launches": ((8 if tc else 4) + (1 if args.shared else 0)) * steps,
         "clocks": clocks,
     }
     if rank == 0:
@@ -375,20 +401,20 @@ def _opts(args):
     return dict(path=args.path, split=args.split, tiles=args.tiles, depth=args.depth)
 
 
-def _tc_path(args, cfg):
+def _tc_path(args, cfg, pairs, experts):
     """Whether the projections take the tcgen05 path (the library's rule for
     the workspace calls: widths divisible by 128 / 256, and path 2, or path 0
     with at least 2 routed rows per expert on average)."""
     if args.path == 1 or cfg.inter % 128 or cfg.hidden % 256:
         return False
-    return args.path == 2 or cfg.pairs >= 2 * cfg.experts
+    return args.path == 2 or pairs >= 2 * experts
 
 
-def _uses_prefill(args, cfg):
+def _uses_prefill(args, pairs, experts):
     """Many rows per expert: the tcgen05 kernel runs 128-row passes and is tensor-bound."""
     if args.tiles:
         return args.tiles * 8 > 16
-    return (cfg.pairs + cfg.experts - 1) // cfg.experts > 16
+    return (pairs + experts - 1) // experts > 16
 
 
 def run_e2e(layers, prob, bufs, ws, dev, stream, steps, warmup, args, world):
@@ -471,21 +497,30 @@ def _oracle_sample(prob):
     return sub
 
 
-def _oracle_step(sub):
+def _oracle_step(sub, shared=None):
     import oracle as orc
     cfg = sub.cfg
     fns = [lambda e, mm=mm: sub.expert_weight(mm, e, cache=True) for mm in (0, 1, 2)]
-    orc.moe_forward(sub.x_bf16, sub.topk_ids, sub.topk_weights, cfg.experts, *fns,
-                    hidden=cfg.hidden, inter=cfg.inter)
+    if shared is None:
+        orc.moe_forward(sub.x_bf16, sub.topk_ids, sub.topk_weights, cfg.experts, *fns,
+                        hidden=cfg.hidden, inter=cfg.inter)
+    else:
+        orc.moe_forward_shared(sub.x_bf16, sub.topk_ids, sub.topk_weights, cfg.experts, *fns,
+                               hidden=cfg.hidden, inter=cfg.inter, shared=shared)
 
 
-def cpu_baseline(prob, budget_s=12.0):
+def _shared_weights(sub, shared: bool):
+    return tuple(sub.shared_weight(mm) for mm in (0, 1, 2)) if shared else None
+
+
+def cpu_baseline(prob, budget_s=12.0, shared=False):
     sub = _oracle_sample(prob)
-    _oracle_step(sub)  # draws (and caches) the sample's expert bytes
+    sh = _shared_weights(sub, shared)
+    _oracle_step(sub, sh)  # draws (and caches) the sample's expert bytes
     t0 = time.perf_counter()
     n = 0
     while True:
-        _oracle_step(sub)
+        _oracle_step(sub, sh)
         n += 1
         if time.perf_counter() - t0 > budget_s:
             break
@@ -493,8 +528,9 @@ def cpu_baseline(prob, budget_s=12.0):
     return {"value": sub.cfg.tokens * n / dt, "unit": "tokens/s", "cores": _oracle_threads(),
             "kind": "oracle",
             "sample": f"{n} fp64 oracle forwards of the first {sub.cfg.tokens} token(s) of "
-                      f"{prob.cfg.name} (route sort, dequantise the routed experts, gate+up SiLU, "
-                      f"down, blend), weight bytes pre-drawn, {dt:.1f} s"}
+                      f"{prob.cfg.name}{' with the shared expert' if shared else ''} (route sort, "
+                      f"dequantise the experts, gate+up SiLU, down, blend), weight bytes "
+                      f"pre-drawn, {dt:.1f} s"}
 
 
 def run_reference(args, rank, world):
@@ -505,21 +541,22 @@ def run_reference(args, rank, world):
     steps = args.steps if args.steps is not None else 5
     warmup = max(args.warmup, 3)
     sub = _oracle_sample(prob)
+    sh = _shared_weights(sub, args.shared)
     for _ in range(min(warmup, 1) if steps > 20 else warmup):
-        _oracle_step(sub)
+        _oracle_step(sub, sh)
     t0 = time.perf_counter()
     for _ in range(steps):
-        _oracle_step(sub)
+        _oracle_step(sub, sh)
     dt = time.perf_counter() - t0
     value = sub.cfg.tokens * steps / dt
     cores = _oracle_threads()
     sample = (f"each step: fp64 oracle forward of the first {sub.cfg.tokens} token(s) of "
-              f"{prob.cfg.name}")
+              f"{prob.cfg.name}{' with the shared expert' if args.shared else ''}")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": 0, "steps": steps, "warmup": warmup, "ms_per_step": dt * 1e3 / steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": prob.cfg.name, "hidden": prob.cfg.hidden, "inter": prob.cfg.inter,
+            "config": {"workload": prob.cfg.name + ("+shared" if args.shared else ""), "hidden": prob.cfg.hidden, "inter": prob.cfg.inter,
                        "experts": prob.cfg.experts, "topk": prob.cfg.topk, "tokens": prob.cfg.tokens},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
@@ -527,11 +564,82 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_check_scales(args, rank, world, local):
+    """nvfp4_moe_check_scales over the gate, up and down scale tables of every
+    expert of the workload (one launch per projection, HBM-bound byte scan)."""
+    import torch
+    import nvfp4_weight_quantized_moe_b200 as nvm
+    from workloads import make_problem
+    from workloads.device import upload_layer
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    prob = make_problem(args.config)
+    cfg = prob.cfg
+    layer = upload_layer(prob, dev)
+    projs = (layer.gate, layer.up, layer.down)
+    bad = torch.zeros(3, cfg.experts, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    scale_bytes = sum(p.scale.numel() for p in projs)
+
+    def one():
+        for i, p in enumerate(projs):
+            nvm.check_scales(p.tables, cfg.experts, p.n, p.k, bad[i], stream=stream)
+
+    steps = args.steps if args.steps is not None else 200
+    warmup = max(args.warmup, 3)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            one()
+    stream.synchronize()
+    if int(bad.sum().item()) != 0:
+        raise RuntimeError("generated scales reported invalid")
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        one()
+    sampler = ClockSampler(local)
+    sampler.start()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    sampler.mark(True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(steps):
+            g.replay()
+        ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    sampler.mark(False)
+    clocks = sampler.stop()
+    ms = ev0.elapsed_time(ev1) / steps
+    hbm, _, _, peak_kind = measured_peaks()
+    gbs = scale_bytes / (ms * 1e-3) / 1e9
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    line = {
+        "metric": "NVFP4 block-scale check GB/s (load time)", "value": gbs, "unit": "GB/s",
+        "n_gpus": 1, "steps": steps, "warmup": warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic",
+        "config": {"workload": cfg.name + " scale tables", "experts": cfg.experts,
+                   "bytes_per_step": scale_bytes,
+                   "l2": f"three tables of {scale_bytes / 3e6:.0f} MB each, L2 {l2 / 1e6:.0f} MB"},
+        "roofline": {"kernel": "check_scales_kernel", "bound": "hbm", "achieved": gbs, "peak": hbm,
+                     "unit": "GB/s", "frac": gbs / hbm, "peak_source": f"{peak_kind} HBM copy",
+                     "traffic": None},
+        "gpu_launches": 3 * steps,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
     rank, world, local = dist_info()
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.op == "check_scales":
+        run_check_scales(args, rank, world, local)
         return
     run_ours(args, rank, world, local)
 

@@ -9,7 +9,9 @@
  *   3. nvfp4_moe_down          y   = act Wd^T, FP32, per sorted row
  *   4. nvfp4_moe_blend         out[t] = sum_s w[t,s] * y[pos(t,s)], token order
  *
- * plus the load-time twin builder nvfp4_moe_transpose_u8.
+ * plus the load-time twin builder nvfp4_moe_transpose_u8, the load-time scale
+ * check nvfp4_moe_check_scales and nvfp4_moe_append_shared, which brings a
+ * shared expert into the same four steps.
  *
  * Launch order.  The kernels use programmatic dependent launch: each may start
  * while the previous kernel on the stream is still running and waits for it
@@ -329,6 +331,58 @@ NVFP4_MOE_API int nvfp4_moe_forward(const uint16_t* x, const int32_t* topk_ids,
  */
 NVFP4_MOE_API int nvfp4_moe_transpose_u8(const uint8_t* src, uint8_t* dst, uint32_t rows, uint32_t cols,
                            cudaStream_t stream);
+
+/*
+ * Shared expert.  The launcher docs of nvfp4_moe_grouped.rs
+ * (moe_expert_gate_up_act_nvfp4_grouped, moe_expert_down_act_nvfp4_grouped)
+ * run a shared expert in the same gate+up and down launches as the routed
+ * experts: one row per token, its own weights, outputs laid out by token.
+ * Here it enters the forward as one more routing slot per token:
+ *
+ *   ids_out     i32 [num_tokens, topk + 1]  out: slots 0..topk-1 = topk_ids;
+ *               slot topk = num_experts + t / shared_rows
+ *   weights_out f32 [num_tokens, topk + 1]  out: slots 0..topk-1 = topk_weights;
+ *               slot topk = shared_weights[t], or 1 when shared_weights is NULL
+ *   shared_weights f32 [num_tokens] or NULL
+ *
+ * The caller's three tables have num_experts + S entries, S =
+ * nvfp4_moe_shared_slots(num_tokens, shared_rows), entries num_experts ..
+ * num_experts + S - 1 all holding the shared expert's weights (same shapes
+ * as a routed expert).  Run the forward on ids_out / weights_out with topk + 1
+ * slots and num_experts + S experts: out then adds shared_weights[t] times
+ * the shared expert's output, and because the shared entries sort after
+ * every routed expert, in token order, rows expert_offsets[num_experts] ..
+ * + num_tokens - 1 of act and y are the shared expert's SiLU product and down
+ * output for tokens 0 .. num_tokens - 1 (sh_act and sh_down_out).  Each block
+ * of shared_rows tokens gets its own CTAs in the projections; a block size
+ * near the routed rows per expert keeps the work even.
+ * ESHAPE if num_experts + S > 1024 or num_tokens * (topk + 1) > 1<<24;
+ * EINVAL for shared_rows == 0 or a NULL required pointer.
+ */
+NVFP4_MOE_API int nvfp4_moe_append_shared(const int32_t* topk_ids, const float* topk_weights,
+                                          const float* shared_weights, uint32_t num_tokens,
+                                          uint32_t topk, uint32_t num_experts,
+                                          uint32_t shared_rows, int32_t* ids_out,
+                                          float* weights_out, cudaStream_t stream);
+
+/* Host helper: table entries the shared expert takes, ceil(num_tokens / shared_rows)
+ * (0 for shared_rows == 0). */
+NVFP4_MOE_API uint32_t nvfp4_moe_shared_slots(uint32_t num_tokens, uint32_t shared_rows);
+
+/*
+ * Load-time check of one projection's E4M3 block scales
+ * (nvfp4_tc_lean_repack in nvfp4_moe_grouped.rs flags a negative or NaN
+ * scale, after which the matrix is unusable).  For each expert e of the table
+ * with non-NULL packed_ptrs[e] and scale_ptrs[e], ADDS to bad[e] the number of
+ * its n * k / 16 scale codes that are NaN (0x7F, 0xFF) or negative (0x81 ..
+ * 0xFE; 0x80 is -0 and passes).  bad: u32 [num_experts], device, zeroed by
+ * the caller before the first check it collects.  scale2 is not read.
+ * k % 256 == 0 (every scale row is whole 16-byte vectors), 1 <= num_experts
+ * <= 1024, n * k / 16 < 2^32.  Bit-exact; the order of the adds does not
+ * change the counts.
+ */
+NVFP4_MOE_API int nvfp4_moe_check_scales(nvfp4_expert_tables t, uint32_t num_experts, uint32_t n,
+                                         uint32_t k, uint32_t* bad, cudaStream_t stream);
 
 /* Host helper: launch bound on active experts, min(num_experts, num_pairs). */
 NVFP4_MOE_API uint32_t nvfp4_moe_active_cap(uint32_t num_experts, uint32_t num_pairs);

@@ -15,7 +15,9 @@ from ._binding import (  # noqa: F401
     LaunchOpts,
     NVFP4MoEError,
     active_cap,
+    append_shared,
     blend,
+    check_scales,
     device_error,
     down,
     down_ws,
@@ -24,6 +26,7 @@ from ._binding import (  # noqa: F401
     gate_up_silu,
     gate_up_silu_ws,
     route_sort,
+    shared_slots,
     transpose_u8,
     workspace_bytes,
 )

@@ -82,6 +82,10 @@ _sig = {
                                   ExpertTables, ctypes.POINTER(Buffers), c_u32, c_u32, c_u32, c_u32,
                                   c_u32, ctypes.POINTER(LaunchOpts), c_void_p, ctypes.c_size_t,
                                   c_void_p]),
+    "nvfp4_moe_append_shared": (c_int, [c_void_p, c_void_p, c_void_p, c_u32, c_u32, c_u32, c_u32,
+                                        c_void_p, c_void_p, c_void_p]),
+    "nvfp4_moe_shared_slots": (c_u32, [c_u32, c_u32]),
+    "nvfp4_moe_check_scales": (c_int, [ExpertTables, c_u32, c_u32, c_u32, c_void_p, c_void_p]),
     "nvfp4_moe_workspace_bytes": (ctypes.c_size_t, [c_u32, c_u32, c_u32, c_u32]),
     "nvfp4_moe_device_error": (c_int, [c_int]),
     "nvfp4_moe_active_cap": (c_u32, [c_u32, c_u32]),
@@ -195,6 +199,38 @@ def transpose_u8(src, dst, stream=None) -> None:
         raise ValueError("dst must be [cols, rows]")
     _check("nvfp4_moe_transpose_u8", _lib.nvfp4_moe_transpose_u8(
         _ptr(src, torch.uint8, "src"), _ptr(dst, torch.uint8, "dst"), rows, cols, _stream(stream)))
+
+
+def shared_slots(num_tokens: int, shared_rows: int) -> int:
+    """Table entries the shared expert takes: ceil(num_tokens / shared_rows)."""
+    return int(_lib.nvfp4_moe_shared_slots(num_tokens, shared_rows))
+
+
+def append_shared(topk_ids, topk_weights, num_experts, shared_rows, ids_out, weights_out,
+                  shared_weights=None, stream=None) -> None:
+    """nvfp4_moe_append_shared: routing [M, k+1] with the shared expert as slot k."""
+    m, k = topk_ids.shape
+    if tuple(ids_out.shape) != (m, k + 1) or tuple(weights_out.shape) != (m, k + 1):
+        raise ValueError("ids_out and weights_out must be [M, topk + 1]")
+    if tuple(topk_weights.shape) != (m, k):
+        raise ValueError("topk_weights must be [M, topk]")
+    if shared_weights is not None and shared_weights.numel() != m:
+        raise ValueError("shared_weights must hold one value per token")
+    _check("nvfp4_moe_append_shared", _lib.nvfp4_moe_append_shared(
+        _ptr(topk_ids, torch.int32, "topk_ids"), _ptr(topk_weights, torch.float32, "topk_weights"),
+        _ptr(shared_weights, torch.float32, "shared_weights"), m, k, num_experts, shared_rows,
+        _ptr(ids_out, torch.int32, "ids_out"), _ptr(weights_out, torch.float32, "weights_out"),
+        _stream(stream)))
+
+
+def check_scales(tables: ExpertTables, num_experts, n, k, bad, stream=None) -> None:
+    """nvfp4_moe_check_scales: add each expert's count of NaN / negative scale codes to bad."""
+    if bad.numel() < num_experts:
+        raise ValueError("bad must hold num_experts counters")
+    if bad.dtype not in (torch.int32, torch.uint32):
+        raise TypeError("bad: expected 32-bit counters")
+    _check("nvfp4_moe_check_scales", _lib.nvfp4_moe_check_scales(
+        tables, num_experts, n, k, _ptr(bad, None, "bad"), _stream(stream)))
 
 
 def workspace_bytes(num_tokens, topk, hidden, inter) -> int:

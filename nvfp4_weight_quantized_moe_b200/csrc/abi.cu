@@ -379,6 +379,40 @@ int nvfp4_moe_forward(const uint16_t* x, const int32_t* topk_ids, const float* t
                          hidden, stream);
 }
 
+uint32_t nvfp4_moe_shared_slots(uint32_t num_tokens, uint32_t shared_rows) {
+  if (shared_rows == 0) return 0;
+  return (uint32_t)(((uint64_t)num_tokens + shared_rows - 1) / shared_rows);
+}
+
+int nvfp4_moe_append_shared(const int32_t* topk_ids, const float* topk_weights,
+                            const float* shared_weights, uint32_t num_tokens, uint32_t topk,
+                            uint32_t num_experts, uint32_t shared_rows, int32_t* ids_out,
+                            float* weights_out, cudaStream_t stream) {
+  if (shared_rows == 0) return NVFP4_MOE_EINVAL;
+  if (topk == 0 || num_experts == 0 ||
+      (uint64_t)num_experts + nvfp4_moe_shared_slots(num_tokens, shared_rows) > kMaxExperts ||
+      (uint64_t)num_tokens * (topk + 1) > kMaxPairs)
+    return NVFP4_MOE_ESHAPE;
+  if (num_tokens == 0) return NVFP4_MOE_OK;
+  if (topk_ids == nullptr || topk_weights == nullptr || ids_out == nullptr ||
+      weights_out == nullptr)
+    return NVFP4_MOE_EINVAL;
+  return status_of(launch_append_shared(topk_ids, topk_weights, shared_weights, ids_out,
+                                        weights_out, num_tokens, topk, num_experts, shared_rows,
+                                        stream));
+}
+
+int nvfp4_moe_check_scales(nvfp4_expert_tables t, uint32_t num_experts, uint32_t n, uint32_t k,
+                           uint32_t* bad, cudaStream_t stream) {
+  if (num_experts == 0 || num_experts > kMaxExperts || n == 0 || k == 0 || k % 256 != 0 ||
+      (uint64_t)n * (k / 16) > 0xFFFFFFFFull)
+    return NVFP4_MOE_ESHAPE;
+  if (t.packed_ptrs == nullptr || t.scale_ptrs == nullptr || bad == nullptr)
+    return NVFP4_MOE_EINVAL;
+  return status_of(launch_check_scales(t.packed_ptrs, t.scale_ptrs, num_experts,
+                                       (uint64_t)n * (k / 16), bad, stream));
+}
+
 int nvfp4_moe_transpose_u8(const uint8_t* src, uint8_t* dst, uint32_t rows, uint32_t cols,
                            cudaStream_t stream) {
   if (rows == 0 || cols == 0) return NVFP4_MOE_OK;

@@ -63,6 +63,15 @@ cudaError_t launch_blend(const float* y, const float* topk_weights, const int32_
                          float* out_f32, uint16_t* out_bf16, uint32_t num_tokens, uint32_t topk,
                          uint32_t hidden, cudaStream_t stream);
 
+cudaError_t launch_append_shared(const int32_t* ids, const float* w, const float* shared_w,
+                                 int32_t* ids_out, float* w_out, uint32_t num_tokens,
+                                 uint32_t topk, uint32_t num_experts, uint32_t shared_rows,
+                                 cudaStream_t stream);
+
+cudaError_t launch_check_scales(const void* const* packed_ptrs, const void* const* scale_ptrs,
+                                uint32_t num_experts, uint64_t bytes_per_expert, uint32_t* bad,
+                                cudaStream_t stream);
+
 cudaError_t launch_transpose_u8(const uint8_t* src, uint8_t* dst, uint32_t rows, uint32_t cols,
                                 cudaStream_t stream);
 

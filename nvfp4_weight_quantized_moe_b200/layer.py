@@ -50,14 +50,21 @@ class NVFP4Projection:
 
 
 class MoEBuffers:
-    """Outputs and intermediates of one forward, for M tokens."""
+    """Outputs and intermediates of one forward, for M tokens.
+
+    With a shared expert, ``topk`` and ``num_experts`` count its slot and
+    table entries, and ``topk_ids`` / ``topk_weights`` hold the appended
+    routing [M, topk] that nvfp4_moe_append_shared writes.
+    """
 
     def __init__(self, num_tokens: int, topk: int, num_experts: int, hidden: int, inter: int,
-                 device, out_bf16: bool = False):
+                 device, out_bf16: bool = False, shared: bool = False):
         p = num_tokens * topk
         i32 = dict(dtype=torch.int32, device=device)
         f32 = dict(dtype=torch.float32, device=device)
         self.num_tokens, self.topk = num_tokens, topk
+        self.topk_ids = torch.empty(max(num_tokens, 1), topk, **i32) if shared else None
+        self.topk_weights = torch.empty(max(num_tokens, 1), topk, **f32) if shared else None
         self.expert_offsets = torch.empty(num_experts + 1, **i32)
         self.sorted_pair_ids = torch.empty(max(p, 1), **i32)
         self.pair_pos = torch.empty(max(p, 1), **i32)
@@ -77,10 +84,32 @@ class MoEBuffers:
             self.out_bf16.data_ptr() if self.out_bf16 is not None else None)
 
 
-class NVFP4MoE:
-    """The grouped NVFP4 expert forward of one layer."""
+class _Tables:
+    """Expert tables of one projection with the shared expert's entries appended."""
 
-    def __init__(self, gate: NVFP4Projection, up: NVFP4Projection, down: NVFP4Projection, topk: int):
+    def __init__(self, routed: NVFP4Projection, shared: NVFP4Projection, slots: int):
+        dev = routed.packed.device
+        sp, ss = shared.packed_ptrs[:1], shared.scale_ptrs[:1]
+        self.packed_ptrs = torch.cat([routed.packed_ptrs, sp.expand(slots)]).contiguous()
+        self.scale_ptrs = torch.cat([routed.scale_ptrs, ss.expand(slots)]).contiguous()
+        self.scale2 = torch.cat([routed.scale2, shared.scale2[:1].expand(slots)]).to(dev).contiguous()
+        self.tables = B.ExpertTables(self.packed_ptrs.data_ptr(), self.scale_ptrs.data_ptr(),
+                                     self.scale2.data_ptr())
+
+
+class NVFP4MoE:
+    """The grouped NVFP4 expert forward of one layer, optionally with a shared expert.
+
+    ``shared`` = (gate, up, down) projections of one expert (E = 1) with the
+    routed experts' shapes: every token also runs it, in the same gate+up and
+    down launches (nvfp4_moe_append_shared), and ``out`` adds its output times
+    the per-token ``shared_weights`` given to :meth:`forward` (1 by default).
+    ``shared_rows`` tokens share one table entry of the shared expert, and so
+    one group of CTAs; by default about the routed rows per expert.
+    """
+
+    def __init__(self, gate: NVFP4Projection, up: NVFP4Projection, down: NVFP4Projection, topk: int,
+                 shared=None, shared_rows: int = 0):
         if not (gate.num_experts == up.num_experts == down.num_experts):
             raise ValueError("expert counts differ")
         if gate.n != up.n or gate.k != up.k or down.n != gate.k or down.k != gate.n:
@@ -89,20 +118,60 @@ class NVFP4MoE:
         self.num_experts = gate.num_experts
         self.hidden, self.inter = gate.k, gate.n
         self.topk = topk
+        self.shared = None
+        self.shared_rows = int(shared_rows)
+        if shared is not None:
+            sg, su, sd = shared
+            for sp, rp in ((sg, gate), (su, up), (sd, down)):
+                if sp.num_experts != 1 or (sp.n, sp.k) != (rp.n, rp.k):
+                    raise ValueError("the shared expert is one expert with the routed shapes")
+            self.shared = (sg, su, sd)
+        self._ext = {}
+
+    # -- shared expert bookkeeping ------------------------------------------------
+    def rows_per_shared_slot(self, num_tokens: int) -> int:
+        """Tokens per shared table entry for a batch of num_tokens."""
+        if self.shared_rows:
+            rows = self.shared_rows
+        else:
+            mean = -(-num_tokens * self.topk // self.num_experts)
+            rows = max(16, -(-mean // 16) * 16)
+        room = 1024 - self.num_experts
+        if room < 1:
+            raise ValueError("no table entries left for the shared expert")
+        return max(rows, -(-num_tokens // room))
+
+    def _ext_tables(self, slots: int):
+        if slots not in self._ext:
+            self._ext[slots] = tuple(_Tables(r, s, slots)
+                                     for r, s in zip((self.gate, self.up, self.down), self.shared))
+        return self._ext[slots]
+
+    def _route_shape(self, num_tokens: int):
+        """(slots per token, table entries) of a batch."""
+        if self.shared is None:
+            return self.topk, self.num_experts
+        slots = B.shared_slots(num_tokens, self.rows_per_shared_slot(num_tokens))
+        return self.topk + 1, self.num_experts + slots
 
     def buffers(self, num_tokens: int, out_bf16: bool = False) -> MoEBuffers:
-        return MoEBuffers(num_tokens, self.topk, self.num_experts, self.hidden, self.inter,
-                          self.gate.packed.device, out_bf16)
+        k, e = self._route_shape(num_tokens)
+        if self.shared is not None:
+            e = 1024  # the library's largest table: enough entries for any batch size
+        return MoEBuffers(num_tokens, k, e, self.hidden, self.inter, self.gate.packed.device,
+                          out_bf16, shared=self.shared is not None)
 
     def workspace(self, num_tokens: int) -> torch.Tensor:
         """Device workspace of the tcgen05 path for batches of up to num_tokens."""
-        n = B.workspace_bytes(num_tokens, self.topk, self.hidden, self.inter)
+        k, _ = self._route_shape(num_tokens)
+        n = B.workspace_bytes(num_tokens, k, self.hidden, self.inter)
         return torch.empty(max(n, 1), dtype=torch.uint8, device=self.gate.packed.device)
 
     def forward(self, x: torch.Tensor, topk_ids: torch.Tensor, topk_weights: torch.Tensor,
                 bufs: Optional[MoEBuffers] = None, path: int = 0, split: int = 0,
                 tiles: int = 0, depth: int = 0, workspace: Optional[torch.Tensor] = None,
-                stream=None, steps: bool = False) -> MoEBuffers:
+                stream=None, steps: bool = False,
+                shared_weights: Optional[torch.Tensor] = None) -> MoEBuffers:
         """Run the four steps on ``stream``; results land in ``bufs`` (returned).
         One library call (nvfp4_moe_forward) by default; ``steps=True`` makes the
         four single-step calls instead (same kernels, same results).
@@ -110,36 +179,63 @@ class NVFP4MoE:
         path / split / tiles / depth are the launch options of the two
         projections (0 = chosen from the shape); see nvfp4_moe_launch_opts.
         With a ``workspace`` (see :meth:`workspace`) the projections may take
-        the tcgen05 path."""
+        the tcgen05 path.  With a shared expert, the routing is first extended
+        by one slot per token (one more library call) and ``shared_weights``
+        (f32 [M] or None for 1) weighs its output."""
         m = x.shape[0]
         if bufs is None:
             bufs = self.buffers(m)
         if m > bufs.num_tokens:
             raise ValueError("buffers were sized for fewer tokens")
+        gate_t, up_t, down_t = self.gate.tables, self.up.tables, self.down.tables
+        topk, num_experts = self.topk, self.num_experts
+        if self.shared is not None:
+            rows = self.rows_per_shared_slot(m)
+            slots = B.shared_slots(m, rows)
+            if num_experts + slots > bufs.active_experts.numel():
+                raise ValueError("buffers hold too few expert entries for this batch")
+            ids, ws = bufs.topk_ids[:m], bufs.topk_weights[:m]
+            B.append_shared(topk_ids, topk_weights, num_experts, rows, ids, ws,
+                            shared_weights=shared_weights, stream=stream)
+            topk_ids, topk_weights = ids, ws
+            gate_t, up_t, down_t = (t.tables for t in self._ext_tables(slots))
+            topk, num_experts = topk + 1, num_experts + slots
+        elif shared_weights is not None:
+            raise ValueError("shared_weights given to a layer without a shared expert")
         if not steps:
-            B.forward(x, topk_ids, topk_weights, self.gate.tables, self.up.tables, self.down.tables,
-                      bufs.c_buffers, self.num_experts, self.hidden, self.inter, workspace=workspace,
-                      path=path, split=split, tiles=tiles, depth=depth, stream=stream)
+            B.forward(x, topk_ids, topk_weights, gate_t, up_t, down_t, bufs.c_buffers, num_experts,
+                      self.hidden, self.inter, workspace=workspace, path=path, split=split,
+                      tiles=tiles, depth=depth, stream=stream)
             return bufs
-        p = m * self.topk
-        cap = B.active_cap(self.num_experts, p)
-        B.route_sort(topk_ids, self.num_experts, bufs.expert_offsets, bufs.sorted_pair_ids,
-                     bufs.pair_pos, bufs.active_experts, bufs.active_count, bufs.status,
-                     stream=stream)
+        p = m * topk
+        cap = B.active_cap(num_experts, p)
+        B.route_sort(topk_ids, num_experts, bufs.expert_offsets[:num_experts + 1],
+                     bufs.sorted_pair_ids, bufs.pair_pos, bufs.active_experts[:num_experts],
+                     bufs.active_count, bufs.status, stream=stream)
         opts = dict(path=path, split=split, tiles=tiles, depth=depth, stream=stream)
         if workspace is None:
-            B.gate_up_silu(x, self.gate.tables, self.up.tables, bufs.act, bufs.expert_offsets,
-                           bufs.sorted_pair_ids, bufs.active_experts, bufs.active_count,
-                           self.inter, self.hidden, cap, m, self.topk, **opts)
-            B.down(bufs.act, self.down.tables, bufs.y, bufs.expert_offsets, bufs.active_experts,
-                   bufs.active_count, self.hidden, self.inter, cap, m, self.topk, **opts)
+            B.gate_up_silu(x, gate_t, up_t, bufs.act, bufs.expert_offsets, bufs.sorted_pair_ids,
+                           bufs.active_experts, bufs.active_count, self.inter, self.hidden, cap, m,
+                           topk, **opts)
+            B.down(bufs.act, down_t, bufs.y, bufs.expert_offsets, bufs.active_experts,
+                   bufs.active_count, self.hidden, self.inter, cap, m, topk, **opts)
         else:
-            B.gate_up_silu_ws(x, self.gate.tables, self.up.tables, bufs.act, bufs.expert_offsets,
+            B.gate_up_silu_ws(x, gate_t, up_t, bufs.act, bufs.expert_offsets,
                               bufs.sorted_pair_ids, bufs.active_experts, bufs.active_count,
-                              self.inter, self.hidden, cap, m, self.topk, self.num_experts,
-                              workspace, **opts)
-            B.down_ws(bufs.act, self.down.tables, bufs.y, bufs.expert_offsets,
-                      bufs.active_experts, bufs.active_count, self.hidden, self.inter, cap, m,
-                      self.topk, self.num_experts, workspace, **opts)
+                              self.inter, self.hidden, cap, m, topk, num_experts, workspace, **opts)
+            B.down_ws(bufs.act, down_t, bufs.y, bufs.expert_offsets, bufs.active_experts,
+                      bufs.active_count, self.hidden, self.inter, cap, m, topk, num_experts,
+                      workspace, **opts)
         B.blend(bufs.y, topk_weights, bufs.pair_pos, bufs.out, bufs.out_bf16, stream=stream)
         return bufs
+
+    def shared_rows_of(self, bufs: MoEBuffers, m: int):
+        """(sh_act [M, I], sh_out [M, H]) views of the last forward's shared rows.
+
+        They start at sorted position expert_offsets[E] (read from the device,
+        which synchronises): the kept routed pairs all sort before them.
+        """
+        if self.shared is None:
+            raise ValueError("no shared expert")
+        lo = int(bufs.expert_offsets[self.num_experts].item())
+        return bufs.act[lo:lo + m], bufs.y[lo:lo + m]

@@ -122,3 +122,25 @@ def test_workspace_calls_check_size_and_alignment_on_the_host(lib):
     # path 2 with a width the tcgen05 kernels do not take
     assert L.nvfp4_moe_down_ws(p8, t, p8, p8, p8, p8, 128, inter, cap, tokens, topk, experts,
                                ctypes.byref(opts), ctypes.c_void_p(1 << 20), need, None) == 2
+
+
+def test_shared_and_scale_check_calls_validate_on_the_host(lib):
+    import nvfp4_weight_quantized_moe_b200._binding as B
+    L = B._lib
+    p8 = ctypes.c_void_p(8)
+    assert L.nvfp4_moe_shared_slots(8192, 512) == 16
+    assert L.nvfp4_moe_shared_slots(7, 2) == 4
+    assert L.nvfp4_moe_shared_slots(0, 16) == 0
+    assert L.nvfp4_moe_shared_slots(5, 0) == 0
+    # shared_rows = 0; too many table entries (1000 + 32); no tokens (nothing launched)
+    assert L.nvfp4_moe_append_shared(p8, p8, None, 4, 2, 8, 0, p8, p8, None) == 1
+    assert L.nvfp4_moe_append_shared(p8, p8, None, 512, 2, 1000, 16, p8, p8, None) == 2
+    assert L.nvfp4_moe_append_shared(None, None, None, 0, 2, 8, 16, None, None, None) == 0
+    assert L.nvfp4_moe_append_shared(None, p8, None, 4, 2, 8, 16, p8, p8, None) == 1
+    t = B.ExpertTables(8, 8, None)
+    # k not a multiple of 256; 0 or > 1024 experts; NULL counters or tables
+    assert L.nvfp4_moe_check_scales(t, 4, 128, 300, p8, None) == 2
+    assert L.nvfp4_moe_check_scales(t, 0, 128, 256, p8, None) == 2
+    assert L.nvfp4_moe_check_scales(t, 1025, 128, 256, p8, None) == 2
+    assert L.nvfp4_moe_check_scales(t, 4, 128, 256, None, None) == 1
+    assert L.nvfp4_moe_check_scales(B.ExpertTables(None, 8, None), 4, 128, 256, p8, None) == 1

@@ -425,3 +425,198 @@ def test_forward_full_size_sampled(name, ws):
     mid = int(np.random.default_rng(99).integers(1, prob.cfg.tokens - 1))
     tokens = [0, mid, prob.cfg.tokens - 1]
     _check_sampled(prob, bufs, tokens)
+
+
+# --------------------------------------------------------------------------- #
+# Shared expert: appended routing slots through the same launches
+# --------------------------------------------------------------------------- #
+
+@pytest.mark.parametrize("m,k,e,rows,weighted", [(1, 2, 8, 16, False), (7, 3, 5, 2, True),
+                                                 (33, 8, 128, 16, True), (70, 2, 9, 64, False),
+                                                 (300, 8, 256, 7, True)])
+def test_append_shared_bit_exact(m, k, e, rows, weighted):
+    _need_gpu()
+    import nvfp4_weight_quantized_moe_b200 as nvm
+    rng = np.random.default_rng(m * 7 + e)
+    ids = rng.integers(0, e, (m, k)).astype(np.int32)
+    w = rng.random((m, k)).astype(np.float32)
+    sw = rng.random(m).astype(np.float32) if weighted else None
+    ids_out = torch.full((m, k + 1), -7, dtype=torch.int32, device="cuda")
+    w_out = torch.full((m, k + 1), float("nan"), dtype=torch.float32, device="cuda")
+    nvm.append_shared(torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda(), e, rows, ids_out,
+                      w_out, shared_weights=None if sw is None else torch.from_numpy(sw).cuda())
+    torch.cuda.synchronize()
+    ref_ids, ref_w = orc.append_shared_routing(ids, w, e, rows, sw)
+    np.testing.assert_array_equal(ids_out.cpu().numpy(), ref_ids)
+    np.testing.assert_array_equal(w_out.cpu().numpy().view(np.uint32), ref_w.view(np.uint32))
+    assert nvm.shared_slots(m, rows) == -(-m // rows)
+
+
+def _shared_ref(prob, sw):
+    cfg = prob.cfg
+    shared = tuple(prob.shared_weight(mt) for mt in (MATRIX_GATE, MATRIX_UP, MATRIX_DOWN))
+    return orc.moe_forward_shared(prob.x_bf16, prob.topk_ids, prob.topk_weights, cfg.experts,
+                                  *_fns(prob), hidden=cfg.hidden, inter=cfg.inter, shared=shared,
+                                  shared_weights=sw)
+
+
+def _gpu_forward_shared(prob, sw=None, shared_rows=0, ws=False, layer=None, **opts):
+    from workloads.device import upload_inputs, upload_layer
+    import nvfp4_weight_quantized_moe_b200 as nvm
+    layer = layer or upload_layer(prob, shared=True, shared_rows=shared_rows)
+    x, ids, w = upload_inputs(prob)
+    bufs = layer.buffers(prob.cfg.tokens, out_bf16=True)
+    for t in (bufs.act, bufs.y, bufs.out):
+        t.fill_(float("nan"))
+    workspace = layer.workspace(prob.cfg.tokens) if ws else None
+    if workspace is not None:
+        workspace.fill_(0xFF)
+    swd = None if sw is None else torch.from_numpy(sw).cuda()
+    layer.forward(x, ids, w, bufs, workspace=workspace, shared_weights=swd, **opts)
+    torch.cuda.synchronize()
+    assert nvm.device_error() == 0
+    return layer, bufs
+
+
+SHARED_CASES = [("tiny", 0, False), ("ragged", 2, True), ("hot", 16, True), ("zipf", 0, False),
+                ("longk", 1, True)]
+
+
+@pytest.mark.parametrize("ws", [False, True], ids=["decode-path", "tcgen05"])
+@pytest.mark.parametrize("name,rows,weighted", SHARED_CASES)
+def test_forward_with_shared_expert(name, rows, weighted, ws):
+    _need_gpu()
+    prob = make_problem(SMALL[name])
+    cfg = prob.cfg
+    sw = (np.random.default_rng(cfg.seed).random(cfg.tokens).astype(np.float32)
+          if weighted else None)
+    opts = dict(path=2) if ws else {}
+    layer, bufs = _gpu_forward_shared(prob, sw, rows, ws=ws, **opts)
+    ref = _shared_ref(prob, sw)
+    # The sort of the appended routing is bit-exact; the shared rows come last.
+    r = layer.rows_per_shared_slot(cfg.tokens)
+    slots = -(-cfg.tokens // r)
+    ids2, _ = orc.append_shared_routing(prob.topk_ids, prob.topk_weights, cfg.experts, r, sw)
+    rs = orc.route_sort(ids2, cfg.experts + slots)
+    e2 = cfg.experts + slots
+    np.testing.assert_array_equal(bufs.expert_offsets.cpu().numpy()[:e2 + 1], rs.expert_offsets)
+    np.testing.assert_array_equal(bufs.sorted_pair_ids.cpu().numpy(), rs.sorted_pair_ids)
+    np.testing.assert_array_equal(bufs.pair_pos.cpu().numpy(), rs.pair_pos)
+    sh_act, sh_out = layer.shared_rows_of(bufs, cfg.tokens)
+    _close(sh_act.cpu().numpy(), ref["sh_act"], "sh_act")
+    _close(sh_out.cpu().numpy(), ref["sh_out"], "sh_out")
+    _close(bufs.out.cpu().numpy(), ref["out"], "out")
+    ob = bufs.out_bf16.float().cpu().numpy()
+    np.testing.assert_array_equal(ob, bufs.out.bfloat16().float().cpu().numpy())
+
+
+@pytest.mark.parametrize("ws", [False, True], ids=["decode-path", "tcgen05"])
+def test_shared_one_call_equals_four_steps(ws):
+    _need_gpu()
+    prob = make_problem(SMALL["hot"])
+    sw = np.random.default_rng(3).random(prob.cfg.tokens).astype(np.float32)
+    layer, one = _gpu_forward_shared(prob, sw, 16, ws=ws)
+    _, four = _gpu_forward_shared(prob, sw, 16, ws=ws, layer=layer, steps=True)
+    e2 = prob.cfg.experts + -(-prob.cfg.tokens // 16)
+    for f in ("expert_offsets", "sorted_pair_ids", "pair_pos", "act", "y", "out"):
+        a, b = getattr(one, f), getattr(four, f)
+        if f == "expert_offsets":  # the buffer has room for 1024 experts; e2 + 1 are written
+            a, b = a[:e2 + 1], b[:e2 + 1]
+        if a.dtype == torch.float32:
+            a, b = a.view(torch.int32), b.view(torch.int32)
+        assert torch.equal(a, b), f
+
+
+@pytest.mark.parametrize("ws", [False, True], ids=["decode-path", "tcgen05"])
+def test_forward_with_shared_full_decode_m32(ws):
+    _need_gpu()
+    prob = make_problem("decode_m32")
+    _, bufs = _gpu_forward_shared(prob, ws=ws)
+    _close(bufs.out.cpu().numpy(), _shared_ref(prob, None)["out"], "out")
+
+
+def test_forward_with_shared_full_prefill_sampled():
+    """prefill M=8192 with the shared expert (16 shared table entries), sampled tokens."""
+    _need_gpu()
+    prob = make_problem("prefill_m8192")
+    cfg = prob.cfg
+    sw = np.random.default_rng(8).random(cfg.tokens).astype(np.float32)
+    layer, bufs = _gpu_forward_shared(prob, sw, ws=True)
+    assert layer.rows_per_shared_slot(cfg.tokens) == 512
+    tokens = [0, 4097, cfg.tokens - 1]
+    routed = orc.moe_forward_tokens(prob.x_bf16, prob.topk_ids, prob.topk_weights, cfg.experts,
+                                    *_fns(prob), tokens=tokens, hidden=cfg.hidden)
+    shared = tuple(prob.shared_weight(mt) for mt in (MATRIX_GATE, MATRIX_UP, MATRIX_DOWN))
+    sh_act, sh_out = orc.shared_expert(prob.x_bf16[tokens], *shared)
+    ref = routed + sw[tokens, None].astype(np.float64) * sh_out
+    _close(bufs.out.cpu().numpy()[tokens], ref, "out (sampled tokens)")
+    g_act, g_out = layer.shared_rows_of(bufs, cfg.tokens)
+    _close(g_act.cpu().numpy()[tokens], sh_act, "sh_act (sampled tokens)")
+    _close(g_out.cpu().numpy()[tokens], sh_out, "sh_out (sampled tokens)")
+
+
+# --------------------------------------------------------------------------- #
+# Load-time scale check: bit-exact counts
+# --------------------------------------------------------------------------- #
+
+def _scale_table(scales, null=()):
+    """Tables over device scale arrays; packed entries only mark NULL experts."""
+    import nvfp4_weight_quantized_moe_b200 as nvm
+    dev = [torch.from_numpy(s).cuda() for s in scales]
+    sp = torch.tensor([0 if i in null else d.data_ptr() for i, d in enumerate(dev)],
+                      dtype=torch.int64, device="cuda")
+    pp = sp.clone()
+    return dev, sp, pp, nvm.ExpertTables(pp.data_ptr(), sp.data_ptr(), None)
+
+
+@pytest.mark.parametrize("e,n,k,null", [(7, 96, 512, (2,)), (3, 4096, 2048, ()), (1, 16, 256, ())])
+def test_check_scales_counts_bit_exact(e, n, k, null):
+    _need_gpu()
+    import nvfp4_weight_quantized_moe_b200 as nvm
+    rng = np.random.default_rng(e * n + k)
+    scales = []
+    for i in range(e):
+        s = rng.integers(0x18, 0x49, (n, k // 16), dtype=np.uint8)
+        planted = rng.integers(0, s.size, int(rng.integers(0, 40)))
+        s.reshape(-1)[planted] = rng.choice(np.array([0x7F, 0xFF, 0x81, 0xB8, 0xFE, 0x80, 0x7E],
+                                                     dtype=np.uint8), planted.size)
+        scales.append(s)
+    dev, sp, pp, t = _scale_table(scales, null)
+    bad = torch.zeros(e, dtype=torch.int32, device="cuda")
+    nvm.check_scales(t, e, n, k, bad)
+    torch.cuda.synchronize()
+    expect = np.array([0 if i in null else orc.count_bad_scales(s) for i, s in enumerate(scales)])
+    np.testing.assert_array_equal(bad.cpu().numpy(), expect)
+    nvm.check_scales(t, e, n, k, bad)  # the counts accumulate
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(bad.cpu().numpy(), 2 * expect)
+
+
+def test_check_scales_every_code_and_full_down_table():
+    # Every code once per row (128 bad of 256), then the decode M=256 down
+    # projection's scale table (256 experts of 7168 x 2048) with a few planted codes.
+    _need_gpu()
+    import nvfp4_weight_quantized_moe_b200 as nvm
+    codes = np.tile(np.arange(256, dtype=np.uint8), (16, 1))  # 16 rows x k = 4096
+    _, _, _, t = _scale_table([codes])
+    bad = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nvm.check_scales(t, 1, 16, 4096, bad)
+    torch.cuda.synchronize()
+    assert int(bad.item()) == 16 * 128 == orc.count_bad_scales(codes)
+
+    e, n, k = 256, 7168, 2048
+    rng = np.random.default_rng(77)
+    big = rng.integers(0x18, 0x49, (e, n, k // 16), dtype=np.uint8)
+    flat = big.reshape(-1)
+    idx = rng.integers(0, flat.size, 300)
+    flat[idx] = 0xFF
+    flat[idx[:100]] = 0x80  # -0 passes
+    d = torch.from_numpy(big).cuda()
+    ptrs = torch.tensor([d.data_ptr() + i * d.stride(0) for i in range(e)], dtype=torch.int64,
+                        device="cuda")
+    t = nvm.ExpertTables(ptrs.data_ptr(), ptrs.data_ptr(), None)
+    bad = torch.zeros(e, dtype=torch.int32, device="cuda")
+    nvm.check_scales(t, e, n, k, bad)
+    torch.cuda.synchronize()
+    expect = np.array([orc.count_bad_scales(big[i]) for i in range(e)])
+    np.testing.assert_array_equal(bad.cpu().numpy(), expect)

@@ -446,6 +446,29 @@ def test_shared_expert_as_extra_slots_equals_the_plain_definition():
 
 
 # --------------------------------------------------------------------------- #
+# Load-time scale check
+# --------------------------------------------------------------------------- #
+
+def test_bad_scale_count_against_ml_dtypes_over_every_code():
+    codes = np.arange(256, dtype=np.uint8)
+    lib = codes.view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    expect = [int(np.isnan(v) or v < 0) for v in lib]
+    assert [orc.count_bad_scales(np.array([c], dtype=np.uint8)) for c in codes] == expect
+    # Closed form: 0x7F and 0x81..0xFF fail (NaN 0x7F / 0xFF, negatives between),
+    # 0x00..0x7E and -0 (0x80) pass.
+    assert orc.count_bad_scales(codes) == 128
+    assert orc.count_bad_scales(np.array([0x80, 0x7E, 0x00], dtype=np.uint8)) == 0
+    assert orc.count_bad_scales(np.array([[0x7F, 0x81], [0xFF, 0xFE]], dtype=np.uint8)) == 4
+
+
+def test_bad_scale_count_of_generated_scales_is_zero():
+    prob = make_problem(_tiny_cfg())
+    for m in (MATRIX_GATE, MATRIX_UP, MATRIX_DOWN):
+        _, scale, _ = prob.expert_weight(m, 0)
+        assert orc.count_bad_scales(scale) == 0
+
+
+# --------------------------------------------------------------------------- #
 # transpose_u8
 # --------------------------------------------------------------------------- #
 

@@ -30,12 +30,27 @@ def upload_projection(prob: MoEProblem, matrix: int, device="cuda"):
     return NVFP4Projection(packed, scale, scale2, null_experts=prob.null_experts)
 
 
-def upload_layer(prob: MoEProblem, device="cuda"):
+def upload_shared(prob: MoEProblem, device="cuda"):
+    """The shared expert's three projections, each an NVFP4Projection of one expert."""
+    from nvfp4_weight_quantized_moe_b200 import NVFP4Projection
+
+    out = []
+    for matrix in (MATRIX_GATE, MATRIX_UP, MATRIX_DOWN):
+        p, s, s2 = prob.shared_weight(matrix)
+        out.append(NVFP4Projection(torch.from_numpy(p[None]).to(device),
+                                   torch.from_numpy(s[None]).to(device),
+                                   torch.tensor([float(s2)], dtype=torch.float32, device=device)))
+    return tuple(out)
+
+
+def upload_layer(prob: MoEProblem, device="cuda", shared: bool = False, shared_rows: int = 0):
     from nvfp4_weight_quantized_moe_b200 import NVFP4MoE
 
     return NVFP4MoE(upload_projection(prob, MATRIX_GATE, device),
                     upload_projection(prob, MATRIX_UP, device),
-                    upload_projection(prob, MATRIX_DOWN, device), prob.cfg.topk)
+                    upload_projection(prob, MATRIX_DOWN, device), prob.cfg.topk,
+                    shared=upload_shared(prob, device) if shared else None,
+                    shared_rows=shared_rows)
 
 
 def upload_inputs(prob: MoEProblem, device="cuda"):
