@@ -28,6 +28,8 @@ Sources (rustdoc source pages of the "metrale" project; cited by page and item):
   the E4M3 variant as the finite "FN" one (max 448, no infinities).
 * metrale_model_layers/weight_map/expert.rs, ``ExpertWeight::null``: a NULL
   expert is skipped by the MoE kernels.
+* nvfp4_moe_grouped.rs, doc of ``nvfp4_tc_lean_repack``: a negative or NaN
+  block scale leaves the matrix unusable and is flagged at load time.
 * nvfp4_moe_grouped.rs, docs of the two projection launchers: the shared
   expert runs in the same gate+up and down launches as the routed experts,
   over every token, one row per token, with its own weights; its SiLU product
@@ -48,7 +50,9 @@ Readings where the pages are silent (each also listed in the design notes):
 * a NULL expert's rows of ``act`` and ``y`` are zero;
 * the shared expert has the routed experts' shapes (the fused launches take
   one width pair for both) and its down output joins the token's sum with a
-  per-token weight, 1 unless the caller gives one.
+  per-token weight, 1 unless the caller gives one;
+* a "negative" block scale is one whose value is below zero: -0 (0x80) is
+  valid.
 
 Parity pins for every function live in ``tests/test_oracle_pins.py``.
 """
@@ -79,6 +83,7 @@ __all__ = [
     "shared_expert",
     "moe_forward_shared",
     "append_shared_routing",
+    "count_bad_scales",
     "RouteSort",
 ]
 
@@ -424,6 +429,21 @@ def append_shared_routing(topk_ids, topk_weights, num_experts: int, shared_rows:
         ids_out[t, k] = num_experts + t // shared_rows
         w_out[t, k] = 1.0 if shared_weights is None else np.float32(shared_weights[t])
     return ids_out, w_out
+
+
+# --------------------------------------------------------------------------- #
+# Load-time scale check
+# --------------------------------------------------------------------------- #
+
+def count_bad_scales(scale_codes: np.ndarray) -> int:
+    """Number of E4M3 block-scale codes whose value is NaN or below zero.
+
+    nvfp4_moe_grouped.rs, doc of ``nvfp4_tc_lean_repack``: a negative or NaN
+    block scale makes the matrix unusable.  "Negative" is read as a value
+    below zero, so -0 (0x80) passes.
+    """
+    v = _E4M3[np.asarray(scale_codes, dtype=np.uint8).reshape(-1)]
+    return int(np.count_nonzero(np.isnan(v) | (v < 0.0)))
 
 
 # --------------------------------------------------------------------------- #
