@@ -30,6 +30,9 @@ Sources (rustdoc source pages of the "metrale" project; cited by page and item):
   expert is skipped by the MoE kernels.
 * nvfp4_moe_grouped.rs, doc of ``nvfp4_tc_lean_repack``: a negative or NaN
   block scale leaves the matrix unusable and is flagged at load time.
+* metrale_model_arch/tp_shard/quant_shard.rs, ``shard_quantized_nvfp4``:
+  column-parallel keeps a rank's rows of packed and scale, row-parallel a
+  rank's K slice of both; weight_scale_2 is replicated.
 * nvfp4_moe_grouped.rs, docs of the two projection launchers: the shared
   expert runs in the same gate+up and down launches as the routed experts,
   over every token, one row per token, with its own weights; its SiLU product
@@ -84,6 +87,8 @@ __all__ = [
     "moe_forward_shared",
     "append_shared_routing",
     "count_bad_scales",
+    "shard_nvfp4",
+    "expert_owner_range",
     "RouteSort",
 ]
 
@@ -444,6 +449,60 @@ def count_bad_scales(scale_codes: np.ndarray) -> int:
     """
     v = _E4M3[np.asarray(scale_codes, dtype=np.uint8).reshape(-1)]
     return int(np.count_nonzero(np.isnan(v) | (v < 0.0)))
+
+
+# --------------------------------------------------------------------------- #
+# Sharding across ranks
+# --------------------------------------------------------------------------- #
+
+def shard_nvfp4(packed: np.ndarray, scale: np.ndarray, kind: str, rank: int, tp: int
+                ) -> Tuple[np.ndarray, np.ndarray]:
+    """This rank's part of one NVFP4 weight (packed [N, K/2], scale [N, K/16]).
+
+    metrale_model_arch/tp_shard/quant_shard.rs, ``shard_quantized_nvfp4``:
+    "column" (column-parallel) keeps rows rank*N/tp .. (rank+1)*N/tp - 1 of both
+    tensors; "row" (row-parallel) keeps, in every row, the rank's K/2/tp
+    packed bytes and K/16/tp scale bytes; "replicated" (or tp <= 1) keeps all.
+    weight_scale_2 is per tensor and stays the same on every rank.  The page's
+    divisibility rules raise ValueError.
+    """
+    packed = np.asarray(packed, dtype=np.uint8)
+    scale = np.asarray(scale, dtype=np.uint8)
+    n, half_k = packed.shape
+    k = 2 * half_k
+    if k % E2M1_GROUP:
+        raise ValueError("K is not a multiple of the group size")
+    groups = k // E2M1_GROUP
+    if tp <= 1 or kind == "replicated":
+        return packed.copy(), scale.copy()
+    if not 0 <= rank < tp:
+        raise ValueError("rank out of range")
+    if kind == "column":
+        if n % tp:
+            raise ValueError("N not divisible by tp")
+        rows = n // tp
+        return (packed[rank * rows:(rank + 1) * rows].copy(),
+                scale[rank * rows:(rank + 1) * rows].copy())
+    if kind == "row":
+        if k % tp or half_k % tp or groups % tp:
+            raise ValueError("K, K/2 or K/16 not divisible by tp")
+        wb, sb = half_k // tp, groups // tp
+        return (packed[:, rank * wb:(rank + 1) * wb].copy(),
+                scale[:, rank * sb:(rank + 1) * sb].copy())
+    raise ValueError(f"unknown shard kind {kind!r}")
+
+
+def expert_owner_range(num_experts: int, world: int, rank: int) -> Tuple[int, int]:
+    """[lo, hi): the experts rank owns under expert parallelism, in contiguous blocks.
+
+    The pages fix only that a rank runs the experts it does not own as NULL
+    experts (expert.rs, ``ExpertWeight::null``); the reading taken here is
+    blocks of consecutive ids whose sizes differ by at most one:
+    lo = rank * E // world.
+    """
+    if not 0 <= rank < world:
+        raise ValueError("rank out of range")
+    return rank * num_experts // world, (rank + 1) * num_experts // world
 
 
 # --------------------------------------------------------------------------- #

@@ -469,6 +469,88 @@ def test_bad_scale_count_of_generated_scales_is_zero():
 
 
 # --------------------------------------------------------------------------- #
+# Sharding across ranks
+# --------------------------------------------------------------------------- #
+
+@pytest.mark.parametrize("tp", [2, 3, 4])
+def test_shards_reassemble_and_dequantise_to_slices(tp):
+    rng = np.random.default_rng(tp)
+    n, k = 24, 192  # K/16 = 12 and N divisible by 2, 3, 4
+    packed = rng.integers(0, 256, (n, k // 2), dtype=np.uint8)
+    scale = rng.integers(0x18, 0x49, (n, k // 16), dtype=np.uint8)
+    s2 = np.float32(0.75)
+    full = orc.dequantize_nvfp4(packed, scale, s2)
+    cols = [orc.shard_nvfp4(packed, scale, "column", r, tp) for r in range(tp)]
+    np.testing.assert_array_equal(np.vstack([c[0] for c in cols]), packed)
+    np.testing.assert_array_equal(np.vstack([c[1] for c in cols]), scale)
+    rows = [orc.shard_nvfp4(packed, scale, "row", r, tp) for r in range(tp)]
+    np.testing.assert_array_equal(np.hstack([r_[0] for r_ in rows]), packed)
+    np.testing.assert_array_equal(np.hstack([r_[1] for r_ in rows]), scale)
+    for r in range(tp):
+        # A row shard is the rank's K slice of the dense weight; a column shard its rows.
+        np.testing.assert_array_equal(orc.dequantize_nvfp4(*rows[r], s2),
+                                      full[:, r * k // tp:(r + 1) * k // tp])
+        np.testing.assert_array_equal(orc.dequantize_nvfp4(*cols[r], s2),
+                                      full[r * n // tp:(r + 1) * n // tp])
+
+
+def test_shard_rules_follow_the_page():
+    packed = np.zeros((6, 40), dtype=np.uint8)  # K = 80: K/16 = 5
+    scale = np.zeros((6, 5), dtype=np.uint8)
+    with pytest.raises(ValueError):
+        orc.shard_nvfp4(packed, scale, "row", 0, 2)  # K/16 = 5 not divisible by 2
+    with pytest.raises(ValueError):
+        orc.shard_nvfp4(packed, scale, "column", 0, 4)  # N = 6 not divisible by 4
+    p, s_ = orc.shard_nvfp4(packed, scale, "replicated", 1, 4)
+    assert p.shape == packed.shape and s_.shape == scale.shape
+
+
+def _sharded_fns(prob, tp, rank):
+    """Weight callbacks of one tensor-parallel rank: gate/up by rows, down by K."""
+    def fn(m):
+        kind = "row" if m == MATRIX_DOWN else "column"
+
+        def get(e):
+            w = prob.expert_weight(m, e)
+            if w is None:
+                return None
+            p, s_ = orc.shard_nvfp4(w[0], w[1], kind, rank, tp)
+            return p, s_, w[2]
+        return get
+    return [fn(m) for m in (MATRIX_GATE, MATRIX_UP, MATRIX_DOWN)]
+
+
+@pytest.mark.parametrize("tp", [2, 4])
+def test_tensor_parallel_partial_outputs_sum_to_the_full_forward(tp):
+    prob = make_problem(_tiny_cfg(tokens=6, experts=4, topk=2, hidden=64, inter=64, seed=31))
+    cfg = prob.cfg
+    full = _run(prob)["out"]
+    total = np.zeros_like(full)
+    for r in range(tp):
+        res = orc.moe_forward(prob.x_bf16, prob.topk_ids, prob.topk_weights, cfg.experts,
+                              *_sharded_fns(prob, tp, r), hidden=cfg.hidden,
+                              inter=cfg.inter // tp)
+        total += res["out"]
+    np.testing.assert_allclose(total, full, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("world", [2, 3, 8])
+def test_expert_parallel_partial_outputs_sum_to_the_full_forward(world):
+    cfg = _tiny_cfg(tokens=7, experts=8, topk=3, hidden=64, inter=48, seed=32)
+    full = _run(make_problem(cfg))["out"]
+    total = np.zeros_like(full)
+    owned = []
+    for r in range(world):
+        lo, hi = orc.expert_owner_range(cfg.experts, world, r)
+        owned += list(range(lo, hi))
+        assert hi - lo in (cfg.experts // world, -(-cfg.experts // world))
+        prob = make_problem(cfg, null_experts=[e for e in range(cfg.experts) if not lo <= e < hi])
+        total += _run(prob)["out"]
+    assert owned == list(range(cfg.experts))
+    np.testing.assert_allclose(total, full, rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------- #
 # transpose_u8
 # --------------------------------------------------------------------------- #
 
