@@ -63,9 +63,11 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--op", choices=["layer", "check_scales"], default="layer",
-                    help="layer: the forward; check_scales: the load-time scale check over the "
-                         "workload's three projections")
+    ap.add_argument("--op", choices=["layer", "check_scales", "shard"], default="layer",
+                    help="layer: the forward; check_scales / shard: the load-time scale check / "
+                         "tensor-parallel shard (--tp ranks, rank 0) of the workload's three "
+                         "projections")
+    ap.add_argument("--tp", type=int, default=2, help="tensor-parallel ranks for --op shard")
     ap.add_argument("--shared", action="store_true",
                     help="add a shared expert (every token, same launches as the routed experts)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -564,9 +566,11 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def run_check_scales(args, rank, world, local):
-    """nvfp4_moe_check_scales over the gate, up and down scale tables of every
-    expert of the workload (one launch per projection, HBM-bound byte scan)."""
+def run_load_op(args, rank, world, local):
+    """A load-time op over the gate, up and down weights of every expert of the
+    workload, one library call per projection: nvfp4_moe_check_scales (an
+    HBM-bound byte scan of the scale tables) or nvfp4_moe_shard_nvfp4 (rank 0's
+    tensor-parallel shard: gate / up by rows, down by K; bytes read + written)."""
     import torch
     import nvfp4_weight_quantized_moe_b200 as nvm
     from workloads import make_problem
@@ -580,11 +584,22 @@ def run_check_scales(args, rank, world, local):
     projs = (layer.gate, layer.up, layer.down)
     bad = torch.zeros(3, cfg.experts, dtype=torch.int32, device=dev)
     stream = torch.cuda.Stream(device=dev)
-    scale_bytes = sum(p.scale.numel() for p in projs)
+    shard = args.op == "shard"
+    if shard:
+        kinds = (nvm.SHARD_COLUMN, nvm.SHARD_COLUMN, nvm.SHARD_ROW)
+        outs = [nvm.shard_nvfp4(p.packed, p.scale, kd, 0, args.tp) for p, kd in zip(projs, kinds)]
+        moved = 2 * sum(o[0].numel() + o[1].numel() for o in outs)  # read + written
+    else:
+        moved = sum(p.scale.numel() for p in projs)
+    scale_bytes = moved
 
     def one():
         for i, p in enumerate(projs):
-            nvm.check_scales(p.tables, cfg.experts, p.n, p.k, bad[i], stream=stream)
+            if shard:
+                nvm.shard_nvfp4_into(p.packed, p.scale, kinds[i], 0, args.tp, outs[i][0],
+                                     outs[i][1], stream=stream)
+            else:
+                nvm.check_scales(p.tables, cfg.experts, p.n, p.k, bad[i], stream=stream)
 
     steps = args.steps if args.steps is not None else 200
     warmup = max(args.warmup, 3)
@@ -615,17 +630,21 @@ def run_check_scales(args, rank, world, local):
     hbm, _, _, peak_kind = measured_peaks()
     gbs = scale_bytes / (ms * 1e-3) / 1e9
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    what = (f"NVFP4 tensor-parallel shard GB/s (load time, tp={args.tp}, read + written)" if shard
+            else "NVFP4 block-scale check GB/s (load time)")
     line = {
-        "metric": "NVFP4 block-scale check GB/s (load time)", "value": gbs, "unit": "GB/s",
+        "metric": what, "value": gbs, "unit": "GB/s",
         "n_gpus": 1, "steps": steps, "warmup": warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic",
-        "config": {"workload": cfg.name + " scale tables", "experts": cfg.experts,
-                   "bytes_per_step": scale_bytes,
-                   "l2": f"three tables of {scale_bytes / 3e6:.0f} MB each, L2 {l2 / 1e6:.0f} MB"},
-        "roofline": {"kernel": "check_scales_kernel", "bound": "hbm", "achieved": gbs, "peak": hbm,
+        "config": {"workload": cfg.name + (" weights" if shard else " scale tables"),
+                   "experts": cfg.experts, "bytes_per_step": scale_bytes,
+                   "l2": f"three projections, {scale_bytes / 3e6:.0f} MB moved each, "
+                         f"L2 {l2 / 1e6:.0f} MB"},
+        "roofline": {"kernel": "shard_copy_kernel" if shard else "check_scales_kernel",
+                     "bound": "hbm", "achieved": gbs, "peak": hbm,
                      "unit": "GB/s", "frac": gbs / hbm, "peak_source": f"{peak_kind} HBM copy",
                      "traffic": None},
-        "gpu_launches": 3 * steps,
+        "gpu_launches": (6 if shard else 3) * steps,
         "clocks": clocks,
     }
     if rank == 0:
@@ -638,8 +657,8 @@ def main(argv=None):
     if args.impl == "reference":
         run_reference(args, rank, world)
         return
-    if args.op == "check_scales":
-        run_check_scales(args, rank, world, local)
+    if args.op in ("check_scales", "shard"):
+        run_load_op(args, rank, world, local)
         return
     run_ours(args, rank, world, local)
 

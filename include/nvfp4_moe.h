@@ -384,6 +384,33 @@ NVFP4_MOE_API uint32_t nvfp4_moe_shared_slots(uint32_t num_tokens, uint32_t shar
 NVFP4_MOE_API int nvfp4_moe_check_scales(nvfp4_expert_tables t, uint32_t num_experts, uint32_t n,
                                          uint32_t k, uint32_t* bad, cudaStream_t stream);
 
+/*
+ * Tensor-parallel shard of NVFP4 weights at load time (shard_quantized_nvfp4 in
+ * metrale_model_arch/tp_shard/quant_shard.rs).  A stack of num_matrices
+ * matrices [n, k]: packed u8 [num_matrices, n, k/2], scale u8
+ * [num_matrices, n, k/16], back to back.  Writes this rank's part of each into
+ * packed_out / scale_out, stacked the same way:
+ *   NVFP4_MOE_SHARD_COLUMN  rows rank*n/tp .. (rank+1)*n/tp - 1 of both tensors
+ *                           (gate / up: each rank holds n/tp intermediate rows);
+ *                           out [num_matrices, n/tp, k/2] and [.., n/tp, k/16]
+ *   NVFP4_MOE_SHARD_ROW     in every row, bytes rank*k/2/tp .. of packed and
+ *                           rank*k/16/tp .. of scale (down: each rank holds k/tp
+ *                           of the intermediate); out [.., n, k/2/tp], [.., n, k/16/tp]
+ * weight_scale_2 is per tensor and the same on every rank (not touched here).
+ * tp = 1 copies the whole stack.  A rank's partial outputs of the forward then
+ * sum over ranks to the unsharded result (one all-reduce of out).
+ * ESHAPE: k % 16, n % tp (column), k % tp, (k/2) % tp or (k/16) % tp (row).
+ * EINVAL: bad kind, tp == 0, rank >= tp, NULL or overlapping buffers.
+ * The forward's own shape rules (multiples of 256 for k, 64 / 128 for n)
+ * apply to the shards.  Bit-exact.
+ */
+typedef enum { NVFP4_MOE_SHARD_COLUMN = 0, NVFP4_MOE_SHARD_ROW = 1 } nvfp4_moe_shard_kind;
+
+NVFP4_MOE_API int nvfp4_moe_shard_nvfp4(const uint8_t* packed, const uint8_t* scale,
+                                        uint32_t num_matrices, uint32_t n, uint32_t k, int kind,
+                                        uint32_t rank, uint32_t tp, uint8_t* packed_out,
+                                        uint8_t* scale_out, cudaStream_t stream);
+
 /* Host helper: launch bound on active experts, min(num_experts, num_pairs). */
 NVFP4_MOE_API uint32_t nvfp4_moe_active_cap(uint32_t num_experts, uint32_t num_pairs);
 

@@ -10,6 +10,8 @@ from ._binding import (  # noqa: F401
     PATH_AUTO,
     PATH_DECODE,
     PATH_PREFILL,
+    SHARD_COLUMN,
+    SHARD_ROW,
     Buffers,
     ExpertTables,
     LaunchOpts,
@@ -26,8 +28,16 @@ from ._binding import (  # noqa: F401
     gate_up_silu,
     gate_up_silu_ws,
     route_sort,
+    shard_nvfp4,
+    shard_nvfp4_into,
     shared_slots,
     transpose_u8,
     workspace_bytes,
 )
-from .layer import MoEBuffers, NVFP4MoE, NVFP4Projection  # noqa: F401
+from .layer import (  # noqa: F401
+    MoEBuffers,
+    NVFP4MoE,
+    NVFP4Projection,
+    all_reduce_out,
+    expert_owner_range,
+)

@@ -50,6 +50,7 @@ class Buffers(ctypes.Structure):
 
 
 PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
+SHARD_COLUMN, SHARD_ROW = 0, 1
 
 _sig = {
     "nvfp4_moe_route_sort": (c_int, [c_void_p, c_u32, c_u32, c_u32, c_void_p, c_void_p, c_void_p,
@@ -86,6 +87,8 @@ _sig = {
                                         c_void_p, c_void_p, c_void_p]),
     "nvfp4_moe_shared_slots": (c_u32, [c_u32, c_u32]),
     "nvfp4_moe_check_scales": (c_int, [ExpertTables, c_u32, c_u32, c_u32, c_void_p, c_void_p]),
+    "nvfp4_moe_shard_nvfp4": (c_int, [c_void_p, c_void_p, c_u32, c_u32, c_u32, c_int, c_u32, c_u32,
+                                      c_void_p, c_void_p, c_void_p]),
     "nvfp4_moe_workspace_bytes": (ctypes.c_size_t, [c_u32, c_u32, c_u32, c_u32]),
     "nvfp4_moe_device_error": (c_int, [c_int]),
     "nvfp4_moe_active_cap": (c_u32, [c_u32, c_u32]),
@@ -231,6 +234,42 @@ def check_scales(tables: ExpertTables, num_experts, n, k, bad, stream=None) -> N
         raise TypeError("bad: expected 32-bit counters")
     _check("nvfp4_moe_check_scales", _lib.nvfp4_moe_check_scales(
         tables, num_experts, n, k, _ptr(bad, None, "bad"), _stream(stream)))
+
+
+def shard_nvfp4(packed, scale, kind: int, rank: int, tp: int, stream=None):
+    """nvfp4_moe_shard_nvfp4 over a stack [E, N, K/2] / [E, N, K/16] (or one [N, K/2]
+    matrix): returns this rank's packed and scale tensors, newly allocated."""
+    squeeze = packed.dim() == 2
+    p3 = packed.unsqueeze(0) if squeeze else packed
+    s3 = scale.unsqueeze(0) if squeeze else scale
+    e, n, half_k = p3.shape
+    k = 2 * half_k
+    if tuple(s3.shape) != (e, n, k // 16):
+        raise ValueError("scale must be [E, N, K/16]")
+    if kind == SHARD_COLUMN:
+        if tp < 1 or n % tp:
+            raise ValueError("N must be divisible by tp")
+        po = torch.empty((e, n // tp, half_k), dtype=torch.uint8, device=packed.device)
+        so = torch.empty((e, n // tp, k // 16), dtype=torch.uint8, device=packed.device)
+    elif kind == SHARD_ROW:
+        if tp < 1 or half_k % tp or (k // 16) % tp:
+            raise ValueError("K/2 and K/16 must be divisible by tp")
+        po = torch.empty((e, n, half_k // tp), dtype=torch.uint8, device=packed.device)
+        so = torch.empty((e, n, k // 16 // tp), dtype=torch.uint8, device=packed.device)
+    else:
+        raise ValueError("kind must be SHARD_COLUMN or SHARD_ROW")
+    shard_nvfp4_into(p3, s3, kind, rank, tp, po, so, stream=stream)
+    return (po[0], so[0]) if squeeze else (po, so)
+
+
+def shard_nvfp4_into(packed, scale, kind: int, rank: int, tp: int, packed_out, scale_out,
+                     stream=None) -> None:
+    """nvfp4_moe_shard_nvfp4 into caller-allocated [E, ...] outputs."""
+    e, n, half_k = packed.shape
+    _check("nvfp4_moe_shard_nvfp4", _lib.nvfp4_moe_shard_nvfp4(
+        _ptr(packed, torch.uint8, "packed"), _ptr(scale, torch.uint8, "scale"), e, n, 2 * half_k,
+        kind, rank, tp, _ptr(packed_out, torch.uint8, "packed_out"),
+        _ptr(scale_out, torch.uint8, "scale_out"), _stream(stream)))
 
 
 def workspace_bytes(num_tokens, topk, hidden, inter) -> int:

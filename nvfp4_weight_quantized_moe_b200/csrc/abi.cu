@@ -413,6 +413,44 @@ int nvfp4_moe_check_scales(nvfp4_expert_tables t, uint32_t num_experts, uint32_t
                                        (uint64_t)n * (k / 16), bad, stream));
 }
 
+int nvfp4_moe_shard_nvfp4(const uint8_t* packed, const uint8_t* scale, uint32_t num_matrices,
+                          uint32_t n, uint32_t k, int kind, uint32_t rank, uint32_t tp,
+                          uint8_t* packed_out, uint8_t* scale_out, cudaStream_t stream) {
+  if (kind != NVFP4_MOE_SHARD_COLUMN && kind != NVFP4_MOE_SHARD_ROW) return NVFP4_MOE_EINVAL;
+  if (tp == 0 || rank >= tp) return NVFP4_MOE_EINVAL;
+  if (k % 16 != 0) return NVFP4_MOE_ESHAPE;
+  const uint32_t half_k = k / 2, groups = k / 16;
+  if (kind == NVFP4_MOE_SHARD_COLUMN && n % tp != 0) return NVFP4_MOE_ESHAPE;
+  if (kind == NVFP4_MOE_SHARD_ROW && (k % tp != 0 || half_k % tp != 0 || groups % tp != 0))
+    return NVFP4_MOE_ESHAPE;
+  if (num_matrices == 0 || n == 0 || k == 0) return NVFP4_MOE_OK;
+  if (packed == nullptr || scale == nullptr || packed_out == nullptr || scale_out == nullptr)
+    return NVFP4_MOE_EINVAL;
+  const uint64_t mats = num_matrices;
+  auto overlaps = [](const void* a, uint64_t na, const void* b, uint64_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+  };
+  const uint64_t pin = mats * n * half_k, sin = mats * n * groups;
+  const uint64_t pout = pin / tp, sout = sin / tp;
+  if (overlaps(packed, pin, packed_out, pout) || overlaps(scale, sin, scale_out, sout) ||
+      overlaps(packed, pin, scale_out, sout) || overlaps(scale, sin, packed_out, pout))
+    return NVFP4_MOE_EINVAL;
+  cudaError_t err;
+  if (kind == NVFP4_MOE_SHARD_COLUMN) {
+    const uint32_t rows = n / tp;
+    err = launch_shard_copy(packed, packed_out, mats, n, half_k, rows, half_k, rank * rows, 0, stream);
+    if (err == cudaSuccess)
+      err = launch_shard_copy(scale, scale_out, mats, n, groups, rows, groups, rank * rows, 0, stream);
+  } else {
+    const uint32_t wb = half_k / tp, sb = groups / tp;
+    err = launch_shard_copy(packed, packed_out, mats, n, half_k, n, wb, 0, rank * wb, stream);
+    if (err == cudaSuccess)
+      err = launch_shard_copy(scale, scale_out, mats, n, groups, n, sb, 0, rank * sb, stream);
+  }
+  return status_of(err);
+}
+
 int nvfp4_moe_transpose_u8(const uint8_t* src, uint8_t* dst, uint32_t rows, uint32_t cols,
                            cudaStream_t stream) {
   if (rows == 0 || cols == 0) return NVFP4_MOE_OK;

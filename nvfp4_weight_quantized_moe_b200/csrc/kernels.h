@@ -72,6 +72,10 @@ cudaError_t launch_check_scales(const void* const* packed_ptrs, const void* cons
                                 uint32_t num_experts, uint64_t bytes_per_expert, uint32_t* bad,
                                 cudaStream_t stream);
 
+cudaError_t launch_shard_copy(const uint8_t* src, uint8_t* dst, uint64_t mats, uint32_t rows_src,
+                              uint32_t cols_src, uint32_t rows_out, uint32_t cols_out,
+                              uint32_t row_off, uint32_t col_off, cudaStream_t stream);
+
 cudaError_t launch_transpose_u8(const uint8_t* src, uint8_t* dst, uint32_t rows, uint32_t cols,
                                 cudaStream_t stream);
 

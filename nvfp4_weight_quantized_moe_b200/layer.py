@@ -1,7 +1,11 @@
 """Device-side containers for one NVFP4 MoE layer and its four-call forward.
 
 PyTorch here only owns device memory and supplies the stream; every step of
-the forward is one call into the C ABI (``_binding``).
+the forward is one call into the C ABI (``_binding``).  Sharding across ranks
+is set up here too: tensor-parallel shards of the weights (one library call
+per projection) and expert-parallel blocks (NULL table entries for the experts
+a rank does not hold); either way a rank's ``out`` is a partial sum that one
+all-reduce completes (:func:`all_reduce_out`).
 """
 
 from __future__ import annotations
@@ -13,17 +17,38 @@ import torch
 from . import _binding as B
 
 
+def expert_owner_range(num_experts: int, world: int, rank: int):
+    """[lo, hi): the block of consecutive experts rank holds under expert
+    parallelism; block sizes differ by at most one (lo = rank * E // world)."""
+    if not 0 <= rank < world:
+        raise ValueError("rank out of range")
+    return rank * num_experts // world, (rank + 1) * num_experts // world
+
+
+def all_reduce_out(out: torch.Tensor, group=None) -> torch.Tensor:
+    """Sum a rank's partial ``out`` over the process group (in place).
+
+    Expert- and tensor-parallel ranks each produce a partial sum of the layer
+    output; one all-reduce (NCCL on GPUs) completes it on every rank."""
+    import torch.distributed as dist
+    dist.all_reduce(out, op=dist.ReduceOp.SUM, group=group)
+    return out
+
+
 class NVFP4Projection:
     """One NVFP4 projection for every expert, resident on the device.
 
-    packed  u8  [E, N, K/2]  packed E2M1 codes, low nibble = even k
-    scale   u8  [E, N, K/16] E4M3 block scales
-    scale2  f32 [E]          weight_scale_2 per expert
-    Experts listed in ``null_experts`` get NULL table entries (skipped).
+    packed  u8  [B, N, K/2]  packed E2M1 codes, low nibble = even k
+    scale   u8  [B, N, K/16] E4M3 block scales
+    scale2  f32 [B]          weight_scale_2 per expert
+    The tables list ``num_experts`` experts (default B); expert e in
+    [first_expert, first_expert + B) is packed[e - first_expert], every other
+    one, and those in ``null_experts``, a NULL entry (skipped by the forward).
     """
 
     def __init__(self, packed: torch.Tensor, scale: torch.Tensor, scale2: torch.Tensor,
-                 null_experts: Iterable[int] = ()):
+                 null_experts: Iterable[int] = (), first_expert: int = 0,
+                 num_experts: Optional[int] = None):
         if packed.dtype != torch.uint8 or scale.dtype != torch.uint8:
             raise TypeError("packed and scale must be uint8")
         if packed.device.type != "cuda":
@@ -31,13 +56,25 @@ class NVFP4Projection:
         e, n, half_k = packed.shape
         if tuple(scale.shape) != (e, n, half_k * 2 // 16):
             raise ValueError("scale shape must be [E, N, K/16]")
+        total = e if num_experts is None else int(num_experts)
+        if first_expert < 0 or first_expert + e > total:
+            raise ValueError("expert block outside the table")
         self.packed = packed.contiguous()
         self.scale = scale.contiguous()
-        self.scale2 = scale2.to(device=packed.device, dtype=torch.float32).contiguous()
-        self.num_experts, self.n, self.k = e, n, half_k * 2
+        s2 = scale2.to(device=packed.device, dtype=torch.float32).reshape(-1)
+        if s2.numel() != e:
+            raise ValueError("scale2 must hold one value per expert of the block")
+        self.first_expert = first_expert
+        self.num_experts, self.n, self.k = total, n, half_k * 2
         null = set(int(i) for i in null_experts)
-        pp = [0 if i in null else self.packed.data_ptr() + i * self.packed.stride(0) for i in range(e)]
-        sp = [0 if i in null else self.scale.data_ptr() + i * self.scale.stride(0) for i in range(e)]
+        held = lambda i: first_expert <= i < first_expert + e and i not in null
+        pp = [self.packed.data_ptr() + (i - first_expert) * self.packed.stride(0) if held(i) else 0
+              for i in range(total)]
+        sp = [self.scale.data_ptr() + (i - first_expert) * self.scale.stride(0) if held(i) else 0
+              for i in range(total)]
+        s2_full = torch.zeros(total, dtype=torch.float32, device=packed.device)
+        s2_full[first_expert:first_expert + e] = s2
+        self.scale2 = s2_full
         self.packed_ptrs = torch.tensor(pp, dtype=torch.int64, device=packed.device)
         self.scale_ptrs = torch.tensor(sp, dtype=torch.int64, device=packed.device)
         self.tables = B.ExpertTables(self.packed_ptrs.data_ptr(), self.scale_ptrs.data_ptr(),
@@ -47,6 +84,25 @@ class NVFP4Projection:
     def nbytes_per_expert(self) -> int:
         """Packed nibbles + block scales of one expert (the bytes a pass must read)."""
         return self.n * self.k // 2 + self.n * self.k // 16
+
+    def expert_block(self, lo: int, hi: int) -> "NVFP4Projection":
+        """A projection holding copies of experts [lo, hi) only, the others NULL
+        (what an expert-parallel rank keeps resident)."""
+        f = self.first_expert
+        if not f <= lo <= hi <= f + self.packed.shape[0]:
+            raise ValueError("experts not held by this projection")
+        return NVFP4Projection(self.packed[lo - f:hi - f].clone(), self.scale[lo - f:hi - f].clone(),
+                               self.scale2[lo:hi].clone(), first_expert=lo,
+                               num_experts=self.num_experts)
+
+    def shard(self, kind: int, rank: int, tp: int) -> "NVFP4Projection":
+        """This tensor-parallel rank's shard (``B.SHARD_COLUMN``: N / tp rows;
+        ``B.SHARD_ROW``: K / tp of every row), in one library call."""
+        if self.first_expert != 0 or self.packed.shape[0] != self.num_experts:
+            raise ValueError("shard a projection that holds every expert")
+        packed, scale = B.shard_nvfp4(self.packed, self.scale, kind, rank, tp)
+        null = (self.packed_ptrs == 0).nonzero().flatten().tolist()
+        return NVFP4Projection(packed, scale, self.scale2.clone(), null_experts=null)
 
 
 class MoEBuffers:
@@ -127,6 +183,31 @@ class NVFP4MoE:
                     raise ValueError("the shared expert is one expert with the routed shapes")
             self.shared = (sg, su, sd)
         self._ext = {}
+
+    # -- sharding across ranks ---------------------------------------------------
+    def tensor_parallel(self, rank: int, tp: int) -> "NVFP4MoE":
+        """This rank's layer under tensor parallelism: gate and up keep I / tp rows
+        (column-parallel), down I / tp of its K (row-parallel), as
+        shard_quantized_nvfp4 in quant_shard.rs; the shared expert likewise.  The
+        rank's ``out`` is a partial sum (see :func:`all_reduce_out`)."""
+        col, row = B.SHARD_COLUMN, B.SHARD_ROW
+        shared = None
+        if self.shared is not None:
+            sg, su, sd = self.shared
+            shared = (sg.shard(col, rank, tp), su.shard(col, rank, tp), sd.shard(row, rank, tp))
+        return NVFP4MoE(self.gate.shard(col, rank, tp), self.up.shard(col, rank, tp),
+                        self.down.shard(row, rank, tp), self.topk, shared=shared,
+                        shared_rows=self.shared_rows)
+
+    def expert_parallel(self, rank: int, world: int) -> "NVFP4MoE":
+        """This rank's layer under expert parallelism: copies of its block of
+        experts (:func:`expert_owner_range`), NULL entries for the rest.  The
+        shared expert, if any, runs on rank 0 only.  The rank's ``out`` is a
+        partial sum (see :func:`all_reduce_out`)."""
+        lo, hi = expert_owner_range(self.num_experts, world, rank)
+        projs = [p.expert_block(lo, hi) for p in (self.gate, self.up, self.down)]
+        shared = self.shared if rank == 0 else None
+        return NVFP4MoE(*projs, self.topk, shared=shared, shared_rows=self.shared_rows)
 
     # -- shared expert bookkeeping ------------------------------------------------
     def rows_per_shared_slot(self, num_tokens: int) -> int:

@@ -144,3 +144,32 @@ def test_shared_and_scale_check_calls_validate_on_the_host(lib):
     assert L.nvfp4_moe_check_scales(t, 1025, 128, 256, p8, None) == 2
     assert L.nvfp4_moe_check_scales(t, 4, 128, 256, None, None) == 1
     assert L.nvfp4_moe_check_scales(B.ExpertTables(None, 8, None), 4, 128, 256, p8, None) == 1
+
+
+def test_shard_call_validates_on_the_host(lib):
+    import nvfp4_weight_quantized_moe_b200._binding as B
+    L = B._lib
+    a, b, c, d = (ctypes.c_void_p(1 << 20), ctypes.c_void_p(2 << 20), ctypes.c_void_p(3 << 20),
+                  ctypes.c_void_p(4 << 20))
+    col, row = B.SHARD_COLUMN, B.SHARD_ROW
+    assert L.nvfp4_moe_shard_nvfp4(a, b, 1, 64, 256, 7, 0, 2, c, d, None) == 1   # bad kind
+    assert L.nvfp4_moe_shard_nvfp4(a, b, 1, 64, 256, col, 2, 2, c, d, None) == 1  # rank >= tp
+    assert L.nvfp4_moe_shard_nvfp4(a, b, 1, 64, 256, col, 0, 0, c, d, None) == 1  # tp = 0
+    assert L.nvfp4_moe_shard_nvfp4(a, b, 1, 64, 100, col, 0, 2, c, d, None) == 2  # k % 16
+    assert L.nvfp4_moe_shard_nvfp4(a, b, 1, 66, 256, col, 0, 4, c, d, None) == 2  # n % tp
+    assert L.nvfp4_moe_shard_nvfp4(a, b, 1, 64, 80, row, 0, 2, c, d, None) == 2   # k/16 = 5
+    assert L.nvfp4_moe_shard_nvfp4(a, b, 0, 64, 256, row, 0, 2, c, d, None) == 0  # nothing to do
+    assert L.nvfp4_moe_shard_nvfp4(a, None, 1, 64, 256, row, 0, 2, c, d, None) == 1
+    assert L.nvfp4_moe_shard_nvfp4(a, b, 1, 64, 256, row, 0, 2, ctypes.c_void_p((1 << 20) + 64),
+                                   d, None) == 1  # output overlaps the input
+
+
+def test_expert_owner_blocks_match_the_oracle():
+    import oracle as orc
+    from nvfp4_weight_quantized_moe_b200 import expert_owner_range
+    for e in (1, 7, 8, 128, 256, 1000):
+        for world in (1, 2, 3, 8):
+            if world > e:
+                continue
+            for r in range(world):
+                assert expert_owner_range(e, world, r) == orc.expert_owner_range(e, world, r)

@@ -620,3 +620,78 @@ def test_check_scales_every_code_and_full_down_table():
     torch.cuda.synchronize()
     expect = np.array([orc.count_bad_scales(big[i]) for i in range(e)])
     np.testing.assert_array_equal(bad.cpu().numpy(), expect)
+
+
+# --------------------------------------------------------------------------- #
+# Sharding across ranks, each rank's forward run in turn on this GPU
+# --------------------------------------------------------------------------- #
+
+@pytest.mark.parametrize("kind", ["column", "row"])
+@pytest.mark.parametrize("e,n,k,tp", [(3, 96, 512, 2), (2, 48, 768, 3), (1, 64, 320, 5),
+                                       (4, 256, 1536, 6), (2, 26, 208, 13)])
+def test_shard_nvfp4_bit_exact(kind, e, n, k, tp):
+    _need_gpu()
+    import nvfp4_weight_quantized_moe_b200 as nvm
+    if kind == "column" and n % tp or kind == "row" and ((k // 2) % tp or (k // 16) % tp):
+        pytest.skip("shape not shardable at this tp")
+    rng = np.random.default_rng(e * n + k + tp)
+    packed = rng.integers(0, 256, (e, n, k // 2), dtype=np.uint8)
+    scale = rng.integers(0, 256, (e, n, k // 16), dtype=np.uint8)
+    dp, ds = torch.from_numpy(packed).cuda(), torch.from_numpy(scale).cuda()
+    code = nvm.SHARD_COLUMN if kind == "column" else nvm.SHARD_ROW
+    for r in range(tp):
+        po, so = nvm.shard_nvfp4(dp, ds, code, r, tp)
+        torch.cuda.synchronize()
+        for i in range(e):
+            ep, es = orc.shard_nvfp4(packed[i], scale[i], kind, r, tp)
+            np.testing.assert_array_equal(po[i].cpu().numpy(), ep)
+            np.testing.assert_array_equal(so[i].cpu().numpy(), es)
+
+
+# I / tp stays a multiple of 256 for tp = 2, 3, 6 (the down projection's K rule).
+SHARD_CFG = MoEConfig("shard", hidden=512, inter=1536, experts=6, topk=2, tokens=9,
+                      router="uniform", seed=51)
+
+
+def _sum_over_ranks(prob, layers, ws, shared=False, **opts):
+    from workloads.device import upload_inputs
+    import nvfp4_weight_quantized_moe_b200 as nvm
+    x, ids, w = upload_inputs(prob)
+    total = torch.zeros((prob.cfg.tokens, prob.cfg.hidden), dtype=torch.float64, device="cuda")
+    for lay in layers:
+        bufs = lay.buffers(prob.cfg.tokens)
+        bufs.out.fill_(float("nan"))
+        workspace = lay.workspace(prob.cfg.tokens) if ws else None
+        lay.forward(x, ids, w, bufs, workspace=workspace, **opts)
+        total += bufs.out[: prob.cfg.tokens].double()
+    torch.cuda.synchronize()
+    assert nvm.device_error() == 0
+    return total.cpu().numpy()
+
+
+@pytest.mark.parametrize("ws", [False, True], ids=["decode-path", "tcgen05"])
+@pytest.mark.parametrize("tp", [2, 3, 6])
+def test_tensor_parallel_ranks_sum_to_the_full_forward(tp, ws):
+    _need_gpu()
+    from workloads.device import upload_layer
+    prob = make_problem(SHARD_CFG)
+    cfg = prob.cfg
+    full = upload_layer(prob, shared=True)
+    layers = [full.tensor_parallel(r, tp) for r in range(tp)]
+    assert layers[0].inter == cfg.inter // tp
+    got = _sum_over_ranks(prob, layers, ws, **(dict(path=2) if ws else {}))
+    ref = _shared_ref(prob, None)["out"]
+    _close(got, ref, f"sum of {tp} tensor-parallel ranks")
+
+
+@pytest.mark.parametrize("ws", [False, True], ids=["decode-path", "tcgen05"])
+@pytest.mark.parametrize("world", [2, 4])
+def test_expert_parallel_ranks_sum_to_the_full_forward(world, ws):
+    _need_gpu()
+    from workloads.device import upload_layer
+    prob = make_problem(SHARD_CFG)
+    full = upload_layer(prob, shared=True)
+    layers = [full.expert_parallel(r, world) for r in range(world)]
+    got = _sum_over_ranks(prob, layers, ws, **(dict(path=2) if ws else {}))
+    ref = _shared_ref(prob, None)["out"]
+    _close(got, ref, f"sum of {world} expert-parallel ranks")

@@ -60,3 +60,66 @@ def test_bench_cli_defaults():
     args = bench.parse_args([])
     assert args.gpus == 1 and args.config == "decode_m1" and args.impl == "ours"
     assert args.warmup >= 3
+
+
+def _sharded_worker(rank, world, port, mode, results):
+    """One rank: its partial forward from the oracle (no GPU here), then the
+    package's all-reduce of ``out`` over gloo."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    from datetime import timedelta
+    import numpy as np
+    import torch
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        import oracle as orc
+        from nvfp4_weight_quantized_moe_b200 import all_reduce_out, expert_owner_range
+        from workloads import make_problem
+        from workloads.generators import MoEConfig
+        cfg = MoEConfig("shard", hidden=64, inter=64, experts=6, topk=2, tokens=5,
+                        router="uniform", seed=41)
+        inter = cfg.inter
+        if mode == "ep":
+            lo, hi = expert_owner_range(cfg.experts, world, rank)
+            prob = make_problem(cfg, null_experts=[e for e in range(cfg.experts) if not lo <= e < hi])
+            fns = [lambda e, m=m: prob.expert_weight(m, e) for m in (0, 1, 2)]
+        else:
+            prob = make_problem(cfg)
+            inter = cfg.inter // world
+
+            def fn(m):
+                kind = "row" if m == 2 else "column"
+
+                def get(e):
+                    p, s, s2 = prob.expert_weight(m, e)
+                    return (*orc.shard_nvfp4(p, s, kind, rank, world), s2)
+                return get
+            fns = [fn(m) for m in (0, 1, 2)]
+        part = orc.moe_forward(prob.x_bf16, prob.topk_ids, prob.topk_weights, cfg.experts, *fns,
+                               hidden=cfg.hidden, inter=inter)["out"]
+        out = torch.from_numpy(part.copy())
+        all_reduce_out(out)
+        full_prob = make_problem(cfg)
+        full = orc.moe_forward(full_prob.x_bf16, full_prob.topk_ids, full_prob.topk_weights,
+                               cfg.experts, *[lambda e, m=m: full_prob.expert_weight(m, e)
+                                              for m in (0, 1, 2)],
+                               hidden=cfg.hidden, inter=cfg.inter)["out"]
+        results[rank] = float(np.max(np.abs(out.numpy() - full)) / np.max(np.abs(full)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("mode", ["ep", "tp"])
+def test_sharded_partial_outputs_all_reduce_to_the_full_output(mode):
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        results = mgr.dict()
+        procs = [ctx.Process(target=_sharded_worker, args=(r, world, port, mode, results))
+                 for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(timeout=180)
+            assert p.exitcode == 0
+        assert results[0] < 1e-12 and results[1] < 1e-12
