@@ -30,6 +30,9 @@ Sources (rustdoc source pages of the "metrale" project; cited by page and item):
   expert is skipped by the MoE kernels.
 * nvfp4_moe_grouped.rs, doc of ``nvfp4_tc_lean_repack``: a negative or NaN
   block scale leaves the matrix unusable and is flagged at load time.
+* transpose.rs, ``transpose_concat_for_gemm_gs`` / ``_padded`` and the host
+  loops of ``transpose_impl``: several parts' twins side by side along N in a
+  row pitch ``stride``, pad columns zero; group size 16 (NVFP4) or 32 (MXFP4).
 * metrale_model_arch/tp_shard/quant_shard.rs, ``shard_quantized_nvfp4``:
   column-parallel keeps a rank's rows of packed and scale, row-parallel a
   rank's K slice of both; weight_scale_2 is replicated.
@@ -89,6 +92,7 @@ __all__ = [
     "count_bad_scales",
     "shard_nvfp4",
     "expert_owner_range",
+    "transpose_concat",
     "RouteSort",
 ]
 
@@ -524,6 +528,43 @@ def transpose_u8(src: np.ndarray, rows: int, cols: int) -> np.ndarray:
         for j in range(cols):
             t[j * rows + i] = b[i * cols + j]
     return t.reshape(cols, rows)
+
+
+def transpose_concat(parts: Sequence[Tuple[np.ndarray, np.ndarray]], k: int, group_size: int,
+                     stride: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Transposed twins of several NVFP4 weights sharing K, side by side along N.
+
+    transpose.rs, ``transpose_impl`` (behind ``transpose_concat_for_gemm_gs``
+    and ``transpose_concat_for_gemm_padded``), host path: part p with n_p rows
+    lands in columns n_off .. n_off + n_p - 1 of a [K/2, stride] packed twin
+    and a [K/group_size, stride] scale twin, n_off being the rows of the parts
+    before it; columns past the last part are zero.  One part with stride = N
+    is ``transpose_for_gemm_gs``.  Written as the page's byte loops: small
+    inputs only.
+    """
+    if not parts:
+        raise ValueError("empty parts")
+    half_k, groups = k // 2, k // group_size
+    n_total = sum(p.shape[0] for p, _ in parts)
+    if stride < n_total:
+        raise ValueError("stride below the total rows")
+    w = np.zeros(half_k * stride, dtype=np.uint8)
+    sc = np.zeros(groups * stride, dtype=np.uint8)
+    n_off = 0
+    for packed, scale in parts:
+        packed = np.asarray(packed, dtype=np.uint8)
+        scale = np.asarray(scale, dtype=np.uint8)
+        n = packed.shape[0]
+        if packed.shape != (n, half_k) or scale.shape != (n, groups):
+            raise ValueError("part shape does not match k / group_size")
+        pb, sb = packed.reshape(-1), scale.reshape(-1)
+        for i in range(n):
+            for j in range(half_k):
+                w[j * stride + n_off + i] = pb[i * half_k + j]
+            for j in range(groups):
+                sc[j * stride + n_off + i] = sb[i * groups + j]
+        n_off += n
+    return w.reshape(half_k, stride), sc.reshape(groups, stride)
 
 
 def relative_l2(got: np.ndarray, ref: np.ndarray) -> float:

@@ -562,6 +562,30 @@ def test_transpose_u8_against_numpy_and_involution(rows, cols):
     np.testing.assert_array_equal(orc.transpose_u8(t, cols, rows), src)
 
 
+@pytest.mark.parametrize("group", [16, 32])
+def test_transpose_concat_is_side_by_side_transposes_with_zero_pad(group):
+    rng = np.random.default_rng(group)
+    k = 128
+    ns = [5, 1, 12]
+    parts = [(rng.integers(0, 256, (n, k // 2), dtype=np.uint8),
+              rng.integers(0, 256, (n, k // group), dtype=np.uint8)) for n in ns]
+    for stride in (sum(ns), 32):
+        w, sc = orc.transpose_concat(parts, k, group, stride)
+        assert w.shape == (k // 2, stride) and sc.shape == (k // group, stride)
+        np.testing.assert_array_equal(w[:, :sum(ns)], np.hstack([p.T for p, _ in parts]))
+        np.testing.assert_array_equal(sc[:, :sum(ns)], np.hstack([s_.T for _, s_ in parts]))
+        assert not w[:, sum(ns):].any() and not sc[:, sum(ns):].any()
+    # One part, stride = N: the single twin of transpose_for_gemm_gs (transpose_u8 twice).
+    p, s_ = parts[2]
+    w, sc = orc.transpose_concat([parts[2]], k, group, 12)
+    np.testing.assert_array_equal(w, orc.transpose_u8(p, 12, k // 2))
+    np.testing.assert_array_equal(sc, orc.transpose_u8(s_, 12, k // group))
+    with pytest.raises(ValueError):
+        orc.transpose_concat(parts, k, group, sum(ns) - 1)
+    with pytest.raises(ValueError):
+        orc.transpose_concat([], k, group, 8)
+
+
 # --------------------------------------------------------------------------- #
 # Planted mistakes: the pins above must catch them
 # --------------------------------------------------------------------------- #
