@@ -63,10 +63,10 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--op", choices=["layer", "check_scales", "shard"], default="layer",
-                    help="layer: the forward; check_scales / shard: the load-time scale check / "
-                         "tensor-parallel shard (--tp ranks, rank 0) of the workload's three "
-                         "projections")
+    ap.add_argument("--op", choices=["layer", "check_scales", "shard", "twins"], default="layer",
+                    help="layer: the forward; check_scales / shard / twins: the load-time scale "
+                         "check, tensor-parallel shard (--tp ranks, rank 0), or concatenated "
+                         "gate|up transposed twin of every expert of the workload")
     ap.add_argument("--tp", type=int, default=2, help="tensor-parallel ranks for --op shard")
     ap.add_argument("--shared", action="store_true",
                     help="add a shared expert (every token, same launches as the routed experts)")
@@ -585,7 +585,13 @@ def run_load_op(args, rank, world, local):
     bad = torch.zeros(3, cfg.experts, dtype=torch.int32, device=dev)
     stream = torch.cuda.Stream(device=dev)
     shard = args.op == "shard"
-    if shard:
+    twins = args.op == "twins"
+    if twins:
+        tw_out = [(torch.empty((cfg.hidden // 2, 2 * cfg.inter), dtype=torch.uint8, device=dev),
+                   torch.empty((cfg.hidden // 16, 2 * cfg.inter), dtype=torch.uint8, device=dev))
+                  for _ in range(cfg.experts)]
+        moved = 2 * 2 * cfg.experts * (layer.gate.packed[0].numel() + layer.gate.scale[0].numel())
+    elif shard:
         kinds = (nvm.SHARD_COLUMN, nvm.SHARD_COLUMN, nvm.SHARD_ROW)
         outs = [nvm.shard_nvfp4(p.packed, p.scale, kd, 0, args.tp) for p, kd in zip(projs, kinds)]
         moved = 2 * sum(o[0].numel() + o[1].numel() for o in outs)  # read + written
@@ -594,6 +600,12 @@ def run_load_op(args, rank, world, local):
     scale_bytes = moved
 
     def one():
+        if twins:
+            for e in range(cfg.experts):
+                nvm.transpose_concat_into(
+                    [(layer.gate.packed[e], layer.gate.scale[e]), (layer.up.packed[e], layer.up.scale[e])],
+                    16, tw_out[e][0], tw_out[e][1], stream=stream)
+            return
         for i, p in enumerate(projs):
             if shard:
                 nvm.shard_nvfp4_into(p.packed, p.scale, kinds[i], 0, args.tp, outs[i][0],
@@ -631,20 +643,22 @@ def run_load_op(args, rank, world, local):
     gbs = scale_bytes / (ms * 1e-3) / 1e9
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     what = (f"NVFP4 tensor-parallel shard GB/s (load time, tp={args.tp}, read + written)" if shard
+            else "NVFP4 gate|up transposed twins GB/s (load time, read + written)" if twins
             else "NVFP4 block-scale check GB/s (load time)")
     line = {
         "metric": what, "value": gbs, "unit": "GB/s",
         "n_gpus": 1, "steps": steps, "warmup": warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic",
-        "config": {"workload": cfg.name + (" weights" if shard else " scale tables"),
+        "config": {"workload": cfg.name + (" weights" if shard or twins else " scale tables"),
                    "experts": cfg.experts, "bytes_per_step": scale_bytes,
                    "l2": f"three projections, {scale_bytes / 3e6:.0f} MB moved each, "
                          f"L2 {l2 / 1e6:.0f} MB"},
-        "roofline": {"kernel": "shard_copy_kernel" if shard else "check_scales_kernel",
+        "roofline": {"kernel": "shard_copy_kernel" if shard else "transpose_u8_kernel" if twins
+                     else "check_scales_kernel",
                      "bound": "hbm", "achieved": gbs, "peak": hbm,
                      "unit": "GB/s", "frac": gbs / hbm, "peak_source": f"{peak_kind} HBM copy",
                      "traffic": None},
-        "gpu_launches": (6 if shard else 3) * steps,
+        "gpu_launches": (4 * cfg.experts if twins else 6 if shard else 3) * steps,
         "clocks": clocks,
     }
     if rank == 0:
@@ -657,7 +671,7 @@ def main(argv=None):
     if args.impl == "reference":
         run_reference(args, rank, world)
         return
-    if args.op in ("check_scales", "shard"):
+    if args.op in ("check_scales", "shard", "twins"):
         run_load_op(args, rank, world, local)
         return
     run_ours(args, rank, world, local)

@@ -411,6 +411,29 @@ NVFP4_MOE_API int nvfp4_moe_shard_nvfp4(const uint8_t* packed, const uint8_t* sc
                                         uint32_t rank, uint32_t tp, uint8_t* packed_out,
                                         uint8_t* scale_out, cudaStream_t stream);
 
+/*
+ * Load-time concatenated / padded twins (transpose_concat_for_gemm_gs and
+ * transpose_concat_for_gemm_padded in transpose.rs, whose host loops define
+ * the result).  num_parts weights share K; part p is packed u8 [n_p, k/2] and
+ * scale u8 [n_p, k/group_size] (group_size 16 for NVFP4, 32 for MXFP4).
+ * packed_parts, scale_parts and part_rows are HOST arrays of length num_parts
+ * (the first two hold device pointers).  Writes
+ *   packed_out u8 [k/2, stride]          column n_off + i of row j = part p's
+ *   scale_out  u8 [k/group_size, stride] byte (i, j), n_off = rows of parts < p;
+ * columns sum(n_p) .. stride - 1 are zero.  stride = sum(n_p) is the plain
+ * concatenation; one part with stride = n_0 is transpose_for_gemm_gs.  Outputs
+ * must not overlap the inputs or each other.  Bit-exact.
+ * EINVAL: num_parts == 0 (the page rejects empty parts), NULL pointers.
+ * ESHAPE: k odd, group_size == 0 or not dividing k, stride < sum(n_p),
+ * n_p > 2097120.
+ */
+NVFP4_MOE_API int nvfp4_moe_transpose_concat(const uint8_t* const* packed_parts,
+                                             const uint8_t* const* scale_parts,
+                                             const uint32_t* part_rows, uint32_t num_parts,
+                                             uint32_t k, uint32_t group_size, uint32_t stride,
+                                             uint8_t* packed_out, uint8_t* scale_out,
+                                             cudaStream_t stream);
+
 /* Host helper: launch bound on active experts, min(num_experts, num_pairs). */
 NVFP4_MOE_API uint32_t nvfp4_moe_active_cap(uint32_t num_experts, uint32_t num_pairs);
 

@@ -31,6 +31,8 @@ from ._binding import (  # noqa: F401
     shard_nvfp4,
     shard_nvfp4_into,
     shared_slots,
+    transpose_concat,
+    transpose_concat_into,
     transpose_u8,
     workspace_bytes,
 )

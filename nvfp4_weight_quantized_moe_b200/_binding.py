@@ -87,6 +87,9 @@ _sig = {
                                         c_void_p, c_void_p, c_void_p]),
     "nvfp4_moe_shared_slots": (c_u32, [c_u32, c_u32]),
     "nvfp4_moe_check_scales": (c_int, [ExpertTables, c_u32, c_u32, c_u32, c_void_p, c_void_p]),
+    "nvfp4_moe_transpose_concat": (c_int, [ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p),
+                                           ctypes.POINTER(c_u32), c_u32, c_u32, c_u32, c_u32,
+                                           c_void_p, c_void_p, c_void_p]),
     "nvfp4_moe_shard_nvfp4": (c_int, [c_void_p, c_void_p, c_u32, c_u32, c_u32, c_int, c_u32, c_u32,
                                       c_void_p, c_void_p, c_void_p]),
     "nvfp4_moe_workspace_bytes": (ctypes.c_size_t, [c_u32, c_u32, c_u32, c_u32]),
@@ -234,6 +237,44 @@ def check_scales(tables: ExpertTables, num_experts, n, k, bad, stream=None) -> N
         raise TypeError("bad: expected 32-bit counters")
     _check("nvfp4_moe_check_scales", _lib.nvfp4_moe_check_scales(
         tables, num_experts, n, k, _ptr(bad, None, "bad"), _stream(stream)))
+
+
+def transpose_concat(parts, group_size: int = 16, stride: Optional[int] = None, stream=None):
+    """nvfp4_moe_transpose_concat: the [K/2, stride] and [K/group_size, stride] twins of
+    ``parts`` (a list of (packed [n, K/2], scale [n, K/group_size]) device tensors)
+    side by side, pad columns zero; ``stride`` defaults to the total rows."""
+    if not parts:
+        raise ValueError("empty parts")
+    half_k = parts[0][0].shape[1]
+    k = 2 * half_k
+    rows = [int(p.shape[0]) for p, _ in parts]
+    for p, sc in parts:
+        if p.shape[1] != half_k or tuple(sc.shape) != (p.shape[0], k // group_size):
+            raise ValueError("every part must be [n, K/2] and [n, K/group_size]")
+    stride = sum(rows) if stride is None else int(stride)
+    dev = parts[0][0].device
+    w = torch.empty((half_k, stride), dtype=torch.uint8, device=dev)
+    sc_out = torch.empty((k // group_size, stride), dtype=torch.uint8, device=dev)
+    transpose_concat_into(parts, group_size, w, sc_out, stream=stream)
+    return w, sc_out
+
+
+def transpose_concat_into(parts, group_size: int, packed_out, scale_out, stream=None) -> None:
+    """nvfp4_moe_transpose_concat into caller-allocated [K/2, stride] and
+    [K/group_size, stride] outputs."""
+    half_k = parts[0][0].shape[1]
+    k = 2 * half_k
+    rows = [int(p.shape[0]) for p, _ in parts]
+    stride = packed_out.shape[1]
+    if tuple(packed_out.shape) != (half_k, stride) or tuple(scale_out.shape) != (k // group_size, stride):
+        raise ValueError("outputs must be [K/2, stride] and [K/group_size, stride]")
+    n = len(parts)
+    pp = (c_void_p * n)(*[_ptr(p, torch.uint8, "packed part") for p, _ in parts])
+    sp = (c_void_p * n)(*[_ptr(sc, torch.uint8, "scale part") for _, sc in parts])
+    rr = (c_u32 * n)(*rows)
+    _check("nvfp4_moe_transpose_concat", _lib.nvfp4_moe_transpose_concat(
+        pp, sp, rr, n, k, group_size, stride, _ptr(packed_out, torch.uint8, "packed_out"),
+        _ptr(scale_out, torch.uint8, "scale_out"), _stream(stream)))
 
 
 def shard_nvfp4(packed, scale, kind: int, rank: int, tp: int, stream=None):

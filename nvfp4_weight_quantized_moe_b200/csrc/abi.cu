@@ -379,6 +379,42 @@ int nvfp4_moe_forward(const uint16_t* x, const int32_t* topk_ids, const float* t
                          hidden, stream);
 }
 
+int nvfp4_moe_transpose_concat(const uint8_t* const* packed_parts,
+                               const uint8_t* const* scale_parts, const uint32_t* part_rows,
+                               uint32_t num_parts, uint32_t k, uint32_t group_size,
+                               uint32_t stride, uint8_t* packed_out, uint8_t* scale_out,
+                               cudaStream_t stream) {
+  if (num_parts == 0 || packed_parts == nullptr || scale_parts == nullptr || part_rows == nullptr)
+    return NVFP4_MOE_EINVAL;
+  if (k == 0 || k % 2 != 0 || group_size == 0 || k % group_size != 0) return NVFP4_MOE_ESHAPE;
+  uint64_t n_total = 0;
+  for (uint32_t p = 0; p < num_parts; ++p) {
+    if (part_rows[p] > 65535u * 32u) return NVFP4_MOE_ESHAPE;
+    if (part_rows[p] > 0 && (packed_parts[p] == nullptr || scale_parts[p] == nullptr))
+      return NVFP4_MOE_EINVAL;
+    n_total += part_rows[p];
+  }
+  if (stride < n_total) return NVFP4_MOE_ESHAPE;
+  if (stride == 0) return NVFP4_MOE_OK;
+  if (packed_out == nullptr || scale_out == nullptr) return NVFP4_MOE_EINVAL;
+  const uint32_t half_k = k / 2, groups = k / group_size;
+  cudaError_t err = cudaSuccess;
+  uint64_t off = 0;
+  for (uint32_t p = 0; p < num_parts && err == cudaSuccess; ++p) {
+    err = launch_transpose_u8_pitched(packed_parts[p], packed_out, part_rows[p], half_k, stride,
+                                      off, stream);
+    if (err == cudaSuccess)
+      err = launch_transpose_u8_pitched(scale_parts[p], scale_out, part_rows[p], groups, stride,
+                                        off, stream);
+    off += part_rows[p];
+  }
+  if (err == cudaSuccess && stride > n_total) {
+    err = launch_zero_cols(packed_out, half_k, stride, n_total, stream);
+    if (err == cudaSuccess) err = launch_zero_cols(scale_out, groups, stride, n_total, stream);
+  }
+  return status_of(err);
+}
+
 uint32_t nvfp4_moe_shared_slots(uint32_t num_tokens, uint32_t shared_rows) {
   if (shared_rows == 0) return 0;
   return (uint32_t)(((uint64_t)num_tokens + shared_rows - 1) / shared_rows);

@@ -78,6 +78,12 @@ cudaError_t launch_shard_copy(const uint8_t* src, uint8_t* dst, uint64_t mats, u
 
 cudaError_t launch_transpose_u8(const uint8_t* src, uint8_t* dst, uint32_t rows, uint32_t cols,
                                 cudaStream_t stream);
+// Transpose [rows, cols] into columns dst_col_off .. of a [cols, dst_pitch] output.
+cudaError_t launch_transpose_u8_pitched(const uint8_t* src, uint8_t* dst, uint32_t rows,
+                                        uint32_t cols, uint64_t dst_pitch, uint64_t dst_col_off,
+                                        cudaStream_t stream);
+cudaError_t launch_zero_cols(uint8_t* dst, uint64_t rows, uint64_t pitch, uint64_t col_lo,
+                             cudaStream_t stream);
 
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device).
 cudaError_t ensure_dynamic_smem(const void* kernel, int bytes);

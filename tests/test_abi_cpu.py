@@ -173,3 +173,20 @@ def test_expert_owner_blocks_match_the_oracle():
                 continue
             for r in range(world):
                 assert expert_owner_range(e, world, r) == orc.expert_owner_range(e, world, r)
+
+
+def test_transpose_concat_validates_on_the_host(lib):
+    import nvfp4_weight_quantized_moe_b200._binding as B
+    L = B._lib
+    P = ctypes.c_void_p
+    pp = (P * 2)(P(1 << 20), P(2 << 20))
+    sp = (P * 2)(P(3 << 20), P(4 << 20))
+    rr = (ctypes.c_uint32 * 2)(8, 4)
+    out_w, out_s = P(5 << 20), P(6 << 20)
+    assert L.nvfp4_moe_transpose_concat(pp, sp, rr, 0, 64, 16, 12, out_w, out_s, None) == 1  # no parts
+    assert L.nvfp4_moe_transpose_concat(pp, sp, rr, 2, 63, 16, 12, out_w, out_s, None) == 2  # odd k
+    assert L.nvfp4_moe_transpose_concat(pp, sp, rr, 2, 64, 24, 12, out_w, out_s, None) == 2  # group
+    assert L.nvfp4_moe_transpose_concat(pp, sp, rr, 2, 64, 16, 11, out_w, out_s, None) == 2  # stride
+    assert L.nvfp4_moe_transpose_concat(pp, sp, rr, 2, 64, 16, 12, None, out_s, None) == 1
+    nulls = (P * 2)(P(1 << 20), None)
+    assert L.nvfp4_moe_transpose_concat(nulls, sp, rr, 2, 64, 16, 12, out_w, out_s, None) == 1

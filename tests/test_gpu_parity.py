@@ -695,3 +695,25 @@ def test_expert_parallel_ranks_sum_to_the_full_forward(world, ws):
     got = _sum_over_ranks(prob, layers, ws, **(dict(path=2) if ws else {}))
     ref = _shared_ref(prob, None)["out"]
     _close(got, ref, f"sum of {world} expert-parallel ranks")
+
+
+# --------------------------------------------------------------------------- #
+# Concatenated / padded twins: bit-exact
+# --------------------------------------------------------------------------- #
+
+@pytest.mark.parametrize("group", [16, 32])
+@pytest.mark.parametrize("ns,k,pad", [((37,), 256, 0), ((64, 5, 130), 512, 0), ((33, 7), 192, 11),
+                                     ((1536, 1536), 2048, 0), ((100,), 64, 28)])
+def test_transpose_concat_bit_exact(ns, k, pad, group):
+    _need_gpu()
+    import nvfp4_weight_quantized_moe_b200 as nvm
+    rng = np.random.default_rng(sum(ns) + k + pad + group)
+    parts = [(rng.integers(0, 256, (n, k // 2), dtype=np.uint8),
+              rng.integers(0, 256, (n, k // group), dtype=np.uint8)) for n in ns]
+    stride = sum(ns) + pad
+    dparts = [(torch.from_numpy(p).cuda(), torch.from_numpy(s).cuda()) for p, s in parts]
+    w, sc = nvm.transpose_concat(dparts, group, stride)
+    torch.cuda.synchronize()
+    ew, es = orc.transpose_concat(parts, k, group, stride)
+    np.testing.assert_array_equal(w.cpu().numpy(), ew)
+    np.testing.assert_array_equal(sc.cpu().numpy(), es)

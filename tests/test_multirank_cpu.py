@@ -123,3 +123,18 @@ def test_sharded_partial_outputs_all_reduce_to_the_full_output(mode):
             p.join(timeout=180)
             assert p.exitcode == 0
         assert results[0] < 1e-12 and results[1] < 1e-12
+
+
+def test_bench_routes_every_load_time_op():
+    # Each --op other than the layer forward goes to the load-time runner.
+    import bench
+    seen = []
+    orig_load, orig_ours = bench.run_load_op, bench.run_ours
+    bench.run_load_op = lambda args, *a: seen.append(("load", args.op))
+    bench.run_ours = lambda args, *a: seen.append(("layer", args.op))
+    try:
+        for op in ("check_scales", "shard", "twins", "layer"):
+            bench.main(["--op", op])
+    finally:
+        bench.run_load_op, bench.run_ours = orig_load, orig_ours
+    assert seen == [("load", "check_scales"), ("load", "shard"), ("load", "twins"), ("layer", "layer")]
