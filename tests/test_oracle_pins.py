@@ -651,3 +651,61 @@ def test_pins_catch_an_unstable_sort(monkeypatch):
     monkeypatch.setattr(mod, "_stable_order", ties_reversed)
     with pytest.raises(AssertionError):
         test_route_sort_brute_force(33, 8, 128)
+
+
+def test_pins_catch_a_scale_slice_off_by_one_group(monkeypatch):
+    real = orc.shard_nvfp4
+
+    def shifted(packed, scale, kind, rank, tp):
+        p, s_ = real(packed, scale, kind, rank, tp)
+        if kind == "row" and rank > 0:
+            groups = np.asarray(scale).shape[1] // tp
+            s_ = np.asarray(scale)[:, rank * groups - 1:(rank + 1) * groups - 1].copy()
+        return p, s_
+
+    monkeypatch.setattr(orc, "shard_nvfp4", shifted)
+    with pytest.raises(AssertionError):
+        test_shards_reassemble_and_dequantise_to_slices(2)
+
+
+def test_pins_catch_interleaved_shared_slots(monkeypatch):
+    real = orc.append_shared_routing
+
+    def interleaved(ids, w, e, rows, sw=None):
+        ids2, w2 = real(ids, w, e, rows, sw)
+        m = ids2.shape[0]
+        slots = -(-m // rows)
+        ids2[:, -1] = e + np.arange(m) % slots  # round-robin instead of token blocks
+        return ids2, w2
+
+    monkeypatch.setattr(orc, "append_shared_routing", interleaved)
+    with pytest.raises(AssertionError):
+        test_append_shared_routing_layout(33, 8, 128, 16)
+
+
+def test_pins_catch_flagging_negative_zero(monkeypatch):
+    import oracle.nvfp4_moe_oracle as mod
+    real = mod.count_bad_scales
+
+    def sign_bit(codes):
+        c = np.asarray(codes, dtype=np.uint8).reshape(-1)
+        return real(c) + int(np.count_nonzero(c == 0x80))
+
+    monkeypatch.setattr(orc, "count_bad_scales", sign_bit)
+    with pytest.raises(AssertionError):
+        test_bad_scale_count_against_ml_dtypes_over_every_code()
+
+
+def test_pins_catch_a_missing_column_offset_in_the_twins(monkeypatch):
+    def no_offset(parts, k, group, stride):
+        half_k, groups = k // 2, k // group
+        w = np.zeros((half_k, stride), np.uint8)
+        sc = np.zeros((groups, stride), np.uint8)
+        for p, s_ in parts:  # every part written at column 0
+            w[:, :p.shape[0]] = np.asarray(p).T
+            sc[:, :p.shape[0]] = np.asarray(s_).T
+        return w, sc
+
+    monkeypatch.setattr(orc, "transpose_concat", no_offset)
+    with pytest.raises(AssertionError):
+        test_transpose_concat_is_side_by_side_transposes_with_zero_pad(16)
