@@ -109,12 +109,6 @@ def draw_shared_weight(cfg: MoEConfig, matrix: int) -> Tuple[np.ndarray, np.ndar
     return packed, scale
 
 
-def draw_shared_gate(cfg: MoEConfig) -> np.ndarray:
-    """Per-token weight of the shared expert, f32 [M]: the sigmoid of an N(0, 1) logit."""
-    z = np.random.default_rng([cfg.seed, 0, 3]).standard_normal(cfg.tokens)
-    return (1.0 / (1.0 + np.exp(-z))).astype(np.float32)
-
-
 def draw_routing(cfg: MoEConfig) -> Tuple[np.ndarray, np.ndarray]:
     """topk_ids int32 [M, k] and topk_weights f32 [M, k]."""
     m, e, k = cfg.tokens, cfg.experts, cfg.topk
