@@ -356,8 +356,9 @@ NVFP4_MOE_API int nvfp4_moe_transpose_u8(const uint8_t* src, uint8_t* dst, uint3
  * output for tokens 0 .. num_tokens - 1 (sh_act and sh_down_out).  Each block
  * of shared_rows tokens gets its own CTAs in the projections; a block size
  * near the routed rows per expert keeps the work even.
- * ESHAPE if num_experts + S > 1024 or num_tokens * (topk + 1) > 1<<24;
- * EINVAL for shared_rows == 0 or a NULL required pointer.
+ * ESHAPE if topk or num_experts is 0, num_experts + S > 1024 or
+ * num_tokens * (topk + 1) > 1<<24; EINVAL for shared_rows == 0 or a NULL
+ * required pointer.  num_tokens == 0 launches nothing.
  */
 NVFP4_MOE_API int nvfp4_moe_append_shared(const int32_t* topk_ids, const float* topk_weights,
                                           const float* shared_weights, uint32_t num_tokens,
