@@ -6,13 +6,16 @@
 
 One step = one layer forward: route sort, gate+up SiLU, down, blend (the four
 C-ABI calls) over one batch of the workload's synthetic tokens, weights and
-inputs resident in HBM.  ``--shared`` adds the workload's shared expert,
-run by every token inside the same launches (one more routing slot).  The weights rotate over R device replicas (R x the
-routed bytes of a step >= 4 x L2), so every step streams its expert weights
-from HBM.  Steps are replayed from CUDA graphs and timed with CUDA events on
-the launching stream; under torchrun (N > 1) each rank runs an independent
-replica of the workload (weak scaling, no collective on the data path) and the
-time is the max over ranks.
+inputs resident in HBM.  The default workload is prefill M=8192, the largest
+single-GPU one; ``--config`` picks another.  ``--shared`` adds the workload's
+shared expert, run by every token inside the same launches (one more routing
+slot).  The weights rotate over R device replicas (R x the routed bytes of a
+step >= 4 x L2), so every step streams its expert weights from HBM.  The timed
+region is one replay of a CUDA graph holding exactly ``--steps`` forwards,
+bracketed by CUDA events on the launching stream (the median of per-replay
+times of single-step graphs is reported beside it); under torchrun (N > 1)
+each rank runs an independent replica of the workload (weak scaling, no
+collective on the data path) and the time is the max over ranks.
 
 Rank 0 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle
 on the host cores instead (rank 0 only).
@@ -37,23 +40,49 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "NVFP4 MoE layer tokens/s and routed-weight HBM GB/s (% of peak), 1 B200"
-DEFAULT_CONFIG = "decode_m1"
+DEFAULT_CONFIG = "prefill_m8192"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
-# Default timed steps per workload: about a second of GPU time each.
-DEFAULT_STEPS = {"tiny": 20000, "decode_m1": 20000, "decode_m32": 5000, "decode_m256": 500,
+# Default timed steps per workload: a fraction of a second to a second of GPU
+# time each (all of them are captured in one CUDA graph).
+DEFAULT_STEPS = {"tiny": 4000, "decode_m1": 4000, "decode_m32": 2000, "decode_m256": 300,
                  "prefill_m8192": 200}
 
-# DRAM bytes (read + write) of one launch of the dominant kernel (gate+up
-# SiLU) from an ncu capture of the same kernel build and launch shape; see the
-# summaries under profiles/.  Absent for workloads not captured, and cleared
-# whenever that kernel changes.
-NCU_TRAFFIC_BYTES = {
-    ("decode_m1", "mma.sync"): 28357888,      # 28.36 MB read, 0 written (routed gate+up: 28.31 MB)
-    ("decode_m32", "tcgen05"): 335457536,     # 329.50 MB read, 5.96 MB written
-    ("prefill_m8192", "tcgen05"): 4249585000,  # 3.838 GB read, 0.411 GB written (4 token passes)
+# Sources of each projection kernel; their hash names the build an ncu capture
+# was taken from.
+KERNEL_SOURCES = {
+    "tcgen05": ["grouped_tc.cu", "tc_common.cuh", "common.cuh"],
+    "mma.sync": ["grouped_mma.cu", "common.cuh"],
 }
+
+# DRAM bytes (read + write) of one launch of the dominant kernel (gate+up
+# SiLU) from an ncu capture (summaries under profiles/), keyed by workload and
+# kernel, with the hash of that kernel's sources when it was captured.  An
+# entry whose hash no longer matches the sources is stale and not reported.
+NCU_TRAFFIC_BYTES = {
+    ("decode_m1", "mma.sync"): (28357888, "00f418d43112"),
+    ("decode_m32", "tcgen05"): (335457536, "5e2f82da6383"),
+    ("prefill_m8192", "tcgen05"): (4249585000, "5e2f82da6383"),
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """First 12 hex digits of the SHA-256 over a projection kernel's sources."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "nvfp4_weight_quantized_moe_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def ncu_traffic(workload: str, kernel: str):
+    """Captured DRAM bytes per launch, or None when absent or taken from other sources."""
+    entry = NCU_TRAFFIC_BYTES.get((workload, kernel))
+    if entry is None or entry[1] != kernel_source_hash(kernel):
+        return None
+    return entry[0]
 
 
 def parse_args(argv=None):
@@ -263,15 +292,17 @@ def run_ours(args, rank, world, local):
     def step(lay):
         lay.forward(x, ids, w, bufs, workspace=ws, **_opts(args))
 
-    # Graphs: one of R steps (one per replica) plus single-step graphs for remainders.
+    # The timed region is ONE replay of a graph holding exactly `steps` layer
+    # forwards, step i on replica i % R; nothing else is launched inside it.
     with torch.cuda.stream(stream):
         for lay in layers:
             step(lay)
     stream.synchronize()
-    g_all = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_all, stream=stream):
-        for lay in layers:
-            step(lay)
+    g_steps = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_steps, stream=stream):
+        for i in range(steps):
+            step(layers[i % len(layers)])
+    # Single-step graphs, one per replica: warm-up and the per-replay median.
     g_one = []
     for lay in layers:
         g = torch.cuda.CUDAGraph()
@@ -279,15 +310,10 @@ def run_ours(args, rank, world, local):
             step(lay)
         g_one.append(g)
 
-    def run_steps(n):
-        full, rem = divmod(n, len(layers))
-        for _ in range(full):
-            g_all.replay()
-        for i in range(rem):
-            g_one[i].replay()
-
     with torch.cuda.stream(stream):
-        run_steps(warmup)
+        for i in range(warmup):
+            g_one[i % len(layers)].replay()
+        g_steps.replay()  # first replay of the big graph (uploads it), untimed
     stream.synchronize()
 
     sampler = ClockSampler(local)
@@ -299,7 +325,7 @@ def run_ours(args, rank, world, local):
     sampler.mark(True)
     with torch.cuda.stream(stream):
         ev0.record(stream)
-        run_steps(steps)
+        g_steps.replay()
         ev1.record(stream)
     torch.cuda.synchronize(dev)
     sampler.mark(False)
@@ -308,6 +334,19 @@ def run_ours(args, rank, world, local):
     elapsed_ms = reduce_max(ev0.elapsed_time(ev1))
     ms_per_step = elapsed_ms / steps
     tokens_per_s = world * cfg.tokens * steps / (elapsed_ms / 1e3)
+
+    # Median over per-replay event times of single-step graphs (each replay
+    # bracketed by its own events; replicas in turn), after the timed region.
+    n_med = max(5, min(steps, 200))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n_med)]
+    with torch.cuda.stream(stream):
+        for i, (a, b) in enumerate(evs):
+            a.record(stream)
+            g_one[i % len(layers)].replay()
+            b.record(stream)
+    torch.cuda.synchronize(dev)
+    median_ms = reduce_max(statistics.median(a.elapsed_time(b) for a, b in evs))
 
     hbm, tflops, tflops_sus, peak_kind = measured_peaks()
     routed_gbs = world * routed_bytes / (ms_per_step * 1e-3) / 1e9
@@ -351,7 +390,8 @@ def run_ours(args, rank, world, local):
                     "achieved": achieved, "peak": tflops, "unit": "TFLOP/s",
                     "frac": achieved / tflops, "peak_source": f"{peak_kind} bf16 burst",
                     "algorithmic_flops_per_launch": gu_flops, "launch_ms": gu_ms,
-                    "traffic": NCU_TRAFFIC_BYTES.get((cfg.name, "tcgen05"))}
+                    "traffic": ncu_traffic(cfg.name, "tcgen05"),
+                    "traffic_source_hash": kernel_source_hash("tcgen05")}
     else:
         achieved = gu_bytes / (gu_ms * 1e-3) / 1e9
         roofline = {"kernel": "nvfp4_moe_gate_up_silu_ws (tcgen05, 16-row passes)" if tc else
@@ -359,7 +399,8 @@ def run_ours(args, rank, world, local):
                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                     "peak_source": f"{peak_kind} HBM copy", "algorithmic_bytes_per_launch": gu_bytes,
                     "launch_ms": gu_ms,
-                    "traffic": NCU_TRAFFIC_BYTES.get((cfg.name, "tcgen05" if tc else "mma.sync"))}
+                    "traffic": ncu_traffic(cfg.name, "tcgen05" if tc else "mma.sync"),
+                    "traffic_source_hash": kernel_source_hash("tcgen05" if tc else "mma.sync")}
 
     e2e = None if args.no_e2e else run_e2e(layers, prob, bufs, ws, dev, stream, steps, warmup, args, world)
 
@@ -382,6 +423,11 @@ def run_ours(args, rank, world, local):
                          f"{len(layers)} x {routed_bytes/1e6:.1f} MB routed >= 4 x L2 ({l2/1e6:.0f} MB)"
                          if len(layers) > 1 else f"routed bytes {routed_bytes/1e6:.0f} MB > 4 x L2",
                    "parallelism": f"replicas x{world}"},
+        "median_step": {"ms": median_ms, "tokens_per_s": world * cfg.tokens / (median_ms * 1e-3),
+                        "replays": n_med,
+                        "how": "median of per-replay CUDA-event times of single-step graphs"},
+        "timed_region": f"one replay of a CUDA graph of exactly {steps} layer forwards "
+                        f"(step i on weight replica i mod {len(layers)})",
         "routed_weight_gbs": {"value": routed_gbs, "peak": hbm, "frac": routed_gbs / hbm,
                               "bytes_per_step": routed_bytes},
         "roofline": roofline,
@@ -395,7 +441,7 @@ def run_ours(args, rank, world, local):
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
-        del g_all, g_one, gu_graph
+        del g_steps, g_one, gu_graph
         dist.destroy_process_group()
 
 

@@ -249,7 +249,9 @@ NVFP4_MOE_API int nvfp4_moe_down_ws(
  * tcgen05 path does not take (n_inter % 128, k_hidden % 256).  The call never
  * allocates memory.  Its first call on a device looks the scratch array's
  * device address up (cudaGetSymbolAddress) with that device current; make
- * that first call before any stream capture.  All calls share the one array
+ * that first call before any stream capture.  The address is kept for the
+ * life of the process: after cudaDeviceReset of a device, do not call this
+ * entry point on that device again.  All calls share the one array
  * and each call leaves its packed rows there: calls whose kernels overlap on
  * the GPU (different streams, or different host threads) race on it.
  */
@@ -266,6 +268,20 @@ NVFP4_MOE_API int nvfp4_moe_gate_up_silu_noalloc(
  * device; clear != 0 resets it to 0.  Returns -1 if the read itself failed.
  */
 NVFP4_MOE_API int nvfp4_moe_device_error(int clear);
+
+/*
+ * Self-test of the bounded waits behind nvfp4_moe_device_error (the pages have
+ * no counterpart; the device "bad" word that `nvfp4_tc_lean_repack` in
+ * nvfp4_moe_grouped.rs sets for the host to read is the same pattern).  One
+ * thread initialises a barrier that expects one arrival, arrives on it only if
+ * `arrive` is non-zero, then waits on it with the library's bounded wait,
+ * giving up after `cycle_limit` SM clock cycles.  With arrive == 0 the wait
+ * runs out, the device error word becomes 1 and the kernel returns normally
+ * (nothing traps; the context stays usable); with arrive != 0 the word is left
+ * as it was.  cycle_limit == 0 returns NVFP4_MOE_EINVAL.  Asynchronous: read
+ * the result with nvfp4_moe_device_error.
+ */
+NVFP4_MOE_API int nvfp4_moe_wait_selftest(uint32_t cycle_limit, int arrive, cudaStream_t stream);
 
 /*
  * Step 4: router-weighted blend back into token order

@@ -21,6 +21,7 @@ from ._binding import (  # noqa: F401
     blend,
     check_scales,
     device_error,
+    wait_selftest,
     down,
     down_ws,
     exported_symbols,

@@ -94,6 +94,7 @@ _sig = {
                                       c_void_p, c_void_p, c_void_p]),
     "nvfp4_moe_workspace_bytes": (ctypes.c_size_t, [c_u32, c_u32, c_u32, c_u32]),
     "nvfp4_moe_device_error": (c_int, [c_int]),
+    "nvfp4_moe_wait_selftest": (c_int, [c_u32, c_int, c_void_p]),
     "nvfp4_moe_active_cap": (c_u32, [c_u32, c_u32]),
     "nvfp4_moe_status_string": (ctypes.c_char_p, [c_int]),
 }
@@ -320,6 +321,13 @@ def workspace_bytes(num_tokens, topk, hidden, inter) -> int:
 def device_error(clear: bool = True) -> int:
     """The library's device error word (synchronises the device)."""
     return int(_lib.nvfp4_moe_device_error(1 if clear else 0))
+
+
+def wait_selftest(cycle_limit: int, arrive: bool, stream=None) -> None:
+    """nvfp4_moe_wait_selftest: one bounded barrier wait on the device that runs
+    out (arrive=False: the device error word becomes 1) or completes."""
+    _check("nvfp4_moe_wait_selftest", _lib.nvfp4_moe_wait_selftest(
+        cycle_limit, 1 if arrive else 0, _stream(stream)))
 
 
 def _ws(workspace):

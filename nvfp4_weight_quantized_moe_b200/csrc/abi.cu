@@ -28,9 +28,6 @@ cudaError_t ensure_dynamic_smem(const void* kernel, int bytes) {
 
 namespace {
 
-constexpr uint32_t kMaxExperts = 1024;
-constexpr uint64_t kMaxPairs = 1ull << 24;
-
 bool tables_ok(const nvfp4_expert_tables& t) {
   return t.packed_ptrs != nullptr && t.scale_ptrs != nullptr && t.scale2 != nullptr;
 }
@@ -214,15 +211,12 @@ int nvfp4_moe_device_error(int clear) {
   return v;
 }
 
-namespace {
-
-// Token rows per pass of the tcgen05 kernel: 16 for decode-shaped batches (a
-// few rows per expert), 128 when experts carry many rows.
-int plan_tc_rows(uint64_t tokens, uint64_t pairs, uint32_t num_experts, const nvfp4_moe_launch_opts* o) {
-  if (o && o->tiles) return o->tiles * 8;
-  const uint64_t mean = (pairs + num_experts - 1) / num_experts;
-  return mean <= 16 ? 16 : 128;
+int nvfp4_moe_wait_selftest(uint32_t cycle_limit, int arrive, cudaStream_t stream) {
+  if (cycle_limit == 0) return NVFP4_MOE_EINVAL;
+  return status_of(launch_wait_selftest(cycle_limit, arrive != 0, stream));
 }
+
+namespace {
 
 // The tcgen05 kernel covers 128 (gate+up) or 256 (down) output rows per CTA.
 // Chosen automatically from 2 routed rows per expert on average: below that
@@ -266,7 +260,7 @@ int nvfp4_moe_gate_up_silu_ws(const uint16_t* x, nvfp4_expert_tables gate, nvfp4
     return NVFP4_MOE_EINVAL;
   if (workspace_bytes < tc_workspace_bytes(num_tokens, topk, k_hidden, n_inter)) return NVFP4_MOE_EINVAL;
   if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return NVFP4_MOE_EINVAL;
-  const int nt = plan_tc_rows(num_tokens, pairs, num_experts, opts);
+  const int nt = plan_tc_rows(pairs, num_experts, opts ? opts->tiles : 0);
   if (nt != 16 && nt != 128) return NVFP4_MOE_EINVAL;
   GroupedArgs a{};
   a.src = x;
@@ -312,7 +306,7 @@ int nvfp4_moe_down_ws(const float* act, nvfp4_expert_tables down, float* y,
     return NVFP4_MOE_EINVAL;
   if (workspace_bytes < tc_workspace_bytes(num_tokens, topk, n_hidden, k_inter)) return NVFP4_MOE_EINVAL;
   if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return NVFP4_MOE_EINVAL;
-  const int nt = plan_tc_rows(num_tokens, pairs, num_experts, opts);
+  const int nt = plan_tc_rows(pairs, num_experts, opts ? opts->tiles : 0);
   if (nt != 16 && nt != 128) return NVFP4_MOE_EINVAL;
   GroupedArgs a{};
   a.src = act;

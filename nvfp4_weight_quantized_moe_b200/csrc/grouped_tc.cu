@@ -65,7 +65,6 @@ constexpr int kMmaWarp = kProdWarps;            // warp 8
 constexpr int kWLoadWarp = kProdWarps + 1;      // warp 9
 constexpr int kBLoadWarp = kProdWarps + 2;      // warp 10
 constexpr int kThreads = 32 * (kProdWarps + 3);
-constexpr int kMaxExperts = 1024;
 constexpr int kMapsPerExpert = 4;               // packed0, scale0, packed1, scale1
 constexpr size_t kMapBytes = (size_t)kMaxExperts * kMapsPerExpert * sizeof(CUtensorMap);
 
@@ -761,7 +760,7 @@ cudaError_t launch_tc(int mode, int nt, const GroupedArgs& g, void* workspace, u
                       uint32_t hidden, uint32_t inter, uint32_t cap, cudaStream_t stream) {
   const uint64_t pairs = (uint64_t)tokens * g.topk;
   const WsLayout w = ws_layout(workspace, pairs, hidden, inter);
-  if (g.num_experts == 0 || g.num_experts > (uint32_t)kMaxExperts || (nt != 16 && nt != 128))
+  if (g.num_experts == 0 || g.num_experts > kMaxExperts || (nt != 16 && nt != 128))
     return cudaErrorInvalidValue;
   TcArgs a{};
   a.packed0 = g.packed0;
@@ -828,6 +827,25 @@ cudaError_t launch_tc(int mode, int nt, const GroupedArgs& g, void* workspace, u
   a.wmaps = w.maps_down;
   if (nt == 16) return launch_tc_impl<kModeDown, 16>(a, b0, b1, cap, stream);
   return launch_tc_impl<kModeDown, 128>(a, b0, b1, cap, stream);
+}
+
+// One thread initialises an mbarrier that expects one arrival, arrives on it
+// only if `arrive` is set, and waits for its phase with a limit of
+// `cycle_limit` SM clock cycles: the library's bounded wait, which on timeout
+// sets the device error word and returns.
+__global__ void wait_selftest_kernel(uint32_t cycle_limit, int arrive) {
+  __shared__ alignas(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  mbar_init_fence();
+  if (arrive) mbar_arrive(b);
+  mbar_wait(b, 0, (long long)cycle_limit);
+}
+
+cudaError_t launch_wait_selftest(uint32_t cycle_limit, int arrive, cudaStream_t stream) {
+  wait_selftest_kernel<<<1, 32, 0, stream>>>(cycle_limit, arrive);
+  return cudaGetLastError();
 }
 
 cudaError_t read_device_error(int* value, bool clear) {

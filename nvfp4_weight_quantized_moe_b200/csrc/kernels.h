@@ -8,6 +8,20 @@ namespace nvm {
 
 enum { kModeGateUp = 0, kModeDown = 1 };
 
+// Limits shared by every entry point: expert table entries and routed pairs
+// per call.
+constexpr uint32_t kMaxExperts = 1024;
+constexpr uint64_t kMaxPairs = 1ull << 24;
+
+// Token rows per pass of the tcgen05 kernel: 16 for decode-shaped batches (a
+// few rows per expert), 128 when experts carry many rows.  `tiles` > 0 (a
+// launch option) forces tiles * 8.
+inline int plan_tc_rows(uint64_t pairs, uint32_t num_experts, int tiles) {
+  if (tiles > 0) return tiles * 8;
+  const uint64_t mean = (pairs + num_experts - 1) / num_experts;
+  return mean <= 16 ? 16 : 128;
+}
+
 // Arguments of the grouped projection kernels.  Mode gate+up reads BF16 x
 // [M, K] and two weight tables (gate, up) with the same [N, K]; mode down
 // reads FP32 act [P, K] and one table.  `out` is [P, N] FP32 by sorted position.
@@ -53,6 +67,8 @@ size_t tc_gate_up_workspace_bytes(uint64_t pairs, uint64_t hidden);
 cudaError_t launch_tc(int mode, int nt, const GroupedArgs& a, void* workspace, uint32_t tokens,
                       uint32_t hidden, uint32_t inter, uint32_t cap, cudaStream_t stream);
 cudaError_t read_device_error(int* value, bool clear);
+// One bounded barrier wait on the device (self-test of the timeout path).
+cudaError_t launch_wait_selftest(uint32_t cycle_limit, int arrive, cudaStream_t stream);
 
 cudaError_t launch_route_sort(const int32_t* topk_ids, uint32_t num_pairs, uint32_t num_experts,
                               int32_t* expert_offsets, int32_t* sorted_pair_ids, int32_t* pair_pos,

@@ -12,7 +12,9 @@
 // library holds it until the process exits; its size is kept modest for that
 // reason (kStaticScratchBytes).  Host code cannot use the variable's name as a
 // device address, so the address is looked up with cudaGetSymbolAddress, once
-// per device, on that device's first call.
+// per device, on that device's first call.  The cached address belongs to the
+// device's context at that time: after cudaDeviceReset the library must not be
+// called again on that device in this process.
 
 #include <mutex>
 
@@ -64,10 +66,10 @@ extern "C" int nvfp4_moe_gate_up_silu_noalloc(
     const int32_t* active_count, uint32_t n_inter, uint32_t k_hidden, uint32_t cap,
     uint32_t num_tokens, uint32_t topk, uint32_t num_experts, cudaStream_t stream) {
   if (n_inter == 0 || n_inter % 128 != 0 || k_hidden == 0 || k_hidden % 256 != 0 || topk == 0 ||
-      cap > 65535 || num_experts == 0 || num_experts > 1024)
+      cap > 65535 || num_experts == 0 || num_experts > kMaxExperts)
     return NVFP4_MOE_ESHAPE;
   const uint64_t pairs = (uint64_t)num_tokens * topk;
-  if (pairs > (1ull << 24)) return NVFP4_MOE_ESHAPE;
+  if (pairs > kMaxPairs) return NVFP4_MOE_ESHAPE;
   // Requests whose packed rows do not fit the fixed scratch are refused.
   if (gate_up_scratch_bytes(pairs, k_hidden) > kStaticScratchBytes) return NVFP4_MOE_ESHAPE;
   if (pairs == 0 || cap == 0) return NVFP4_MOE_OK;
@@ -80,8 +82,7 @@ extern "C" int nvfp4_moe_gate_up_silu_noalloc(
   if (static_scratch_address(&scratch) != cudaSuccess) return NVFP4_MOE_ECUDA;
   // Nothing in the scratch has to start at zero: the pack kernel writes every
   // packed row and scale before the projection kernel reads them.
-  const uint64_t mean_rows = (pairs + num_experts - 1) / num_experts;
-  const int nt = mean_rows <= 16 ? 16 : 128;
+  const int nt = plan_tc_rows(pairs, num_experts, 0);  // the _ws call's rule
   GroupedArgs a{};
   a.src = x;
   a.packed0 = gate.packed_ptrs;

@@ -37,17 +37,18 @@ NVM_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Wait for the phase with the given parity to complete, giving up after about
-// one second of SM clock (2^31 cycles).  On timeout the device error word is
-// set and false is returned; callers then skip their remaining waits and exit
-// normally.
-NVM_DEV bool mbar_wait(uint32_t bar, uint32_t parity) {
+// Wait for the phase with the given parity to complete, giving up after
+// `limit` SM clock cycles (by default 2^31, about one second).  On timeout the
+// device error word is set and false is returned; callers then skip their
+// remaining waits and exit normally.
+constexpr long long kWaitLimitCycles = 1ll << 31;
+NVM_DEV bool mbar_wait(uint32_t bar, uint32_t parity, long long limit = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (clock64() - t0 > (1ll << 31)) break;
+    if (clock64() - t0 > limit) break;
   }
   atomicExch(&g_device_error, kErrMbarTimeout);
   return false;

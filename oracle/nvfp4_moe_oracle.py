@@ -397,13 +397,16 @@ def shared_expert(x_bf16, gate: Weight, up: Weight, down: Weight) -> Tuple[np.nd
 
 def moe_forward_shared(x_bf16, topk_ids, topk_weights, num_experts, gate_fn, up_fn, down_fn,
                        hidden: int, inter: int, shared: Tuple[Weight, Weight, Weight],
-                       shared_weights: Optional[np.ndarray] = None) -> Dict[str, object]:
+                       shared_weights: Optional[np.ndarray] = None,
+                       routed: Optional[Dict[str, object]] = None) -> Dict[str, object]:
     """The routed forward plus the shared expert: out[t] += c_t * sh_out[t].
 
     c_t is ``shared_weights[t]``, or 1 for every token when it is None.
+    ``routed``, if given, is the result of :func:`moe_forward` on the same
+    routed inputs, already computed (the weight functions are then unused).
     """
-    res = moe_forward(x_bf16, topk_ids, topk_weights, num_experts, gate_fn, up_fn, down_fn,
-                      hidden, inter)
+    res = dict(routed) if routed is not None else moe_forward(
+        x_bf16, topk_ids, topk_weights, num_experts, gate_fn, up_fn, down_fn, hidden, inter)
     sh_act, sh_out = shared_expert(x_bf16, *shared)
     m = sh_out.shape[0]
     c = (np.ones(m) if shared_weights is None

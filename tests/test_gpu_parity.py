@@ -379,6 +379,25 @@ def test_large_activation_range():
         _close(out[t], ref["out"][t], f"out row {t}")
 
 
+def test_bounded_wait_runs_out_reports_and_the_library_still_works():
+    """A barrier wait that nothing completes gives up after its cycle limit, sets the
+    device error word and returns; the word is cleared on read; later forwards run."""
+    _need_gpu()
+    import nvfp4_weight_quantized_moe_b200 as nvm
+    assert nvm.device_error() == 0
+    nvm.wait_selftest(4096, arrive=True)  # the phase completes: no error
+    torch.cuda.synchronize()
+    assert nvm.device_error() == 0
+    nvm.wait_selftest(4096, arrive=False)  # nothing arrives: the wait runs out
+    torch.cuda.synchronize()
+    assert nvm.device_error(clear=True) == 1
+    assert nvm.device_error() == 0
+    prob = make_problem(SMALL["ragged"])
+    for ws in (False, True):
+        _, bufs = _gpu_forward(prob, ws=ws, **(dict(path=2) if ws else {}))
+        _check_full(prob, bufs)
+
+
 # --------------------------------------------------------------------------- #
 # The five workloads at full size
 # --------------------------------------------------------------------------- #
@@ -392,39 +411,37 @@ def test_forward_full_decode(name, ws):
     _check_full(prob, bufs)
 
 
-def _check_sampled(prob, bufs, tokens):
-    cfg = prob.cfg
-    rs = orc.route_sort(prob.topk_ids, cfg.experts)
+# The oracle's full result at the two large sizes, computed once per session
+# (expert blocks spread over host processes; see _oracle_pool.py).
+_FULL_REF = {}
+
+
+def _full_ref(name):
+    if name not in _FULL_REF:
+        from _oracle_pool import moe_forward_pooled
+        _FULL_REF[name] = moe_forward_pooled(CONFIGS[name])
+    return _FULL_REF[name]
+
+
+def _check_against(ref, bufs, cfg):
+    rs = ref["sort"]
     _check_sort(bufs, rs, cfg.experts, cfg.pairs)
-    ref = orc.moe_forward_tokens(prob.x_bf16, prob.topk_ids, prob.topk_weights, cfg.experts,
-                                 *_fns(prob), tokens=tokens, hidden=cfg.hidden)
-    _close(bufs.out.cpu().numpy()[tokens], ref, "out (sampled tokens)")
-    # act / y rows of those tokens' pairs, by sorted position
-    x = orc.bf16_bits_to_f64(prob.x_bf16)
-    act = bufs.act.cpu().numpy()
-    y = bufs.y.cpu().numpy()
-    for t in tokens[:1]:
-        for s in range(cfg.topk):
-            e = int(prob.topk_ids[t, s])
-            pos = int(rs.pair_pos[t * cfg.topk + s])
-            wg = orc.dequantize_nvfp4(*prob.expert_weight(MATRIX_GATE, e, cache=True))
-            wu = orc.dequantize_nvfp4(*prob.expert_weight(MATRIX_UP, e, cache=True))
-            wd = orc.dequantize_nvfp4(*prob.expert_weight(MATRIX_DOWN, e, cache=True))
-            h = orc.silu(wg @ x[t]) * (wu @ x[t])
-            _close(act[pos], h, f"act[{pos}]")
-            _close(y[pos], wd @ h, f"y[{pos}]")
+    kept = int(rs.expert_offsets[-1])
+    _close(bufs.act.cpu().numpy()[:kept], ref["act"][:kept], "act")
+    _close(bufs.y.cpu().numpy()[:kept], ref["y"][:kept], "y")
+    _close(bufs.out.cpu().numpy(), ref["out"], "out")
+    ob = bufs.out_bf16.float().cpu().numpy()
+    np.testing.assert_array_equal(ob, bufs.out.bfloat16().float().cpu().numpy())
 
 
 @pytest.mark.parametrize("ws", [False, True], ids=["decode-path", "tcgen05"])
 @pytest.mark.parametrize("name", ["decode_m256", "prefill_m8192"])
-def test_forward_full_size_sampled(name, ws):
-    """Full-size launch, checked on a seeded sample of tokens (tokens are independent)."""
+def test_forward_full_size_every_element(name, ws):
+    """Full-size launch, every element of act, y and out against the oracle's full forward."""
     _need_gpu()
     prob = make_problem(name)
     _, bufs = _gpu_forward(prob, ws=ws)
-    mid = int(np.random.default_rng(99).integers(1, prob.cfg.tokens - 1))
-    tokens = [0, mid, prob.cfg.tokens - 1]
-    _check_sampled(prob, bufs, tokens)
+    _check_against(_full_ref(name), bufs, prob.cfg)
 
 
 # --------------------------------------------------------------------------- #
@@ -535,24 +552,28 @@ def test_forward_with_shared_full_decode_m32(ws):
     _close(bufs.out.cpu().numpy(), _shared_ref(prob, None)["out"], "out")
 
 
-def test_forward_with_shared_full_prefill_sampled():
-    """prefill M=8192 with the shared expert (16 shared table entries), sampled tokens."""
+def test_forward_with_shared_full_prefill_every_element():
+    """prefill M=8192 with the shared expert (16 shared table entries): every element of
+    out, sh_act, sh_out and the routed rows of act and y against the oracle."""
     _need_gpu()
     prob = make_problem("prefill_m8192")
     cfg = prob.cfg
     sw = np.random.default_rng(8).random(cfg.tokens).astype(np.float32)
     layer, bufs = _gpu_forward_shared(prob, sw, ws=True)
     assert layer.rows_per_shared_slot(cfg.tokens) == 512
-    tokens = [0, 4097, cfg.tokens - 1]
-    routed = orc.moe_forward_tokens(prob.x_bf16, prob.topk_ids, prob.topk_weights, cfg.experts,
-                                    *_fns(prob), tokens=tokens, hidden=cfg.hidden)
     shared = tuple(prob.shared_weight(mt) for mt in (MATRIX_GATE, MATRIX_UP, MATRIX_DOWN))
-    sh_act, sh_out = orc.shared_expert(prob.x_bf16[tokens], *shared)
-    ref = routed + sw[tokens, None].astype(np.float64) * sh_out
-    _close(bufs.out.cpu().numpy()[tokens], ref, "out (sampled tokens)")
+    routed = _full_ref("prefill_m8192")
+    ref = orc.moe_forward_shared(prob.x_bf16, prob.topk_ids, prob.topk_weights, cfg.experts,
+                                 None, None, None, hidden=cfg.hidden, inter=cfg.inter,
+                                 shared=shared, shared_weights=sw, routed=routed)
+    _close(bufs.out.cpu().numpy(), ref["out"], "out")
     g_act, g_out = layer.shared_rows_of(bufs, cfg.tokens)
-    _close(g_act.cpu().numpy()[tokens], sh_act, "sh_act (sampled tokens)")
-    _close(g_out.cpu().numpy()[tokens], sh_out, "sh_out (sampled tokens)")
+    _close(g_act.cpu().numpy(), ref["sh_act"], "sh_act")
+    _close(g_out.cpu().numpy(), ref["sh_out"], "sh_out")
+    # The routed experts sort before the shared entries, in the plain routing's order.
+    kept = int(routed["sort"].expert_offsets[-1])
+    _close(bufs.act.cpu().numpy()[:kept], routed["act"][:kept], "act (routed rows)")
+    _close(bufs.y.cpu().numpy()[:kept], routed["y"][:kept], "y (routed rows)")
 
 
 # --------------------------------------------------------------------------- #

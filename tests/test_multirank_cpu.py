@@ -58,8 +58,19 @@ def test_reduce_max_is_identity_without_a_process_group():
 def test_bench_cli_defaults():
     import bench
     args = bench.parse_args([])
-    assert args.gpus == 1 and args.config == "decode_m1" and args.impl == "ours"
+    # The default workload is the largest single-GPU one (prefill M=8192).
+    assert args.gpus == 1 and args.config == "prefill_m8192" and args.impl == "ours"
     assert args.warmup >= 3
+
+
+def test_ncu_traffic_is_dropped_once_the_kernel_sources_change(monkeypatch):
+    import bench
+    key = ("prefill_m8192", "tcgen05")
+    bytes_, _ = bench.NCU_TRAFFIC_BYTES[key]
+    monkeypatch.setitem(bench.NCU_TRAFFIC_BYTES, key, (bytes_, bench.kernel_source_hash("tcgen05")))
+    assert bench.ncu_traffic(*key) == bytes_
+    monkeypatch.setitem(bench.NCU_TRAFFIC_BYTES, key, (bytes_, "000000000000"))
+    assert bench.ncu_traffic(*key) is None
 
 
 def _sharded_worker(rank, world, port, mode, results):

@@ -395,6 +395,26 @@ def test_forward_with_shared_adds_the_weighted_shared_output():
     np.testing.assert_allclose(sh, res1["sh_out"], rtol=1e-10, atol=1e-12)
 
 
+def test_forward_with_shared_takes_a_precomputed_routed_result():
+    prob = make_problem(_tiny_cfg(tokens=5, experts=4, topk=2, hidden=64, inter=32, seed=23))
+    cfg = prob.cfg
+    fns = [lambda e, m=m: prob.expert_weight(m, e) for m in (MATRIX_GATE, MATRIX_UP, MATRIX_DOWN)]
+    c = np.random.default_rng(6).random(cfg.tokens)
+    routed = orc.moe_forward(prob.x_bf16, prob.topk_ids, prob.topk_weights, cfg.experts, *fns,
+                             hidden=cfg.hidden, inter=cfg.inter)
+    a = orc.moe_forward_shared(prob.x_bf16, prob.topk_ids, prob.topk_weights, cfg.experts, *fns,
+                               hidden=cfg.hidden, inter=cfg.inter, shared=_shared(prob),
+                               shared_weights=c)
+    b = orc.moe_forward_shared(prob.x_bf16, prob.topk_ids, prob.topk_weights, cfg.experts,
+                               None, None, None, hidden=cfg.hidden, inter=cfg.inter,
+                               shared=_shared(prob), shared_weights=c, routed=routed)
+    for key in ("act", "y", "out", "sh_act", "sh_out"):
+        np.testing.assert_array_equal(a[key], b[key])
+    np.testing.assert_array_equal(routed["out"], orc.moe_forward(
+        prob.x_bf16, prob.topk_ids, prob.topk_weights, cfg.experts, *fns, hidden=cfg.hidden,
+        inter=cfg.inter)["out"])  # the routed result was not modified in place
+
+
 @pytest.mark.parametrize("m,k,e,rows", [(1, 2, 8, 1), (7, 3, 5, 2), (33, 8, 128, 16), (40, 1, 3, 64)])
 def test_append_shared_routing_layout(m, k, e, rows):
     rng = np.random.default_rng(m + k + e)
@@ -587,6 +607,41 @@ def test_transpose_concat_is_side_by_side_transposes_with_zero_pad(group):
 
 
 # --------------------------------------------------------------------------- #
+# The parity metric: relative L2 error over all elements
+# --------------------------------------------------------------------------- #
+
+def test_relative_l2_hand_computed_pairs():
+    # ref = (1, 2, 2): |ref| = 3; got - ref = (0.3, 0, 0.4): |diff| = 0.5, ratio 1/6.
+    ref = np.array([1.0, 2.0, 2.0])
+    assert orc.relative_l2(ref + np.array([0.3, 0.0, 0.4]), ref) == pytest.approx(1 / 6, rel=1e-14)
+    # The sign of the error does not matter.
+    assert orc.relative_l2(ref - np.array([0.3, 0.0, 0.4]), ref) == pytest.approx(1 / 6, rel=1e-14)
+    # 2-D: one norm over every element (ref = diag(3, 4): |ref| = 5; one off-diagonal 1: 1/5),
+    # not a mean of per-row ratios (that would give (1/3 + 0) / 2).
+    ref2 = np.array([[3.0, 0.0], [0.0, 4.0]])
+    got2 = ref2 + np.array([[0.0, 1.0], [0.0, 0.0]])
+    assert orc.relative_l2(got2, ref2) == pytest.approx(0.2, rel=1e-14)
+    # A float32 result is compared exactly as given: ref = (3, 4), got = (3, 4.5) as f32.
+    assert orc.relative_l2(np.array([3.0, 4.5], np.float32), np.array([3.0, 4.0])) == 0.1
+    assert orc.relative_l2(ref, ref) == 0.0
+
+
+def test_relative_l2_zero_reference():
+    z = np.zeros(5)
+    assert orc.relative_l2(z, z) == 0.0
+    assert orc.relative_l2(np.array([0.0, 0.0, 0.25, 0.0, 0.0]), z) == math.inf
+
+
+def test_relative_l2_uniform_relative_error_is_that_error():
+    # got = (1 + eps) * ref gives |eps| for any nonzero ref, at any common scale.
+    ref = np.random.default_rng(5).standard_normal(1000)
+    for eps in (1e-3, -2.5e-4, 0.5):
+        assert orc.relative_l2((1 + eps) * ref, ref) == pytest.approx(abs(eps), rel=1e-9)
+        assert orc.relative_l2((1 + eps) * 2.0 ** 60 * ref, 2.0 ** 60 * ref) == pytest.approx(
+            abs(eps), rel=1e-9)
+
+
+# --------------------------------------------------------------------------- #
 # Planted mistakes: the pins above must catch them
 # --------------------------------------------------------------------------- #
 
@@ -709,3 +764,37 @@ def test_pins_catch_a_missing_column_offset_in_the_twins(monkeypatch):
     monkeypatch.setattr(orc, "transpose_concat", no_offset)
     with pytest.raises(AssertionError):
         test_transpose_concat_is_side_by_side_transposes_with_zero_pad(16)
+
+
+def test_pins_catch_a_squared_or_misnormalised_relative_l2(monkeypatch):
+    import oracle.nvfp4_moe_oracle as mod
+    real = mod.relative_l2
+    wrong = [lambda g, r: real(g, r) ** 2,                                      # no square root
+             lambda g, r: float(np.max(np.abs(np.asarray(g, np.float64) - r))
+                                / np.max(np.abs(r))),                          # max norm
+             lambda g, r: float(np.linalg.norm(np.asarray(g, np.float64) - r)
+                                / np.linalg.norm(g))]                          # divided by |got|
+    for fn in wrong:
+        monkeypatch.setattr(orc, "relative_l2", fn)
+        with pytest.raises(AssertionError):
+            test_relative_l2_hand_computed_pairs()
+
+
+# --------------------------------------------------------------------------- #
+# The pooled full-size driver of the oracle (tests/_oracle_pool.py)
+# --------------------------------------------------------------------------- #
+
+def test_pooled_oracle_equals_the_plain_oracle():
+    # Expert blocks run in separate processes with the other experts NULL, then
+    # gathered: the same act, y and out as one plain oracle call.
+    from _oracle_pool import moe_forward_pooled
+    cfg = MoEConfig("pool", hidden=512, inter=256, experts=13, topk=3, tokens=40,
+                    router="zipf", seed=61)
+    prob = make_problem(cfg)
+    fns = [lambda e, m=m: prob.expert_weight(m, e) for m in (MATRIX_GATE, MATRIX_UP, MATRIX_DOWN)]
+    ref = orc.moe_forward(prob.x_bf16, prob.topk_ids, prob.topk_weights, cfg.experts, *fns,
+                          hidden=cfg.hidden, inter=cfg.inter)
+    got = moe_forward_pooled(cfg, workers=3, block=2)
+    np.testing.assert_array_equal(got["sort"].sorted_pair_ids, ref["sort"].sorted_pair_ids)
+    for key in ("act", "y", "out"):
+        np.testing.assert_allclose(got[key], ref[key], rtol=1e-12, atol=1e-300)
