@@ -36,6 +36,11 @@ Sources (rustdoc source pages of the "metrale" project; cited by page and item):
 * metrale_model_arch/tp_shard/quant_shard.rs, ``shard_quantized_nvfp4``:
   column-parallel keeps a rank's rows of packed and scale, row-parallel a
   rank's K slice of both; weight_scale_2 is replicated.
+* metrale_model_arch/nemotron_moe/prefill_weights.rs,
+  ``prepare_prefill_weights``: the routed experts of that model have only an
+  up and a down projection (no gate); the forward of such a non-gated expert
+  is act = f(x Wu^T), y = act Wd^T.  The pages do not name f: it is a
+  parameter here (ReLU squared or SiLU).
 * nvfp4_moe_grouped.rs, docs of the two projection launchers: the shared
   expert runs in the same gate+up and down launches as the routed experts,
   over every token, one row per token, with its own weights; its SiLU product
@@ -88,6 +93,10 @@ __all__ = [
     "transpose_u8",
     "shared_expert",
     "moe_forward_shared",
+    "relu2",
+    "ACTIVATIONS",
+    "up_act",
+    "moe_forward_nongated",
     "append_shared_routing",
     "count_bad_scales",
     "shard_nvfp4",
@@ -373,6 +382,54 @@ def moe_forward_tokens(x_bf16, topk_ids, topk_weights, num_experts, gate_fn, up_
             h = silu(wg @ x[t]) * (wu @ x[t])
             out[i] += w[t, s] * (wd @ h)
     return out
+
+
+# --------------------------------------------------------------------------- #
+# Non-gated experts (up and down only)
+# --------------------------------------------------------------------------- #
+
+def relu2(z: np.ndarray) -> np.ndarray:
+    """Squared ReLU: max(z, 0)^2, float64."""
+    z = np.asarray(z, dtype=np.float64)
+    return np.square(np.maximum(z, 0.0))
+
+
+# Activations of a non-gated expert, by name.
+ACTIVATIONS = {"relu2": relu2, "silu": silu}
+
+
+def up_act(x_bf16: np.ndarray, topk: int, rs: RouteSort, up_fn: WeightFn, inter: int,
+           activation: str) -> np.ndarray:
+    """act [P, I] by sorted position: f(x Wu^T) for a non-gated expert, float64.
+
+    prefill_weights.rs, ``prepare_prefill_weights``: the experts hold only up
+    and down.  ``activation`` names f (a key of ACTIVATIONS).  Rows of a NULL
+    expert, and rows past expert_offsets[E], are zero.
+    """
+    f = ACTIVATIONS[activation]
+    x = bf16_bits_to_f64(x_bf16)
+    p_total = rs.sorted_pair_ids.size
+    act = np.zeros((p_total, inter), dtype=np.float64)
+    for a in range(rs.active_count):
+        e = int(rs.active_experts[a])
+        lo, hi = int(rs.expert_offsets[e]), int(rs.expert_offsets[e + 1])
+        wu = _dense(up_fn, e)
+        if wu is None:
+            continue
+        tokens = rs.sorted_pair_ids[lo:hi] // topk
+        act[lo:hi] = f(x[tokens] @ wu.T)
+    return act
+
+
+def moe_forward_nongated(x_bf16, topk_ids, topk_weights, num_experts, up_fn, down_fn,
+                         hidden: int, inter: int, activation: str) -> Dict[str, object]:
+    """The four steps for non-gated experts: sort, act = f(x Wu^T), down, blend."""
+    topk = np.asarray(topk_ids).shape[1]
+    rs = route_sort(topk_ids, num_experts)
+    act = up_act(x_bf16, topk, rs, up_fn, inter, activation)
+    y = down_proj(act, rs, down_fn, hidden)
+    out = blend(y, topk_weights, rs.pair_pos)
+    return {"sort": rs, "act": act, "y": y, "out": out}
 
 
 # --------------------------------------------------------------------------- #

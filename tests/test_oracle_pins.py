@@ -338,6 +338,81 @@ def test_down_is_linear_in_scale2():
 
 
 # --------------------------------------------------------------------------- #
+# Non-gated experts (up and down only)
+# --------------------------------------------------------------------------- #
+
+def _run_nongated(prob, activation):
+    cfg = prob.cfg
+    fns = [lambda e, m=m: prob.expert_weight(m, e) for m in (MATRIX_UP, MATRIX_DOWN)]
+    return orc.moe_forward_nongated(prob.x_bf16, prob.topk_ids, prob.topk_weights, cfg.experts,
+                                    *fns, hidden=cfg.hidden, inter=cfg.inter,
+                                    activation=activation)
+
+
+def test_relu2_special_values():
+    z = np.array([-3.0, -1e-30, -0.0, 0.0, 0.5, 1.5, 7.0, -np.inf, np.inf])
+    np.testing.assert_array_equal(orc.relu2(z), [0.0, 0.0, 0.0, 0.0, 0.25, 2.25, 49.0, 0.0, np.inf])
+    assert orc.ACTIVATIONS["silu"] is orc.silu
+
+
+@pytest.mark.parametrize("activation", ["relu2", "silu"])
+def test_nongated_forward_brute_force_scalar_loops(activation):
+    prob = make_problem(_tiny_cfg(seed=78))
+    cfg = prob.cfg
+    res = _run_nongated(prob, activation)
+    x = orc.bf16_bits_to_f64(prob.x_bf16)
+    f = ((lambda z: max(z, 0.0) * max(z, 0.0)) if activation == "relu2"
+         else (lambda z: z / (1.0 + math.exp(-z))))
+    for t in range(cfg.tokens):
+        acc = [0.0] * cfg.hidden
+        for s in range(cfg.topk):
+            e = int(prob.topk_ids[t, s])
+            wt = float(prob.topk_weights[t, s])
+            h = [f(sum(_scalar_weight(prob, MATRIX_UP, e, n, k) * x[t, k] for k in range(cfg.hidden)))
+                 for n in range(cfg.inter)]
+            for j in range(cfg.hidden):
+                acc[j] += wt * sum(_scalar_weight(prob, MATRIX_DOWN, e, j, i) * h[i] for i in range(cfg.inter))
+        np.testing.assert_allclose(res["out"][t], acc, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("activation", ["relu2", "silu"])
+def test_nongated_single_expert_weight_one_is_the_dense_mlp(activation):
+    prob = make_problem(_tiny_cfg(experts=1, topk=1, tokens=4, hidden=48, inter=32, seed=79))
+    res = _run_nongated(prob, activation)
+    x = orc.bf16_bits_to_f64(prob.x_bf16)
+    wu = orc.dequantize_nvfp4(*prob.expert_weight(MATRIX_UP, 0))
+    wd = orc.dequantize_nvfp4(*prob.expert_weight(MATRIX_DOWN, 0))
+    z = x @ wu.T
+    h = np.maximum(z, 0.0) ** 2 if activation == "relu2" else z / (1.0 + np.exp(-z))
+    np.testing.assert_allclose(res["out"], h @ wd.T, rtol=1e-13, atol=1e-13)
+
+
+def test_nongated_unit_vector_input_picks_an_up_column():
+    # x = e_j: act = f(column j of Wu) (a transposed operand or the gate's
+    # matrix in its place fails this).
+    prob = make_problem(_tiny_cfg(experts=2, topk=1, tokens=3, seed=80))
+    j = [3, 17, 30]
+    prob.x_bf16[:] = 0
+    for t in range(3):
+        prob.x_bf16[t, j[t]] = 0x3F80
+    res = _run_nongated(prob, "relu2")
+    rs = res["sort"]
+    for t in range(3):
+        e = int(prob.topk_ids[t, 0])
+        wu = orc.dequantize_nvfp4(*prob.expert_weight(MATRIX_UP, e))
+        np.testing.assert_array_equal(res["act"][rs.pair_pos[t]], np.maximum(wu[:, j[t]], 0.0) ** 2)
+
+
+def test_nongated_null_expert_rows_are_zero():
+    prob = make_problem(_tiny_cfg(experts=3, topk=1, tokens=6, seed=81), null_experts=[1])
+    res = _run_nongated(prob, "silu")
+    rs = res["sort"]
+    lo, hi = int(rs.expert_offsets[1]), int(rs.expert_offsets[2])
+    assert hi > lo
+    assert not res["act"][lo:hi].any() and not res["y"][lo:hi].any()
+
+
+# --------------------------------------------------------------------------- #
 # Shared expert
 # --------------------------------------------------------------------------- #
 
@@ -798,3 +873,24 @@ def test_pooled_oracle_equals_the_plain_oracle():
     np.testing.assert_array_equal(got["sort"].sorted_pair_ids, ref["sort"].sorted_pair_ids)
     for key in ("act", "y", "out"):
         np.testing.assert_allclose(got[key], ref[key], rtol=1e-12, atol=1e-300)
+
+
+def test_pins_catch_the_activation_applied_after_down(monkeypatch):
+    import oracle.nvfp4_moe_oracle as mod
+    real_down = mod.down_proj
+
+    def late(x_bf16, topk_ids, topk_weights, num_experts, up_fn, down_fn, hidden, inter,
+             activation):
+        rs = mod.route_sort(topk_ids, num_experts)
+        x = mod.bf16_bits_to_f64(x_bf16)
+        act = np.zeros((rs.sorted_pair_ids.size, inter))
+        for a in range(rs.active_count):
+            e = int(rs.active_experts[a])
+            lo, hi = int(rs.expert_offsets[e]), int(rs.expert_offsets[e + 1])
+            act[lo:hi] = x[rs.sorted_pair_ids[lo:hi] // np.asarray(topk_ids).shape[1]] @ mod._dense(up_fn, e).T
+        y = mod.ACTIVATIONS[activation](real_down(act, rs, down_fn, hidden))
+        return {"sort": rs, "act": act, "y": y, "out": mod.blend(y, topk_weights, rs.pair_pos)}
+
+    monkeypatch.setattr(orc, "moe_forward_nongated", late)
+    with pytest.raises(AssertionError):
+        test_nongated_single_expert_weight_one_is_the_dense_mlp("relu2")
