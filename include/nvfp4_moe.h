@@ -262,6 +262,50 @@ NVFP4_MOE_API int nvfp4_moe_gate_up_silu_noalloc(
     uint32_t num_tokens, uint32_t topk, uint32_t num_experts, cudaStream_t stream);
 
 /*
+ * Activation of a non-gated expert (nvfp4_moe_up_act).
+ */
+typedef enum {
+  NVFP4_MOE_ACT_RELU2 = 1, /* f(z) = max(z, 0)^2 (squared ReLU) */
+  NVFP4_MOE_ACT_SILU = 2   /* f(z) = z / (1 + exp(-z))          */
+} nvfp4_moe_activation;
+
+/*
+ * Step 2 for non-gated experts, which hold only an up and a down projection
+ * (the routed experts whose prefill twins `prepare_prefill_weights` in
+ * nemotron_moe/prefill_weights.rs builds from up and down alone).  The pages
+ * do not name the activation; the caller picks it (nvfp4_moe_activation).
+ *
+ *   x           bf16 bits [num_tokens, k_hidden]
+ *   up          table of [n_inter, k_hidden] NVFP4 weights
+ *   act         f32 [P, n_inter]  out: row r = sorted position r:
+ *               act[r, n] = f(sum_k Wu[n,k] x[t,k]), t = sorted_pair_ids[r] / topk.
+ *               Rows >= kept pairs are untouched; a NULL expert's rows are zero.
+ *   activation  NVFP4_MOE_ACT_RELU2 or NVFP4_MOE_ACT_SILU (else NVFP4_MOE_EINVAL).
+ *   the rest    as for nvfp4_moe_gate_up_silu_ex.
+ * n_inter % 128 == 0.  Step 3 (nvfp4_moe_down) then reads act unchanged.
+ */
+NVFP4_MOE_API int nvfp4_moe_up_act(const uint16_t* x, nvfp4_expert_tables up, float* act,
+                                   const int32_t* expert_offsets, const int32_t* sorted_pair_ids,
+                                   const int32_t* active_experts, const int32_t* active_count,
+                                   uint32_t n_inter, uint32_t k_hidden, uint32_t cap,
+                                   uint32_t num_tokens, uint32_t topk, int activation,
+                                   const nvfp4_moe_launch_opts* opts, cudaStream_t stream);
+
+/*
+ * nvfp4_moe_up_act with a workspace, opening the tcgen05 path under the rules
+ * of nvfp4_moe_gate_up_silu_ws, with an output width that is a multiple of
+ * 256 (two halves of 128 rows of the one matrix per CTA).  The workspace is
+ * sized by nvfp4_moe_workspace_bytes as for the gated layer.
+ */
+NVFP4_MOE_API int nvfp4_moe_up_act_ws(const uint16_t* x, nvfp4_expert_tables up, float* act,
+                                      const int32_t* expert_offsets, const int32_t* sorted_pair_ids,
+                                      const int32_t* active_experts, const int32_t* active_count,
+                                      uint32_t n_inter, uint32_t k_hidden, uint32_t cap,
+                                      uint32_t num_tokens, uint32_t topk, uint32_t num_experts,
+                                      int activation, const nvfp4_moe_launch_opts* opts,
+                                      void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Device error word of the library: 0, or 1 if a tcgen05-path kernel gave up
  * waiting on one of its barriers (its outputs are then not valid).  Kernels
  * never trap; they set this word and exit.  Reading it synchronises the
@@ -338,6 +382,18 @@ NVFP4_MOE_API int nvfp4_moe_forward(const uint16_t* x, const int32_t* topk_ids,
                                     uint32_t topk, uint32_t num_experts, uint32_t hidden,
                                     uint32_t inter, const nvfp4_moe_launch_opts* opts,
                                     void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * The four steps of one layer of non-gated experts in one call:
+ * nvfp4_moe_route_sort, nvfp4_moe_up_act(_ws) with `activation`,
+ * nvfp4_moe_down(_ws) and nvfp4_moe_blend.  Buffers, workspace and errors as
+ * for nvfp4_moe_forward.
+ */
+NVFP4_MOE_API int nvfp4_moe_forward_nongated(
+    const uint16_t* x, const int32_t* topk_ids, const float* topk_weights, nvfp4_expert_tables up,
+    nvfp4_expert_tables down, const nvfp4_moe_buffers* buffers, uint32_t num_tokens, uint32_t topk,
+    uint32_t num_experts, uint32_t hidden, uint32_t inter, int activation,
+    const nvfp4_moe_launch_opts* opts, void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * Load-time twin builder: byte transpose [rows, cols] -> [cols, rows]

@@ -6,6 +6,7 @@ containers.  Importing it without the built library raises ImportError.
 """
 
 from ._binding import (  # noqa: F401
+    ACTIVATIONS,
     LIB_PATH,
     PATH_AUTO,
     PATH_DECODE,
@@ -26,6 +27,7 @@ from ._binding import (  # noqa: F401
     down_ws,
     exported_symbols,
     forward,
+    forward_nongated,
     gate_up_silu,
     gate_up_silu_ws,
     route_sort,
@@ -35,6 +37,8 @@ from ._binding import (  # noqa: F401
     transpose_concat,
     transpose_concat_into,
     transpose_u8,
+    up_act,
+    up_act_ws,
     workspace_bytes,
 )
 from .layer import (  # noqa: F401

@@ -50,6 +50,8 @@ class Buffers(ctypes.Structure):
 
 
 PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
+# nvfp4_moe_activation: the activation of a non-gated expert.
+ACTIVATIONS = {"relu2": 1, "silu": 2}
 SHARD_COLUMN, SHARD_ROW = 0, 1
 
 _sig = {
@@ -83,6 +85,16 @@ _sig = {
                                   ExpertTables, ctypes.POINTER(Buffers), c_u32, c_u32, c_u32, c_u32,
                                   c_u32, ctypes.POINTER(LaunchOpts), c_void_p, ctypes.c_size_t,
                                   c_void_p]),
+    "nvfp4_moe_up_act": (c_int, [c_void_p, ExpertTables, c_void_p, c_void_p, c_void_p, c_void_p,
+                                 c_void_p, c_u32, c_u32, c_u32, c_u32, c_u32, c_int,
+                                 ctypes.POINTER(LaunchOpts), c_void_p]),
+    "nvfp4_moe_up_act_ws": (c_int, [c_void_p, ExpertTables, c_void_p, c_void_p, c_void_p, c_void_p,
+                                    c_void_p, c_u32, c_u32, c_u32, c_u32, c_u32, c_u32, c_int,
+                                    ctypes.POINTER(LaunchOpts), c_void_p, ctypes.c_size_t, c_void_p]),
+    "nvfp4_moe_forward_nongated": (c_int, [c_void_p, c_void_p, c_void_p, ExpertTables, ExpertTables,
+                                           ctypes.POINTER(Buffers), c_u32, c_u32, c_u32, c_u32, c_u32,
+                                           c_int, ctypes.POINTER(LaunchOpts), c_void_p,
+                                           ctypes.c_size_t, c_void_p]),
     "nvfp4_moe_append_shared": (c_int, [c_void_p, c_void_p, c_void_p, c_u32, c_u32, c_u32, c_u32,
                                         c_void_p, c_void_p, c_void_p]),
     "nvfp4_moe_shared_slots": (c_u32, [c_u32, c_u32]),
@@ -378,3 +390,57 @@ def forward(x, topk_ids, topk_weights, gate: ExpertTables, up: ExpertTables, dow
         _ptr(x, None, "x"), _ptr(topk_ids, torch.int32, "topk_ids"),
         _ptr(topk_weights, torch.float32, "topk_weights"), gate, up, down, ctypes.byref(buffers),
         m, k, num_experts, hidden, inter, _opts(path, split, tiles, depth), wp, wn, _stream(stream)))
+
+
+def _activation(activation) -> int:
+    if activation not in ACTIVATIONS:
+        raise ValueError(f"activation must be one of {sorted(ACTIVATIONS)}")
+    return ACTIVATIONS[activation]
+
+
+def up_act(x, up: ExpertTables, act, expert_offsets, sorted_pair_ids, active_experts, active_count,
+           n_inter, k_hidden, cap, num_tokens, topk, activation, path=0, split=0, tiles=0, depth=0,
+           stream=None) -> None:
+    """nvfp4_moe_up_act: act = f(x Wu^T) by sorted position (non-gated experts)."""
+    if x.dtype not in (torch.bfloat16, torch.uint16, torch.int16):
+        raise TypeError("x: expected bf16 (or its uint16 bits)")
+    _check("nvfp4_moe_up_act", _lib.nvfp4_moe_up_act(
+        _ptr(x, None, "x"), up, _ptr(act, torch.float32, "act"),
+        _ptr(expert_offsets, torch.int32, "expert_offsets"),
+        _ptr(sorted_pair_ids, torch.int32, "sorted_pair_ids"),
+        _ptr(active_experts, torch.int32, "active_experts"),
+        _ptr(active_count, torch.int32, "active_count"),
+        n_inter, k_hidden, cap, num_tokens, topk, _activation(activation),
+        _opts(path, split, tiles, depth), _stream(stream)))
+
+
+def up_act_ws(x, up: ExpertTables, act, expert_offsets, sorted_pair_ids, active_experts,
+              active_count, n_inter, k_hidden, cap, num_tokens, topk, num_experts, activation,
+              workspace, path=0, split=0, tiles=0, depth=0, stream=None) -> None:
+    """nvfp4_moe_up_act_ws: nvfp4_moe_up_act with a workspace (tcgen05 path)."""
+    if x.dtype not in (torch.bfloat16, torch.uint16, torch.int16):
+        raise TypeError("x: expected bf16 (or its uint16 bits)")
+    wp, wn = _ws(workspace)
+    _check("nvfp4_moe_up_act_ws", _lib.nvfp4_moe_up_act_ws(
+        _ptr(x, None, "x"), up, _ptr(act, torch.float32, "act"),
+        _ptr(expert_offsets, torch.int32, "expert_offsets"),
+        _ptr(sorted_pair_ids, torch.int32, "sorted_pair_ids"),
+        _ptr(active_experts, torch.int32, "active_experts"),
+        _ptr(active_count, torch.int32, "active_count"),
+        n_inter, k_hidden, cap, num_tokens, topk, num_experts, _activation(activation),
+        _opts(path, split, tiles, depth), wp, wn, _stream(stream)))
+
+
+def forward_nongated(x, topk_ids, topk_weights, up: ExpertTables, down: ExpertTables,
+                     buffers: Buffers, num_experts, hidden, inter, activation, workspace=None,
+                     path=0, split=0, tiles=0, depth=0, stream=None) -> None:
+    """nvfp4_moe_forward_nongated: the four steps of a layer of non-gated experts."""
+    if x.dtype not in (torch.bfloat16, torch.uint16, torch.int16):
+        raise TypeError("x: expected bf16 (or its uint16 bits)")
+    m, k = topk_ids.shape
+    wp, wn = (None, 0) if workspace is None else _ws(workspace)
+    _check("nvfp4_moe_forward_nongated", _lib.nvfp4_moe_forward_nongated(
+        _ptr(x, None, "x"), _ptr(topk_ids, torch.int32, "topk_ids"),
+        _ptr(topk_weights, torch.float32, "topk_weights"), up, down, ctypes.byref(buffers),
+        m, k, num_experts, hidden, inter, _activation(activation), _opts(path, split, tiles, depth),
+        wp, wn, _stream(stream)))

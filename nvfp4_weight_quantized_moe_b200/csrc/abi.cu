@@ -54,7 +54,7 @@ DecodePlan plan_decode(int mode, uint64_t tokens, uint64_t pairs, uint32_t num_e
   }
   if (p.tiles < 1) p.tiles = 1;
   if (p.tiles == 3 || p.tiles > 4) p.tiles = 4;
-  if (mode == kModeDown && p.tiles > 2) p.tiles = 2;
+  if (mode != kModeGateUp && p.tiles > 2) p.tiles = 2;
   if (o && o->tiles) p.tiles = o->tiles;
   const uint64_t active = cap < pairs ? cap : pairs;
   auto ctas = [&](int split) {
@@ -324,6 +324,89 @@ int nvfp4_moe_down_ws(const float* act, nvfp4_expert_tables down, float* y,
   return status_of(launch_tc(kModeDown, nt, a, workspace, num_tokens, n_hidden, k_inter, cap, stream));
 }
 
+int nvfp4_moe_up_act(const uint16_t* x, nvfp4_expert_tables up, float* act,
+                     const int32_t* expert_offsets, const int32_t* sorted_pair_ids,
+                     const int32_t* active_experts, const int32_t* active_count,
+                     uint32_t n_inter, uint32_t k_hidden, uint32_t cap, uint32_t num_tokens,
+                     uint32_t topk, int activation, const nvfp4_moe_launch_opts* opts,
+                     cudaStream_t stream) {
+  if (activation != NVFP4_MOE_ACT_RELU2 && activation != NVFP4_MOE_ACT_SILU) return NVFP4_MOE_EINVAL;
+  if (n_inter == 0 || n_inter % 128 != 0 || k_hidden == 0 || k_hidden % 256 != 0 || topk == 0 ||
+      cap > 65535)
+    return NVFP4_MOE_ESHAPE;
+  const uint64_t pairs = (uint64_t)num_tokens * topk;
+  if (pairs > kMaxPairs) return NVFP4_MOE_ESHAPE;
+  if (pairs == 0 || cap == 0) return NVFP4_MOE_OK;
+  if (x == nullptr || act == nullptr || expert_offsets == nullptr || sorted_pair_ids == nullptr ||
+      active_experts == nullptr || active_count == nullptr || !tables_ok(up))
+    return NVFP4_MOE_EINVAL;
+  const int path = opts ? opts->path : 0;
+  if (path != 0 && path != 1) return NVFP4_MOE_EINVAL;
+  const DecodePlan plan = plan_decode(kModeUpAct, num_tokens, pairs, cap, cap, n_inter, opts);
+  if (!grouped_plan_supported(kModeUpAct, plan)) return NVFP4_MOE_EINVAL;
+  GroupedArgs a{};
+  a.src = x;
+  a.packed0 = up.packed_ptrs;
+  a.scale0 = up.scale_ptrs;
+  a.s2_0 = up.scale2;
+  a.out = act;
+  a.offsets = expert_offsets;
+  a.sorted_pair_ids = sorted_pair_ids;
+  a.active_experts = active_experts;
+  a.active_count = active_count;
+  a.N = n_inter;
+  a.K = k_hidden;
+  a.topk = topk;
+  a.activation = activation;
+  return status_of(launch_grouped(kModeUpAct, plan, a, cap, stream));
+}
+
+int nvfp4_moe_up_act_ws(const uint16_t* x, nvfp4_expert_tables up, float* act,
+                        const int32_t* expert_offsets, const int32_t* sorted_pair_ids,
+                        const int32_t* active_experts, const int32_t* active_count,
+                        uint32_t n_inter, uint32_t k_hidden, uint32_t cap, uint32_t num_tokens,
+                        uint32_t topk, uint32_t num_experts, int activation,
+                        const nvfp4_moe_launch_opts* opts, void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream) {
+  const int path = opts ? opts->path : 0;
+  if (path < 0 || path > 2) return NVFP4_MOE_EINVAL;
+  if (activation != NVFP4_MOE_ACT_RELU2 && activation != NVFP4_MOE_ACT_SILU) return NVFP4_MOE_EINVAL;
+  if (!use_tc(n_inter, 256, (uint64_t)num_tokens * topk, num_experts, opts)) {
+    if (path == 2) return NVFP4_MOE_ESHAPE;
+    return nvfp4_moe_up_act(x, up, act, expert_offsets, sorted_pair_ids, active_experts, active_count,
+                            n_inter, k_hidden, cap, num_tokens, topk, activation, opts, stream);
+  }
+  if (k_hidden == 0 || k_hidden % 256 != 0 || topk == 0 || cap > 65535 || num_experts == 0 ||
+      num_experts > kMaxExperts)
+    return NVFP4_MOE_ESHAPE;
+  const uint64_t pairs = (uint64_t)num_tokens * topk;
+  if (pairs > kMaxPairs) return NVFP4_MOE_ESHAPE;
+  if (pairs == 0 || cap == 0) return NVFP4_MOE_OK;
+  if (x == nullptr || act == nullptr || expert_offsets == nullptr || sorted_pair_ids == nullptr ||
+      active_experts == nullptr || active_count == nullptr || !tables_ok(up) || workspace == nullptr)
+    return NVFP4_MOE_EINVAL;
+  if (workspace_bytes < tc_workspace_bytes(num_tokens, topk, k_hidden, n_inter)) return NVFP4_MOE_EINVAL;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return NVFP4_MOE_EINVAL;
+  const int nt = plan_tc_rows(pairs, num_experts, opts ? opts->tiles : 0);
+  if (nt != 16 && nt != 128) return NVFP4_MOE_EINVAL;
+  GroupedArgs a{};
+  a.src = x;
+  a.packed0 = up.packed_ptrs;
+  a.scale0 = up.scale_ptrs;
+  a.s2_0 = up.scale2;
+  a.out = act;
+  a.offsets = expert_offsets;
+  a.sorted_pair_ids = sorted_pair_ids;
+  a.active_experts = active_experts;
+  a.active_count = active_count;
+  a.N = n_inter;
+  a.K = k_hidden;
+  a.topk = topk;
+  a.num_experts = num_experts;
+  a.activation = activation;
+  return status_of(launch_tc(kModeUpAct, nt, a, workspace, num_tokens, k_hidden, n_inter, cap, stream));
+}
+
 int nvfp4_moe_blend(const float* y, const float* topk_weights, const int32_t* pair_pos,
                     float* out_f32, uint16_t* out_bf16, uint32_t num_tokens, uint32_t topk,
                     uint32_t hidden, cudaStream_t stream) {
@@ -364,6 +447,43 @@ int nvfp4_moe_forward(const uint16_t* x, const int32_t* topk_ids, const float* t
     st = nvfp4_moe_gate_up_silu_ex(x, gate, up, b->act, b->expert_offsets, b->sorted_pair_ids,
                                    b->active_experts, b->active_count, inter, hidden, cap, num_tokens,
                                    topk, opts, stream);
+    if (st != NVFP4_MOE_OK) return st;
+    st = nvfp4_moe_down_ex(b->act, down, b->y, b->expert_offsets, b->active_experts, b->active_count,
+                           hidden, inter, cap, num_tokens, topk, opts, stream);
+  }
+  if (st != NVFP4_MOE_OK) return st;
+  return nvfp4_moe_blend(b->y, topk_weights, b->pair_pos, b->out_f32, b->out_bf16, num_tokens, topk,
+                         hidden, stream);
+}
+
+int nvfp4_moe_forward_nongated(const uint16_t* x, const int32_t* topk_ids,
+                               const float* topk_weights, nvfp4_expert_tables up,
+                               nvfp4_expert_tables down, const nvfp4_moe_buffers* b,
+                               uint32_t num_tokens, uint32_t topk, uint32_t num_experts,
+                               uint32_t hidden, uint32_t inter, int activation,
+                               const nvfp4_moe_launch_opts* opts, void* workspace,
+                               size_t workspace_bytes, cudaStream_t stream) {
+  if (b == nullptr) return NVFP4_MOE_EINVAL;
+  if (activation != NVFP4_MOE_ACT_RELU2 && activation != NVFP4_MOE_ACT_SILU) return NVFP4_MOE_EINVAL;
+  const uint64_t pairs = (uint64_t)num_tokens * topk;
+  if (pairs > kMaxPairs) return NVFP4_MOE_ESHAPE;
+  const uint32_t cap = nvfp4_moe_active_cap(num_experts, (uint32_t)pairs);
+  int st = nvfp4_moe_route_sort(topk_ids, num_tokens, topk, num_experts, b->expert_offsets,
+                                b->sorted_pair_ids, b->pair_pos, b->active_experts, b->active_count,
+                                b->status, stream);
+  if (st != NVFP4_MOE_OK) return st;
+  if (workspace != nullptr) {
+    st = nvfp4_moe_up_act_ws(x, up, b->act, b->expert_offsets, b->sorted_pair_ids, b->active_experts,
+                             b->active_count, inter, hidden, cap, num_tokens, topk, num_experts,
+                             activation, opts, workspace, workspace_bytes, stream);
+    if (st != NVFP4_MOE_OK) return st;
+    st = nvfp4_moe_down_ws(b->act, down, b->y, b->expert_offsets, b->active_experts, b->active_count,
+                           hidden, inter, cap, num_tokens, topk, num_experts, opts, workspace,
+                           workspace_bytes, stream);
+  } else {
+    st = nvfp4_moe_up_act(x, up, b->act, b->expert_offsets, b->sorted_pair_ids, b->active_experts,
+                          b->active_count, inter, hidden, cap, num_tokens, topk, activation, opts,
+                          stream);
     if (st != NVFP4_MOE_OK) return st;
     st = nvfp4_moe_down_ex(b->act, down, b->y, b->expert_offsets, b->active_experts, b->active_count,
                            hidden, inter, cap, num_tokens, topk, opts, stream);

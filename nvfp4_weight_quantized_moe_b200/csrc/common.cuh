@@ -116,6 +116,13 @@ NVM_DEV float warp_max(float v) {
 // fast divide returns 0, the limit of SiLU there.
 NVM_DEV float silu_f32(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
+// Activation of a non-gated expert: 1 = squared ReLU, 2 = SiLU (the values of
+// nvfp4_moe_activation).
+NVM_DEV float activation_f32(int act, float z) {
+  if (act == 1) return z > 0.0f ? z * z : 0.0f;
+  return silu_f32(z);
+}
+
 // ---------------------------------------------------------------------------
 // Programmatic dependent launch and L2 prefetch
 // ---------------------------------------------------------------------------

@@ -1,10 +1,13 @@
 // Grouped NVFP4 expert projections for decode-shaped batches (few rows per
-// expert): gate+up with the fused FP32 SiLU product, and down.
+// expert): gate+up with the fused FP32 SiLU product, down, and the up
+// projection of a non-gated expert with its activation.
 //
 // Operation: metrale_model_layers/layers/ops/nvfp4_moe_grouped.rs,
 // `moe_expert_gate_up_act_nvfp4_grouped` and `moe_expert_down_act_nvfp4_grouped`:
 // one launch covers every active expert (grid y = slot in the device list of
-// active experts, bounded by `cap`), output rows are sorted positions.
+// active experts, bounded by `cap`), output rows are sorted positions.  The
+// non-gated mode serves experts with only up and down projections
+// (metrale_model_arch/nemotron_moe/prefill_weights.rs, `prepare_prefill_weights`).
 //
 // Design (sm_100a).  The weights are the bytes that matter.  Every expert
 // weight byte is streamed from HBM once per pass with 16-byte
@@ -33,7 +36,7 @@
 // FP32.  act is split into f16 hi + lo (two MMAs) so the down projection keeps
 // about 22 bits of the FP32 SiLU product.
 //
-// Pipeline.  A CTA (4 warps) owns 64 (gate+up) or 128 (down) output rows of one
+// Pipeline.  A CTA (4 warps) owns 64 (gate+up) or 128 (down, up+activation) output rows of one
 // expert over all of K; with S > 1 its warps split K S ways over 64/S or 128/S
 // rows and add their sums through shared memory at the end (one row per
 // expert needs that parallelism).  Per 256-k chunk, the activation rows of the
@@ -58,9 +61,9 @@ struct Cfg {
   static constexpr int NQ = WARPS / S;
   static constexpr int ROWS_PER_WARP = MODE == kModeGateUp ? 16 : 32;
   static constexpr int ROWS_PER_CTA = NQ * ROWS_PER_WARP;
-  static constexpr int PLANES = MODE == kModeGateUp ? 1 : 2;
+  static constexpr int PLANES = MODE == kModeDown ? 2 : 1;
   static constexpr int GROUP = 8 * TILES;
-  static constexpr int BPE = MODE == kModeGateUp ? 2 : 4;         // bytes per activation element
+  static constexpr int BPE = MODE == kModeDown ? 4 : 2;           // bytes per activation element
   static constexpr int ITEMS = S * GROUP;                           // row-chunks per iteration
   static constexpr int FRAG_BYTES = PLANES * S * TILES * kTileChunkBytes;  // one buffer
   static constexpr int RAW_BYTES = ITEMS * 256 * BPE;                        // one stage
@@ -112,12 +115,13 @@ __global__ void __launch_bounds__(128) grouped_mma_kernel(GroupedArgs a) {
   const int s = warp % S, q = warp / S;
   const int g = lane >> 2, c = lane & 3;
 
-  // Gate+up reads the route sort's outputs at once, so it waits for the previous
-  // kernel first.  Down starts before gate+up has finished: the route sort's
-  // outputs are complete by the time it launches (gate+up lets it launch only
-  // after its own wait), and the weights are never written, so down looks up
-  // its expert and starts fetching its weights before it waits for act.
-  if (MODE == kModeGateUp) {
+  // Gate+up (and up+activation) reads the route sort's outputs at once, so it
+  // waits for the previous kernel first.  Down starts before gate+up has
+  // finished: the route sort's outputs are complete by the time it launches
+  // (gate+up lets it launch only after its own wait), and the weights are never
+  // written, so down looks up its expert and starts fetching its weights before
+  // it waits for act.
+  if (MODE != kModeDown) {
     griddep_wait();
     griddep_launch_dependents();
   }
@@ -187,7 +191,7 @@ __global__ void __launch_bounds__(128) grouped_mma_kernel(GroupedArgs a) {
   for (int t = 0; t < 2; ++t) {
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      const int n = nw + (MODE == kModeDown ? 16 * t : 0) + g + 8 * r;
+      const int n = nw + (MODE != kModeGateUp ? 16 * t : 0) + g + 8 * r;
       const uint8_t* pb = (MODE == kModeGateUp && t == 1) ? P1 : P0;
       const uint8_t* sb = (MODE == kModeGateUp && t == 1) ? S1 : S0;
       wp[t][r] = pb + (size_t)n * (K >> 1) + (size_t)my_ch0 * 128 + c * 32;
@@ -225,7 +229,7 @@ __global__ void __launch_bounds__(128) grouped_mma_kernel(GroupedArgs a) {
     __syncthreads();  // the previous group is done with shared memory
     if (tid < C::GROUP) {
       int src = -1;
-      if (tid < nrows) src = MODE == kModeGateUp ? a.sorted_pair_ids[g0 + tid] / (int)a.topk : g0 + tid;
+      if (tid < nrows) src = MODE != kModeDown ? a.sorted_pair_ids[g0 + tid] / (int)a.topk : g0 + tid;
       rowsrc[tid] = src;
     }
     __syncthreads();
@@ -254,7 +258,7 @@ __global__ void __launch_bounds__(128) grouped_mma_kernel(GroupedArgs a) {
         uint8_t* dst = frag + buf * C::FRAG_BYTES + (ss * TILES + (r >> 3)) * kTileChunkBytes;
         float f[8];
         int u0[C::BPE / 2];  // first 4-k unit of each 16-byte piece
-        if (MODE == kModeGateUp) {
+        if (MODE != kModeDown) {
           const uint4 v = *reinterpret_cast<const uint4*>(rp + lane * 16);
           const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -276,7 +280,7 @@ __global__ void __launch_bounds__(128) grouped_mma_kernel(GroupedArgs a) {
         for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
         const int ex = f16_range_exponent(warp_max(m));
         const float mul = exp2i(-ex);
-        if (MODE == kModeGateUp) {
+        if (MODE != kModeDown) {
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             uint2 o;
@@ -466,6 +470,9 @@ __global__ void __launch_bounds__(128) grouped_mma_kernel(GroupedArgs a) {
               const float gv = acc[0][u][i] * s2a;
               const float uv = acc[1][u][i] * s2b;
               orow[n] = silu_f32(gv) * uv;
+            } else if (MODE == kModeUpAct) {
+              orow[n] = activation_f32(a.activation, acc[0][u][i] * s2a);
+              orow[n + 16] = activation_f32(a.activation, acc[1][u][i] * s2a);
             } else {
               orow[n] = acc[0][u][i] * s2a;
               orow[n + 16] = acc[1][u][i] * s2a;
@@ -507,6 +514,13 @@ cudaError_t launch_grouped(int mode, const DecodePlan& p, const GroupedArgs& a, 
   NVM_CASE(kModeDown, 1, 2, 2)
   NVM_CASE(kModeDown, 1, 1, 3)
   NVM_CASE(kModeDown, 1, 2, 3)
+  // Up+activation: the down kernel's row layout over BF16 token rows.
+  NVM_CASE(kModeUpAct, 4, 1, 2)
+  NVM_CASE(kModeUpAct, 2, 1, 2)
+  NVM_CASE(kModeUpAct, 1, 1, 2)
+  NVM_CASE(kModeUpAct, 1, 2, 2)
+  NVM_CASE(kModeUpAct, 1, 1, 3)
+  NVM_CASE(kModeUpAct, 1, 2, 3)
 #undef NVM_CASE
   return cudaErrorInvalidValue;
 }

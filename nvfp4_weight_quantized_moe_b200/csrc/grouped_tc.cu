@@ -1,5 +1,6 @@
 // Grouped NVFP4 expert projections on the sm_100a tensor cores (tcgen05),
-// gate+up with the fused FP32 SiLU product and down, for any rows per expert.
+// gate+up with the fused FP32 SiLU product, down, and the up projection of a
+// non-gated expert with its activation, for any rows per expert.
 //
 // Operation: metrale_model_layers/layers/ops/nvfp4_moe_grouped.rs,
 // `moe_expert_gate_up_act_nvfp4_grouped` and `moe_expert_down_act_nvfp4_grouped`
@@ -7,7 +8,8 @@
 // rows are sorted positions).
 //
 // Design.  A CTA owns 128 weight rows of one expert (for gate+up: 128 gate rows
-// and the same 128 up rows; for down: 256 rows as two halves) and walks the
+// and the same 128 up rows; for down and up+activation: 256 rows of the one
+// matrix as two halves) and walks the
 // expert's sorted token rows in groups of NT.  Every operand moves by TMA:
 //   * Warp 9 (one thread) loads weight tiles: per 256 k, for each of the two
 //     128-row matrices, 128 rows x 128 bytes of packed nibbles (128-byte
@@ -88,7 +90,7 @@ constexpr uint32_t pow2_at_least(uint32_t v) {
 // and up, or the two row halves of down).
 template <int MODE, int NT>
 struct TcCfg {
-  static constexpr int PLANES = MODE == kModeGateUp ? 1 : 2;  // down: f16 hi + lo
+  static constexpr int PLANES = MODE == kModeDown ? 2 : 1;  // down: f16 hi + lo
   static constexpr int ROWS_PER_CTA = MODE == kModeGateUp ? 128 : 256;
   static constexpr int B_PLANE_BYTES = NT * kStageK * 2;       // NT rows x 64 k, f16
   static constexpr int B_SLOT_BYTES = PLANES * B_PLANE_BYTES;
@@ -305,6 +307,7 @@ struct TcArgs {
   const int32_t* active_experts;
   const int32_t* active_count;
   uint32_t N, K;
+  int activation;             // up+activation: kActRelu2 or kActSilu
 };
 
 // Registers: 128-token tiles run one CTA per SM, 16-token tiles two.  The
@@ -447,12 +450,15 @@ __global__ void __launch_bounds__(kThreads) __maxnreg__(NT <= 16 ? 80 : 168)
   } else if (warp == kMmaWarp) {
     // ================= MMA issuer =================
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_f16_f32(128, NT);
       for (int g = 0; g < ngroups; ++g) {
         if (g > 0) {
           wait(bar_dfree, (g - 1) & 1);  // the epilogue has read the previous group's D
           tc_fence_after();
         }
+        // A group short of NT rows (an expert's last) runs its MMAs with N =
+        // its rows rounded up to 16: MMA time scales with N.
+        const int rows_g = min(NT, row_hi - (row_lo + g * NT));
+        const uint32_t idesc = idesc_f16_f32(128, NT > 16 ? (rows_g + 15) & ~15 : NT);
         for (int st = 0; st < nst; ++st) {
           const uint32_t ga = (uint32_t)(g * nst + st);
           const uint32_t aslot = ga % C::SA, bslot = ga % C::SB;
@@ -497,7 +503,8 @@ __global__ void __launch_bounds__(kThreads) __maxnreg__(NT <= 16 ? 80 : 168)
     const int tbase = pmat * HALF;
     const int n = n0 + prow;
 
-    // Down: read D and store it directly, then hand D back to the MMA.
+    // Down (and up+activation): read D and store it directly (through the
+    // activation for up+activation), then hand D back to the MMA.
     auto epilogue_down = [&](int g) {
       const int g0 = row_lo + g * NT;
       const int nrows = min(NT, row_hi - g0);
@@ -524,8 +531,15 @@ __global__ void __launch_bounds__(kThreads) __maxnreg__(NT <= 16 ? 80 : 168)
             const float xm = __shfl_sync(0xffffffffu, xm_l, tt + j);
             if (ok && t < nrows) {
               float* dst = a.out + (size_t)(g0 + t) * N + n;
-              dst[0] = __uint_as_float(d0[j]) * xm * s2a;
-              dst[128] = __uint_as_float(d1[j]) * xm * s2a;
+              const float v0 = __uint_as_float(d0[j]) * xm * s2a;
+              const float v1 = __uint_as_float(d1[j]) * xm * s2a;
+              if constexpr (MODE == kModeUpAct) {
+                dst[0] = activation_f32(a.activation, v0);
+                dst[128] = activation_f32(a.activation, v1);
+              } else {
+                dst[0] = v0;
+                dst[128] = v1;
+              }
             }
           }
         }
@@ -773,6 +787,7 @@ cudaError_t launch_tc(int mode, int nt, const GroupedArgs& g, void* workspace, u
   a.active_count = g.active_count;
   a.N = g.N;
   a.K = g.K;
+  a.activation = g.activation;
 
   // Templates of the weight maps (address replaced per expert on the device):
   // nibbles [N, K/2] u8 in 128 x 128-byte boxes with 128-byte swizzle, scales
@@ -802,6 +817,24 @@ cudaError_t launch_tc(int mode, int nt, const GroupedArgs& g, void* workspace, u
     a.wmaps = w.maps_gu;
     if (nt == 16) return launch_tc_impl<kModeGateUp, 16>(a, b0, b1, cap, stream);
     return launch_tc_impl<kModeGateUp, 128>(a, b0, b1, cap, stream);
+  }
+  if (mode == kModeUpAct) {
+    // x packed as for gate+up; one weight table, two row halves per CTA.
+    err = launch_pdl(pack_x_sorted_kernel, dim3((unsigned)((pairs + 7) / 8)), dim3(256), 0, stream,
+                     static_cast<const uint16_t*>(g.src), (int)pairs, (int)g.K, (int)g.topk, g.sorted_pair_ids,
+                     g.offsets + g.num_experts, w.xs, w.xexp);
+    if (err != cudaSuccess) return err;
+    err = launch_pdl(build_weight_maps_kernel, dim3(g.num_experts), dim3(128), 0, stream, t_nib, t_scale,
+                     g.packed0, g.scale0, g.packed0, g.scale0, 2, w.maps_gu);
+    if (err != cudaSuccess) return err;
+    err = make_map_2d(&b0, w.xs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, pairs, g.K, box_rows, kStageK,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+    if (err != cudaSuccess) return err;
+    b1 = b0;
+    a.bexp = w.xexp;
+    a.wmaps = w.maps_gu;
+    if (nt == 16) return launch_tc_impl<kModeUpAct, 16>(a, b0, b1, cap, stream);
+    return launch_tc_impl<kModeUpAct, 128>(a, b0, b1, cap, stream);
   }
   // Rows past offsets[E] (dropped pairs) are not packed: offsets[E] bounds the grid's work.
   {

@@ -6,7 +6,11 @@
 
 namespace nvm {
 
-enum { kModeGateUp = 0, kModeDown = 1 };
+// Projection modes: gate+up with the fused SiLU product; down; the up
+// projection of a non-gated expert followed by an activation.
+enum { kModeGateUp = 0, kModeDown = 1, kModeUpAct = 2 };
+// Activations of a non-gated expert (the values of nvfp4_moe_activation).
+enum { kActRelu2 = 1, kActSilu = 2 };
 
 // Limits shared by every entry point: expert table entries and routed pairs
 // per call.
@@ -24,7 +28,8 @@ inline int plan_tc_rows(uint64_t pairs, uint32_t num_experts, int tiles) {
 
 // Arguments of the grouped projection kernels.  Mode gate+up reads BF16 x
 // [M, K] and two weight tables (gate, up) with the same [N, K]; mode down
-// reads FP32 act [P, K] and one table.  `out` is [P, N] FP32 by sorted position.
+// reads FP32 act [P, K] and one table; mode up+activation reads BF16 x and
+// one table.  `out` is [P, N] FP32 by sorted position.
 struct GroupedArgs {
   const void* src;
   const void* const* packed0;
@@ -40,6 +45,7 @@ struct GroupedArgs {
   const int32_t* active_count;
   uint32_t N, K, topk;
   uint32_t num_experts;
+  int activation;  // mode up+activation: kActRelu2 or kActSilu
 };
 
 // Launch shape of the decode path (grouped_mma.cu):

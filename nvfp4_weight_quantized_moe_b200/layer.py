@@ -156,6 +156,11 @@ class _Tables:
 class NVFP4MoE:
     """The grouped NVFP4 expert forward of one layer, optionally with a shared expert.
 
+    ``gate=None`` makes a layer of non-gated experts (up and down only, as the
+    experts whose twins ``prepare_prefill_weights`` builds in
+    nemotron_moe/prefill_weights.rs): act = f(x Wu^T) with f = ``activation``
+    ("relu2" or "silu"), then down and blend as usual.
+
     ``shared`` = (gate, up, down) projections of one expert (E = 1) with the
     routed experts' shapes: every token also runs it, in the same gate+up and
     down launches (nvfp4_moe_append_shared), and ``out`` adds its output times
@@ -164,15 +169,24 @@ class NVFP4MoE:
     one group of CTAs; by default about the routed rows per expert.
     """
 
-    def __init__(self, gate: NVFP4Projection, up: NVFP4Projection, down: NVFP4Projection, topk: int,
-                 shared=None, shared_rows: int = 0):
-        if not (gate.num_experts == up.num_experts == down.num_experts):
+    def __init__(self, gate: Optional[NVFP4Projection], up: NVFP4Projection, down: NVFP4Projection,
+                 topk: int, shared=None, shared_rows: int = 0, activation: Optional[str] = None):
+        if gate is None:
+            if activation not in B.ACTIVATIONS:
+                raise ValueError(f"a non-gated layer needs activation in {sorted(B.ACTIVATIONS)}")
+            if shared is not None:
+                raise ValueError("the shared expert is built for gated layers only")
+        elif activation is not None:
+            raise ValueError("activation applies to non-gated layers (gate=None)")
+        ref = gate if gate is not None else up
+        if not (ref.num_experts == up.num_experts == down.num_experts):
             raise ValueError("expert counts differ")
-        if gate.n != up.n or gate.k != up.k or down.n != gate.k or down.k != gate.n:
+        if ref.n != up.n or ref.k != up.k or down.n != up.k or down.k != up.n:
             raise ValueError("gate/up must be [I, H] and down [H, I]")
         self.gate, self.up, self.down = gate, up, down
-        self.num_experts = gate.num_experts
-        self.hidden, self.inter = gate.k, gate.n
+        self.activation = activation
+        self.num_experts = up.num_experts
+        self.hidden, self.inter = up.k, up.n
         self.topk = topk
         self.shared = None
         self.shared_rows = int(shared_rows)
@@ -195,9 +209,10 @@ class NVFP4MoE:
         if self.shared is not None:
             sg, su, sd = self.shared
             shared = (sg.shard(col, rank, tp), su.shard(col, rank, tp), sd.shard(row, rank, tp))
-        return NVFP4MoE(self.gate.shard(col, rank, tp), self.up.shard(col, rank, tp),
-                        self.down.shard(row, rank, tp), self.topk, shared=shared,
-                        shared_rows=self.shared_rows)
+        gate = self.gate.shard(col, rank, tp) if self.gate is not None else None
+        return NVFP4MoE(gate, self.up.shard(col, rank, tp), self.down.shard(row, rank, tp),
+                        self.topk, shared=shared, shared_rows=self.shared_rows,
+                        activation=self.activation)
 
     def expert_parallel(self, rank: int, world: int) -> "NVFP4MoE":
         """This rank's layer under expert parallelism: copies of its block of
@@ -205,9 +220,11 @@ class NVFP4MoE:
         shared expert, if any, runs on rank 0 only.  The rank's ``out`` is a
         partial sum (see :func:`all_reduce_out`)."""
         lo, hi = expert_owner_range(self.num_experts, world, rank)
-        projs = [p.expert_block(lo, hi) for p in (self.gate, self.up, self.down)]
+        projs = [p.expert_block(lo, hi) if p is not None else None
+                 for p in (self.gate, self.up, self.down)]
         shared = self.shared if rank == 0 else None
-        return NVFP4MoE(*projs, self.topk, shared=shared, shared_rows=self.shared_rows)
+        return NVFP4MoE(*projs, self.topk, shared=shared, shared_rows=self.shared_rows,
+                        activation=self.activation)
 
     # -- shared expert bookkeeping ------------------------------------------------
     def rows_per_shared_slot(self, num_tokens: int) -> int:
@@ -239,14 +256,14 @@ class NVFP4MoE:
         k, e = self._route_shape(num_tokens)
         if self.shared is not None:
             e = 1024  # the library's largest table: enough entries for any batch size
-        return MoEBuffers(num_tokens, k, e, self.hidden, self.inter, self.gate.packed.device,
+        return MoEBuffers(num_tokens, k, e, self.hidden, self.inter, self.up.packed.device,
                           out_bf16, shared=self.shared is not None)
 
     def workspace(self, num_tokens: int) -> torch.Tensor:
         """Device workspace of the tcgen05 path for batches of up to num_tokens."""
         k, _ = self._route_shape(num_tokens)
         n = B.workspace_bytes(num_tokens, k, self.hidden, self.inter)
-        return torch.empty(max(n, 1), dtype=torch.uint8, device=self.gate.packed.device)
+        return torch.empty(max(n, 1), dtype=torch.uint8, device=self.up.packed.device)
 
     def forward(self, x: torch.Tensor, topk_ids: torch.Tensor, topk_weights: torch.Tensor,
                 bufs: Optional[MoEBuffers] = None, path: int = 0, split: int = 0,
@@ -268,6 +285,9 @@ class NVFP4MoE:
             bufs = self.buffers(m)
         if m > bufs.num_tokens:
             raise ValueError("buffers were sized for fewer tokens")
+        if self.gate is None:
+            return self._forward_nongated(x, topk_ids, topk_weights, bufs, path, split, tiles,
+                                          depth, workspace, stream, steps, shared_weights)
         gate_t, up_t, down_t = self.gate.tables, self.up.tables, self.down.tables
         topk, num_experts = self.topk, self.num_experts
         if self.shared is not None:
@@ -307,6 +327,36 @@ class NVFP4MoE:
             B.down_ws(bufs.act, down_t, bufs.y, bufs.expert_offsets, bufs.active_experts,
                       bufs.active_count, self.hidden, self.inter, cap, m, topk, num_experts,
                       workspace, **opts)
+        B.blend(bufs.y, topk_weights, bufs.pair_pos, bufs.out, bufs.out_bf16, stream=stream)
+        return bufs
+
+    def _forward_nongated(self, x, topk_ids, topk_weights, bufs, path, split, tiles, depth,
+                          workspace, stream, steps, shared_weights) -> MoEBuffers:
+        if shared_weights is not None:
+            raise ValueError("shared_weights given to a layer without a shared expert")
+        opts = dict(path=path, split=split, tiles=tiles, depth=depth, stream=stream)
+        if not steps:
+            B.forward_nongated(x, topk_ids, topk_weights, self.up.tables, self.down.tables,
+                               bufs.c_buffers, self.num_experts, self.hidden, self.inter,
+                               self.activation, workspace=workspace, **opts)
+            return bufs
+        m, topk, e = x.shape[0], self.topk, self.num_experts
+        cap = B.active_cap(e, m * topk)
+        B.route_sort(topk_ids, e, bufs.expert_offsets[:e + 1], bufs.sorted_pair_ids,
+                     bufs.pair_pos, bufs.active_experts[:e], bufs.active_count, bufs.status,
+                     stream=stream)
+        if workspace is None:
+            B.up_act(x, self.up.tables, bufs.act, bufs.expert_offsets, bufs.sorted_pair_ids,
+                     bufs.active_experts, bufs.active_count, self.inter, self.hidden, cap, m, topk,
+                     self.activation, **opts)
+            B.down(bufs.act, self.down.tables, bufs.y, bufs.expert_offsets, bufs.active_experts,
+                   bufs.active_count, self.hidden, self.inter, cap, m, topk, **opts)
+        else:
+            B.up_act_ws(x, self.up.tables, bufs.act, bufs.expert_offsets, bufs.sorted_pair_ids,
+                        bufs.active_experts, bufs.active_count, self.inter, self.hidden, cap, m,
+                        topk, e, self.activation, workspace, **opts)
+            B.down_ws(bufs.act, self.down.tables, bufs.y, bufs.expert_offsets, bufs.active_experts,
+                      bufs.active_count, self.hidden, self.inter, cap, m, topk, e, workspace, **opts)
         B.blend(bufs.y, topk_weights, bufs.pair_pos, bufs.out, bufs.out_bf16, stream=stream)
         return bufs
 

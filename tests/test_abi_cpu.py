@@ -84,6 +84,30 @@ def test_host_validation_rejects_bad_shapes_without_a_gpu(lib):
                                    ctypes.byref(bad), None) == 1, opts
 
 
+def test_nongated_calls_check_activation_and_shapes_on_the_host(lib):
+    import nvfp4_weight_quantized_moe_b200._binding as B
+    L = B._lib
+    t = B.ExpertTables(8, 8, 8)
+    p8 = ctypes.c_void_p(8)
+    # unknown activation (0, 3), then N not a multiple of 128, K not a multiple of 256
+    for act in (0, 3):
+        assert L.nvfp4_moe_up_act(p8, t, p8, p8, p8, p8, p8, 256, 512, 1, 1, 1, act, None, None) == 1
+    assert L.nvfp4_moe_up_act(p8, t, p8, p8, p8, p8, p8, 192, 512, 1, 1, 1, 1, None, None) == 2
+    assert L.nvfp4_moe_up_act(p8, t, p8, p8, p8, p8, p8, 256, 320, 1, 1, 1, 2, None, None) == 2
+    # NULL up table with work to do; no tokens is a no-op
+    t0 = B.ExpertTables(None, None, None)
+    assert L.nvfp4_moe_up_act(p8, t0, p8, p8, p8, p8, p8, 256, 512, 1, 1, 1, 1, None, None) == 1
+    assert L.nvfp4_moe_up_act(p8, t0, p8, p8, p8, p8, p8, 256, 512, 1, 0, 1, 1, None, None) == 0
+    # tcgen05 path forced on a width that is not a multiple of 256; short workspace
+    opts = B.LaunchOpts(2, 0, 0, 0)
+    assert L.nvfp4_moe_up_act_ws(p8, t, p8, p8, p8, p8, p8, 384, 512, 8, 64, 4, 8, 1,
+                                 ctypes.byref(opts), ctypes.c_void_p(1 << 20), 1 << 30, None) == 2
+    assert L.nvfp4_moe_up_act_ws(p8, t, p8, p8, p8, p8, p8, 512, 512, 8, 64, 4, 8, 1,
+                                 ctypes.byref(opts), ctypes.c_void_p(1 << 20), 1024, None) == 1
+    assert L.nvfp4_moe_forward_nongated(p8, p8, p8, t, t, None, 1, 1, 8, 512, 512, 1, None, None, 0,
+                                        None) == 1
+
+
 def test_active_cap_and_status_strings(lib):
     import nvfp4_weight_quantized_moe_b200 as m
     assert m.active_cap(128, 8) == 8 and m.active_cap(8, 65536) == 8

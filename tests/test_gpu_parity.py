@@ -577,6 +577,97 @@ def test_forward_with_shared_full_prefill_every_element():
 
 
 # --------------------------------------------------------------------------- #
+# Non-gated experts (up and down only) with a chosen activation
+# --------------------------------------------------------------------------- #
+
+def _nongated_ref(prob, activation):
+    cfg = prob.cfg
+    fns = [lambda e, m=m: prob.expert_weight(m, e, cache=True) for m in (MATRIX_UP, MATRIX_DOWN)]
+    return orc.moe_forward_nongated(prob.x_bf16, prob.topk_ids, prob.topk_weights, cfg.experts,
+                                    *fns, hidden=cfg.hidden, inter=cfg.inter, activation=activation)
+
+
+def _check_nongated(prob, bufs, activation):
+    ref = _nongated_ref(prob, activation)
+    rs = ref["sort"]
+    _check_sort(bufs, rs, prob.cfg.experts, prob.cfg.pairs)
+    kept = int(rs.expert_offsets[-1])
+    _close(bufs.act.cpu().numpy()[:kept], ref["act"][:kept], "act")
+    _close(bufs.y.cpu().numpy()[:kept], ref["y"][:kept], "y")
+    _close(bufs.out.cpu().numpy(), ref["out"], "out")
+
+
+def _gpu_forward_nongated(prob, activation, ws=False, null=(), **opts):
+    from workloads.device import upload_inputs, upload_layer
+    import nvfp4_weight_quantized_moe_b200 as nvm
+    layer = upload_layer(prob, activation=activation)
+    x, ids, w = upload_inputs(prob)
+    bufs = layer.buffers(prob.cfg.tokens)
+    for t in (bufs.act, bufs.y, bufs.out):
+        t.fill_(float("nan"))
+    workspace = layer.workspace(prob.cfg.tokens) if ws else None
+    if workspace is not None:
+        workspace.fill_(0xFF)
+    layer.forward(x, ids, w, bufs, workspace=workspace, **opts)
+    torch.cuda.synchronize()
+    assert nvm.device_error() == 0
+    return layer, bufs
+
+
+# (path options): decode kernel automatic and forced shapes; tcgen05 16- and 128-row passes.
+NONGATED_PATHS = [dict(), dict(path=1, split=4, tiles=1, depth=2), dict(path=1, split=1, tiles=2, depth=3),
+                  dict(ws=True, path=2, tiles=2), dict(ws=True, path=2, tiles=16)]
+
+
+@pytest.mark.parametrize("opts", NONGATED_PATHS, ids=lambda o: "-".join(f"{k}{v}" for k, v in o.items()) or "auto")
+@pytest.mark.parametrize("activation", ["relu2", "silu"])
+@pytest.mark.parametrize("name", ["tiny", "ragged", "hot", "zipf", "longk"])
+def test_nongated_forward_small(name, activation, opts):
+    _need_gpu()
+    prob = make_problem(SMALL[name])
+    _, bufs = _gpu_forward_nongated(prob, activation, **opts)
+    _check_nongated(prob, bufs, activation)
+
+
+@pytest.mark.parametrize("ws", [False, True], ids=["decode-path", "tcgen05"])
+def test_nongated_null_experts_and_four_step_calls(ws):
+    _need_gpu()
+    prob = make_problem(SMALL["hot"], null_experts=[0, 4])
+    opts = dict(ws=True, path=2) if ws else {}
+    _, one = _gpu_forward_nongated(prob, "relu2", **opts)
+    _check_nongated(prob, one, "relu2")
+    _, four = _gpu_forward_nongated(prob, "relu2", steps=True, **opts)
+    for f in ("act", "y", "out"):
+        assert torch.equal(getattr(one, f).view(torch.int32), getattr(four, f).view(torch.int32)), f
+
+
+@pytest.mark.parametrize("ws", [False, True], ids=["decode-path", "tcgen05"])
+def test_nongated_full_decode_m32(ws):
+    # The skewed decode workload's shapes (H4096, I1536, 128 experts) as a non-gated layer.
+    _need_gpu()
+    prob = make_problem("decode_m32")
+    _, bufs = _gpu_forward_nongated(prob, "relu2", ws=ws)
+    _check_nongated(prob, bufs, "relu2")
+
+
+def test_nongated_rejects_an_unknown_activation():
+    _need_gpu()
+    import nvfp4_weight_quantized_moe_b200 as nvm
+    from nvfp4_weight_quantized_moe_b200 import _binding as B
+    prob = make_problem(SMALL["tiny"])
+    layer, bufs = _gpu_forward_nongated(prob, "silu")
+    cfg = prob.cfg
+    from workloads.device import upload_inputs
+    x, ids, w = upload_inputs(prob)
+    st = B._lib.nvfp4_moe_up_act(x.data_ptr(), layer.up.tables, bufs.act.data_ptr(),
+                                 bufs.expert_offsets.data_ptr(), bufs.sorted_pair_ids.data_ptr(),
+                                 bufs.active_experts.data_ptr(), bufs.active_count.data_ptr(),
+                                 cfg.inter, cfg.hidden, 2, cfg.tokens, cfg.topk, 7, None, None)
+    assert st == 1
+    assert nvm.device_error() == 0
+
+
+# --------------------------------------------------------------------------- #
 # Load-time scale check: bit-exact counts
 # --------------------------------------------------------------------------- #
 

@@ -43,14 +43,17 @@ def upload_shared(prob: MoEProblem, device="cuda"):
     return tuple(out)
 
 
-def upload_layer(prob: MoEProblem, device="cuda", shared: bool = False, shared_rows: int = 0):
+def upload_layer(prob: MoEProblem, device="cuda", shared: bool = False, shared_rows: int = 0,
+                 activation=None):
+    """The problem's layer on the device; ``activation`` given: a non-gated layer
+    (up and down only) with that activation."""
     from nvfp4_weight_quantized_moe_b200 import NVFP4MoE
 
-    return NVFP4MoE(upload_projection(prob, MATRIX_GATE, device),
-                    upload_projection(prob, MATRIX_UP, device),
+    gate = None if activation is not None else upload_projection(prob, MATRIX_GATE, device)
+    return NVFP4MoE(gate, upload_projection(prob, MATRIX_UP, device),
                     upload_projection(prob, MATRIX_DOWN, device), prob.cfg.topk,
                     shared=upload_shared(prob, device) if shared else None,
-                    shared_rows=shared_rows)
+                    shared_rows=shared_rows, activation=activation)
 
 
 def upload_inputs(prob: MoEProblem, device="cuda"):
