@@ -678,6 +678,8 @@ __global__ void __launch_bounds__(kThreads) __maxnreg__(NT <= 16 ? 80 : 168)
   }
 }
 
+#include "grouped_tc_pair.cuh"
+
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
@@ -774,8 +776,10 @@ cudaError_t launch_tc(int mode, int nt, const GroupedArgs& g, void* workspace, u
                       uint32_t hidden, uint32_t inter, uint32_t cap, cudaStream_t stream) {
   const uint64_t pairs = (uint64_t)tokens * g.topk;
   const WsLayout w = ws_layout(workspace, pairs, hidden, inter);
-  if (g.num_experts == 0 || g.num_experts > kMaxExperts || (nt != 16 && nt != 128))
+  if (g.num_experts == 0 || g.num_experts > kMaxExperts || (nt != 16 && nt != 128 && nt != kPairNT))
     return cudaErrorInvalidValue;
+  // 192-row passes run the pair kernel: 64-row weight boxes, 96-row token boxes.
+  const bool pair = nt == kPairNT;
   TcArgs a{};
   a.packed0 = g.packed0;
   a.packed1 = g.packed1 != nullptr ? g.packed1 : g.packed0;
@@ -793,13 +797,14 @@ cudaError_t launch_tc(int mode, int nt, const GroupedArgs& g, void* workspace, u
   // nibbles [N, K/2] u8 in 128 x 128-byte boxes with 128-byte swizzle, scales
   // [N, K/16] u8 in 128 x 16-byte boxes.
   CUtensorMap t_nib, t_scale, b0, b1;
-  cudaError_t err = make_map_2d(&t_nib, workspace, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.N, g.K / 2, 128,
+  const uint32_t w_rows = pair ? kPairWBoxRows : 128;
+  cudaError_t err = make_map_2d(&t_nib, workspace, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.N, g.K / 2, w_rows,
                                 kTileK / 2, CU_TENSOR_MAP_SWIZZLE_128B);
   if (err != cudaSuccess) return err;
-  err = make_map_2d(&t_scale, workspace, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.N, g.K / 16, 128, kTileK / 16,
+  err = make_map_2d(&t_scale, workspace, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.N, g.K / 16, w_rows, kTileK / 16,
                     CU_TENSOR_MAP_SWIZZLE_NONE);
   if (err != cudaSuccess) return err;
-  const uint32_t box_rows = (uint32_t)nt;
+  const uint32_t box_rows = pair ? (uint32_t)kPairHalf : (uint32_t)nt;
 
   if (mode == kModeGateUp) {
     err = launch_pdl(pack_x_sorted_kernel, dim3((unsigned)((pairs + 7) / 8)), dim3(256), 0, stream,
@@ -815,6 +820,7 @@ cudaError_t launch_tc(int mode, int nt, const GroupedArgs& g, void* workspace, u
     b1 = b0;
     a.bexp = w.xexp;
     a.wmaps = w.maps_gu;
+    if (pair) return launch_tc_pair_impl<kModeGateUp>(a, b0, b1, cap, stream);
     if (nt == 16) return launch_tc_impl<kModeGateUp, 16>(a, b0, b1, cap, stream);
     return launch_tc_impl<kModeGateUp, 128>(a, b0, b1, cap, stream);
   }
@@ -833,6 +839,7 @@ cudaError_t launch_tc(int mode, int nt, const GroupedArgs& g, void* workspace, u
     b1 = b0;
     a.bexp = w.xexp;
     a.wmaps = w.maps_gu;
+    if (pair) return launch_tc_pair_impl<kModeUpAct>(a, b0, b1, cap, stream);
     if (nt == 16) return launch_tc_impl<kModeUpAct, 16>(a, b0, b1, cap, stream);
     return launch_tc_impl<kModeUpAct, 128>(a, b0, b1, cap, stream);
   }
@@ -858,6 +865,7 @@ cudaError_t launch_tc(int mode, int nt, const GroupedArgs& g, void* workspace, u
   if (err != cudaSuccess) return err;
   a.bexp = w.aexp;
   a.wmaps = w.maps_down;
+  if (pair) return launch_tc_pair_impl<kModeDown>(a, b0, b1, cap, stream);
   if (nt == 16) return launch_tc_impl<kModeDown, 16>(a, b0, b1, cap, stream);
   return launch_tc_impl<kModeDown, 128>(a, b0, b1, cap, stream);
 }

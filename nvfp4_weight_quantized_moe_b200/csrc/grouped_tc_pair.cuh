@@ -1,0 +1,401 @@
+// Pair form of the tcgen05 projection kernel, for experts with many token
+// rows (prefill-shaped batches).  Part of grouped_tc.cu (included there once,
+// after the one-CTA kernel): it uses that file's packing, tensor maps and
+// arguments.
+//
+// A cluster of two CTAs runs tcgen05.mma.cta_group::2: M = 256 weight rows
+// (128 per CTA, each decoded into its own CTA's tensor memory) times N = up to
+// 192 token rows (each CTA loads half of the token tile into its own shared
+// memory), FP32 accumulators in both CTAs' tensor memory (each CTA holds its
+// 128 rows x all N columns).  Per FLOP this halves the decode work and the
+// tensor-memory stores of the one-CTA kernel at 128-token passes and cuts its
+// shared-memory traffic by a third, which is what bounded that kernel's MMA
+// rate.
+//
+// Rows.  Gate+up: CTA r of the pair owns outputs n0 + 64 r .. + 63, and its
+// 128 A rows interleave them: TMEM lane 2j holds gate row n0 + 64 r + j, lane
+// 2j + 1 the up row of the same n, so the SiLU(gate) * up epilogue pairs
+// neighbouring lanes with one shuffle.  Down and up+activation: CTA r owns 128
+// consecutive rows n0 + 128 r .. + 127 of the one matrix.
+//
+// Roles (15 warps per CTA), synchronised by mbarriers only:
+//   warps 0-7   decoders: TMEM lane 32 (w % 4) + l, k half w / 4 of each
+//               64-k stage; 16 nibble bytes and 2 scales per stage from the
+//               weight tile in shared memory, exact E2M1 x E4M3 -> f16,
+//               tcgen05.st into a 4-stage A ring; each warp then arrives on the
+//               first CTA's full_a barrier (the peer's warps remotely);
+//   warp 8      first CTA: MMA issuer (one thread): waits for both CTAs' A
+//               stage and token tile, issues the pair MMAs into one of two D
+//               buffers, commits each stage and each pass to barriers in both
+//               CTAs (multicast commit);
+//   warp 9      weight tiles by TMA (its CTA's 128 rows, 256 k per tile);
+//   warp 10     token tiles by TMA, its half of each 64-k stage, completion
+//               signalled on the first CTA's full_b barrier (pair TMA form);
+//   warps 11-14 epilogue: tcgen05.ld of the finished D buffer, FP32 scaling,
+//               SiLU(g) * u or the activation, stores by sorted position, then
+//               the D buffer is handed back (remote arrive for the peer).
+// D is double-buffered, so a pass's epilogue overlaps the next pass's MMAs.
+// Every wait is bounded; on timeout the CTA flags the device error word and
+// skips its remaining waits; both CTAs meet at a cluster barrier before the
+// tensor memory is freed.
+
+namespace {
+
+constexpr int kPairNT = 192;                // token rows per pass of the pair (MMA N, max)
+constexpr int kPairHalf = kPairNT / 2;      // token rows each CTA loads
+constexpr int kPairMmaWarp = 8;
+constexpr int kPairWLoadWarp = 9;
+constexpr int kPairBLoadWarp = 10;
+constexpr int kPairEpiWarp0 = 11;           // warps 11..14
+constexpr int kPairThreads = 32 * 15;
+constexpr int kPairWBoxRows = 64;           // rows per weight TMA box
+constexpr int kPairWNib = 128 * 128;        // nibble bytes of a CTA's weight tile (128 rows x 256 k)
+constexpr int kPairWSlot = kPairWNib + 128 * 16;
+
+template <int MODE>
+struct PairCfg {
+  static constexpr int PLANES = MODE == kModeDown ? 2 : 1;           // down: f16 hi + lo
+  static constexpr int ROWS_PER_PAIR = MODE == kModeGateUp ? 128 : 256;  // outputs n per pair
+  static constexpr int B_PLANE_BYTES = kPairHalf * kStageK * 2;      // 96 rows x 64 k f16
+  static constexpr int B_SLOT_BYTES = PLANES * B_PLANE_BYTES;
+  static constexpr int A_COLS = 32;                                   // TMEM columns per A stage
+  static constexpr int D_COLS = kPairNT;                              // per D buffer
+  static constexpr int SA = 4;
+  static constexpr int WS = 2;
+  static constexpr int SB = MODE == kModeDown ? 4 : 8;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int OFF_W = 0;
+  static constexpr int OFF_B = WS * kPairWSlot;
+  static constexpr int OFF_BAR = OFF_B + SB * B_SLOT_BYTES;
+  // full_w[WS], empty_w[WS], full_b[SB], mma_done[SB], full_a[SA], done[2], dfree[2]
+  static constexpr int NBAR = 2 * WS + 2 * SB + SA + 4;
+  static constexpr int OFF_TMEM = OFF_BAR + 8 * NBAR;
+  static constexpr int OFF_ABORT = OFF_TMEM + 16;
+  static constexpr int SMEM = OFF_ABORT + 16 + 1024;
+  static_assert(2 * D_COLS + SA * A_COLS <= (int)TMEM_COLS, "TMEM budget");
+  static_assert(B_PLANE_BYTES % 1024 == 0 && kPairWSlot % 1024 == 0, "TMA tiles stay 1024-byte aligned");
+  static_assert(SB >= SA, "mma_done also tracks the A ring");
+  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+};
+
+}  // namespace
+
+template <int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
+    grouped_tc_pair_kernel(const TcArgs a, const __grid_constant__ CUtensorMap tm_b0,
+                           const __grid_constant__ CUtensorMap tm_b1) {
+  using C = PairCfg<MODE>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t s_base = (raw_base + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (s_base - raw_base);
+  const uint32_t full_w = s_base + C::OFF_BAR;
+  const uint32_t empty_w = full_w + 8 * C::WS;
+  const uint32_t full_b = empty_w + 8 * C::WS;   // used in the first CTA
+  const uint32_t mma_done = full_b + 8 * C::SB;  // both CTAs (multicast commit)
+  const uint32_t full_a = mma_done + 8 * C::SB;  // used in the first CTA
+  const uint32_t bar_done = full_a + 8 * C::SA;  // [2], both CTAs (multicast commit)
+  const uint32_t bar_dfree = bar_done + 16;      // [2], used in the first CTA
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_ABORT);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();
+  griddep_wait();
+  griddep_launch_dependents();
+  // Both CTAs of a pair read the same slot and expert, so they take the same
+  // early exits and the same loop counts.
+  const int slot_idx = blockIdx.y;
+  if (slot_idx >= *a.active_count) return;
+  const int e = a.active_experts[slot_idx];
+  const int row_lo = a.offsets[e], row_hi = a.offsets[e + 1];
+  const int N = (int)a.N, K = (int)a.K;
+  const int n_cta = (int)(blockIdx.x >> 1) * C::ROWS_PER_PAIR + (int)rank * (C::ROWS_PER_PAIR / 2);
+  if (a.packed0[e] == nullptr || (MODE == kModeGateUp && a.packed1[e] == nullptr)) {
+    // NULL expert: this CTA's outputs of its rows are zero.
+    constexpr int W = C::ROWS_PER_PAIR / 2;
+    for (int i = tid; i < (row_hi - row_lo) * W; i += kPairThreads)
+      a.out[(size_t)(row_lo + i / W) * N + n_cta + i % W] = 0.0f;
+    return;
+  }
+  const int ngroups = (row_hi - row_lo + kPairNT - 1) / kPairNT;
+  if (ngroups <= 0) return;
+  const int nst = K / kStageK;
+  const int ntile = K / kTileK;
+
+  // ---- set-up: barriers, tensor memory, then both CTAs meet ----
+  if (tid == 0) {
+    for (int s = 0; s < C::WS; ++s) {
+      mbar_init(full_w + 8 * s, 1);
+      mbar_init(empty_w + 8 * s, 8);
+    }
+    for (int s = 0; s < C::SB; ++s) {
+      mbar_init(full_b + 8 * s, 1);
+      mbar_init(mma_done + 8 * s, 1);
+    }
+    for (int s = 0; s < C::SA; ++s) mbar_init(full_a + 8 * s, 16);  // 8 decoder warps per CTA
+    for (int d = 0; d < 2; ++d) {
+      mbar_init(bar_done + 8 * d, 1);
+      mbar_init(bar_dfree + 8 * d, 8);  // 4 epilogue warps per CTA
+    }
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  if (warp == kPairMmaWarp) {
+    tmem_alloc_pair(smem_u32(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the first CTA's barriers exist before any remote arrive or TMA signal
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t tmem_a = tmem + 2 * C::D_COLS;  // A ring after the two D buffers
+
+  auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+    if (*abort_flag) return false;
+    if (mbar_wait(bar, parity)) return true;
+    *abort_flag = 1;
+    return false;
+  };
+  auto wait_cl = [&](uint32_t bar, uint32_t parity) -> bool {
+    if (*abort_flag) return false;
+    if (mbar_wait_cluster(bar, parity)) return true;
+    *abort_flag = 1;
+    return false;
+  };
+  // MMAs of stage x have completed (frees B slot x % SB and A slot x % SA).
+  auto wait_mma = [&](uint32_t x) -> bool { return wait(mma_done + 8 * (x % C::SB), (x / C::SB) & 1); };
+  // Token rows of pass g: the MMA's N is its rows rounded up to 32; each CTA
+  // loads N / 2 of them.
+  auto pass_n = [&](int g) -> int {
+    const int rows = min(kPairNT, row_hi - (row_lo + g * kPairNT));
+    return (rows + 31) & ~31;
+  };
+
+  if (warp == kPairWLoadWarp) {
+    // ================= weight tile loader (both CTAs) =================
+    if (lane == 0) {
+      const CUtensorMap* m = a.wmaps + (size_t)e * kMapsPerExpert;
+      const CUtensorMap* nib0 = m;
+      const CUtensorMap* sc0 = m + 1;
+      const CUtensorMap* nib1 = MODE == kModeGateUp ? m + 2 : m;
+      const CUtensorMap* sc1 = MODE == kModeGateUp ? m + 3 : m + 1;
+      tmap_acquire(nib0);
+      tmap_acquire(sc0);
+      if (MODE == kModeGateUp) {
+        tmap_acquire(nib1);
+        tmap_acquire(sc1);
+      }
+      // Gate+up: 64 gate rows then the same 64 up rows; else 128 rows in two boxes.
+      const int y0 = n_cta, y1 = MODE == kModeGateUp ? n_cta : n_cta + kPairWBoxRows;
+      uint32_t issued = 0;
+      for (int g = 0; g < ngroups && !*abort_flag; ++g) {
+        for (int kt = 0; kt < ntile; ++kt) {
+          const uint32_t slot = issued % C::WS, round = issued / C::WS;
+          if (round > 0 && !wait(empty_w + 8 * slot, (round - 1) & 1)) break;
+          const uint32_t dst = s_base + C::OFF_W + slot * kPairWSlot;
+          const uint32_t bar = full_w + 8 * slot;
+          mbar_arrive_expect_tx(bar, kPairWSlot);
+          tma_load_2d(dst, nib0, kt * (kTileK / 2), y0, bar);
+          tma_load_2d(dst + kPairWNib / 2, nib1, kt * (kTileK / 2), y1, bar);
+          tma_load_2d(dst + kPairWNib, sc0, kt * (kTileK / 16), y0, bar);
+          tma_load_2d(dst + kPairWNib + kPairWBoxRows * 16, sc1, kt * (kTileK / 16), y1, bar);
+          ++issued;
+        }
+      }
+      for (uint32_t i = issued > (uint32_t)C::WS ? issued - C::WS : 0; i < issued; ++i)
+        mbar_wait(full_w + 8 * (i % C::WS), (i / C::WS) & 1);
+    }
+  } else if (warp == kPairBLoadWarp) {
+    // ================= token tile loader (both CTAs, half each) =================
+    if (lane == 0) {
+      const uint32_t lead_full_b = mapa_shared(full_b, 0);
+      uint32_t issued = 0;
+      for (int g = 0; g < ngroups && !*abort_flag; ++g) {
+        const int half = pass_n(g) / 2;
+        const int y = row_lo + g * kPairNT + (int)rank * half;
+        for (int st = 0; st < nst; ++st) {
+          const uint32_t slot = issued % C::SB, round = issued / C::SB;
+          if (round > 0 && !wait_mma(issued - C::SB)) break;
+          const uint32_t dst = s_base + C::OFF_B + slot * C::B_SLOT_BYTES;
+          // The first CTA's barrier counts both CTAs' bytes.
+          if (rank == 0) mbar_arrive_expect_tx(full_b + 8 * slot, 2 * C::B_SLOT_BYTES);
+          tma_load_2d_pair(dst, &tm_b0, st * kStageK, y, lead_full_b + 8 * slot);
+          if constexpr (MODE == kModeDown)
+            tma_load_2d_pair(dst + C::B_PLANE_BYTES, &tm_b1, st * kStageK, y, lead_full_b + 8 * slot);
+          ++issued;
+        }
+      }
+      // The last tiles are consumed by the pair's last MMAs: wait for their
+      // completion (which also means the loads have landed).
+      for (uint32_t i = issued > (uint32_t)C::SB ? issued - C::SB : 0; i < issued; ++i)
+        mbar_wait(mma_done + 8 * (i % C::SB), (i / C::SB) & 1);
+    }
+  } else if (warp == kPairMmaWarp) {
+    // ================= MMA issuer (first CTA) =================
+    if (rank == 0 && lane == 0) {
+      for (int g = 0; g < ngroups; ++g) {
+        const int db = g & 1;
+        if (g >= 2) {
+          wait_cl(bar_dfree + 8 * db, ((g >> 1) - 1) & 1);  // both epilogues read pass g - 2
+          tc_fence_after();
+        }
+        const uint32_t idesc = idesc_f16_f32(256, pass_n(g));
+        const uint32_t dcol = tmem + db * C::D_COLS;
+        for (int st = 0; st < nst; ++st) {
+          const uint32_t ga = (uint32_t)(g * nst + st);
+          const uint32_t aslot = ga % C::SA, bslot = ga % C::SB;
+          if (!wait_cl(full_a + 8 * aslot, (ga / C::SA) & 1)) break;
+          if (!wait_cl(full_b + 8 * bslot, (ga / C::SB) & 1)) break;
+          tc_fence_after();
+          const uint32_t bbase = s_base + C::OFF_B + bslot * C::B_SLOT_BYTES;
+          const uint32_t abase = tmem_a + aslot * C::A_COLS;
+#pragma unroll
+          for (int s = 0; s < 4; ++s) {
+            const uint32_t acc = (st > 0 || s > 0) ? 1u : 0u;
+            tc_mma_pair_f16_ts(dcol, abase + s * 8, smem_desc_sw128(bbase + s * 32), idesc, acc);
+            if constexpr (MODE == kModeDown)
+              tc_mma_pair_f16_ts(dcol, abase + s * 8, smem_desc_sw128(bbase + C::B_PLANE_BYTES + s * 32), idesc, 1u);
+          }
+          tc_commit_pair(mma_done + 8 * bslot, 0x3);
+        }
+        tc_commit_pair(bar_done + 8 * db, 0x3);  // also after a timeout: nothing waits on MMAs in flight
+      }
+      // No MMA may still run when the tensor memory is freed.
+      mbar_wait(bar_done + 8 * ((ngroups - 1) & 1), ((ngroups - 1) >> 1) & 1);
+    }
+  } else if (warp < 8) {
+    // ================= decoders (both CTAs) =================
+    const int q = warp & 3, kh = warp >> 2;
+    const int L = 32 * q + lane;  // TMEM lane = A row
+    const int R = MODE == kModeGateUp ? ((L & 1) ? 64 + (L >> 1) : (L >> 1)) : L;  // row in the weight tile
+    const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+    const int swz = R & 7;
+    const uint32_t lead_full_a = mapa_shared(full_a, 0);
+    for (int g = 0; g < ngroups; ++g) {
+      for (int kt = 0; kt < ntile; ++kt) {
+        const uint32_t gw = (uint32_t)(g * ntile + kt);
+        const uint32_t wslot = gw % C::WS;
+        wait(full_w + 8 * wslot, (gw / C::WS) & 1);
+        const uint8_t* wtile = smem + C::OFF_W + wslot * kPairWSlot;
+        const uint8_t* nrow = wtile + R * 128;
+        const uint4 sc4 = *reinterpret_cast<const uint4*>(wtile + kPairWNib + R * 16);
+        const uint32_t scw[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t ga = gw * 4 + j;
+          const uint32_t aslot = ga % C::SA;
+          // k 64 j + 32 kh .. + 31 of this row: one 16-byte chunk, two block scales.
+          const uint4 qv = *reinterpret_cast<const uint4*>(nrow + (((2 * j + kh) ^ swz) << 4));
+          uint32_t sclo, schi;  // f16x2 of scale bytes (4 j, 4 j + 1) and (4 j + 2, 4 j + 3)
+          e4m3x4_to_f16x2x2(scw[j], sclo, schi);
+          const uint32_t sc = kh ? schi : sclo;  // (first 16 k, second 16 k) of this half
+          const uint32_t wv[4] = {qv.x, qv.y, qv.z, qv.w};
+          uint32_t v[16];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t scl = i < 2 ? bcast_lo(sc) : bcast_hi(sc);
+            uint32_t dec[4];
+            e2m1x8_to_f16x2x4(wv[i], dec);
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) v[i * 4 + jj] = hmul2_u32(dec[jj], scl);
+          }
+          if (j == 3) {  // the weight tile is consumed
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty_w + 8 * wslot);
+          }
+          if (ga >= (uint32_t)C::SA) wait_mma(ga - C::SA);  // the A slot's previous MMAs are done
+          tc_fence_after();
+          tmem_st16(tmem_a + lane_off + aslot * C::A_COLS + 16 * kh, v);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(lead_full_a + 8 * aslot);
+        }
+      }
+    }
+  } else if (warp >= kPairEpiWarp0) {
+    // ================= epilogue (both CTAs) =================
+    const int q = warp & 3;
+    const int L = 32 * q + lane;
+    const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+    const float s2a = a.s2_0[e];
+    const float s2b = a.s2_1[e];
+    const uint32_t lead_dfree = mapa_shared(bar_dfree, 0);
+    // Output n of this lane: gate+up pairs lanes (2j: gate, 2j + 1: up of n_cta + j).
+    const int n = MODE == kModeGateUp ? n_cta + (L >> 1) : n_cta + L;
+    const int odd = lane & 1;
+    for (int g = 0; g < ngroups; ++g) {
+      const int db = g & 1;
+      const int g0 = row_lo + g * kPairNT;
+      const int nrows = min(kPairNT, row_hi - g0);
+      bool ok = wait(bar_done + 8 * db, (g >> 1) & 1);
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+      const uint32_t dcol = tmem + lane_off + db * C::D_COLS;
+#pragma unroll 1
+      for (int c0 = 0; c0 < nrows; c0 += 32) {
+        // lane l holds the activation-row scale of token c0 + l
+        const float xm_l = (c0 + lane < nrows) ? a.bexp[g0 + c0 + lane] : 0.0f;
+#pragma unroll 1
+        for (int tt = 0; tt < 32 && c0 + tt < nrows; tt += 8) {
+          uint32_t d[8];
+          tmem_ld8(dcol + c0 + tt, d);
+          tmem_wait_ld();
+          if constexpr (MODE == kModeGateUp) {
+#pragma unroll
+            for (int j = 0; j < 8; j += 2) {
+              // Even lane: gate of tokens t, t + 1; odd lane: up of the same.
+              // After the swap the even lane holds (g, u) of token t, the odd
+              // lane (g, u) of token t + 1.
+              const float mine0 = __uint_as_float(d[j]), mine1 = __uint_as_float(d[j + 1]);
+              const float other = __shfl_xor_sync(0xffffffffu, odd ? mine0 : mine1, 1);
+              const float gv = odd ? other : mine0;
+              const float uv = odd ? mine1 : other;
+              const int tl = tt + j + odd;
+              const float xm = __shfl_sync(0xffffffffu, xm_l, tl);
+              const int t = c0 + tl;
+              if (ok && t < nrows) a.out[(size_t)(g0 + t) * N + n] = silu_f32(gv * xm * s2a) * (uv * xm * s2b);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float xm = __shfl_sync(0xffffffffu, xm_l, tt + j);
+              const int t = c0 + tt + j;
+              float v = __uint_as_float(d[j]) * xm * s2a;
+              if constexpr (MODE == kModeUpAct) v = activation_f32(a.activation, v);
+              if (ok && t < nrows) a.out[(size_t)(g0 + t) * N + n] = v;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(lead_dfree + 8 * db);
+    }
+  }
+
+  __syncthreads();
+  __syncwarp();
+  cluster_sync();  // no more remote arrives, and the pair's MMAs are done
+  if (warp == kPairMmaWarp) {
+    __syncwarp();
+    tmem_dealloc_pair(tmem, C::TMEM_COLS);
+  }
+}
+
+namespace {
+
+template <int MODE>
+cudaError_t launch_tc_pair_impl(const TcArgs& a, const CUtensorMap& b0, const CUtensorMap& b1, uint32_t cap,
+                                cudaStream_t stream) {
+  using C = PairCfg<MODE>;
+  auto kern = grouped_tc_pair_kernel<MODE>;
+  cudaError_t err = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::SMEM);
+  if (err != cudaSuccess) return err;
+  const dim3 grid(2 * (a.N / C::ROWS_PER_PAIR), cap);
+  return launch_pdl(kern, grid, dim3(kPairThreads), C::SMEM, stream, a, b0, b1);
+}
+
+}  // namespace

@@ -17,13 +17,14 @@ enum { kActRelu2 = 1, kActSilu = 2 };
 constexpr uint32_t kMaxExperts = 1024;
 constexpr uint64_t kMaxPairs = 1ull << 24;
 
-// Token rows per pass of the tcgen05 kernel: 16 for decode-shaped batches (a
-// few rows per expert), 128 when experts carry many rows.  `tiles` > 0 (a
-// launch option) forces tiles * 8.
+// Token rows per pass of the tcgen05 kernels: 16 for decode-shaped batches (a
+// few rows per expert, one-CTA kernel); 192 when experts carry many rows (the
+// CTA-pair kernel).  `tiles` > 0 (a launch option) forces tiles * 8: 2 -> 16,
+// 16 -> 128 (one-CTA kernel), 24 -> 192 (pair kernel).
 inline int plan_tc_rows(uint64_t pairs, uint32_t num_experts, int tiles) {
   if (tiles > 0) return tiles * 8;
   const uint64_t mean = (pairs + num_experts - 1) / num_experts;
-  return mean <= 16 ? 16 : 128;
+  return mean <= 16 ? 16 : 192;
 }
 
 // Arguments of the grouped projection kernels.  Mode gate+up reads BF16 x

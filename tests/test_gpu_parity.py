@@ -287,8 +287,9 @@ def test_gate_up_four_tiles():
     _close(bufs.act.cpu().numpy()[:kept], ref["act"][:kept], "act")
 
 
-# tcgen05 path: token rows per pass 16 (tiles=2) or 128 (tiles=16); 0 = from the shape.
-@pytest.mark.parametrize("tiles", [0, 2, 16])
+# tcgen05 path: token rows per pass 16 (tiles=2) or 128 (tiles=16) on the one-CTA
+# kernel, 192 (tiles=24) on the CTA-pair kernel; 0 = from the shape.
+@pytest.mark.parametrize("tiles", [0, 2, 16, 24])
 @pytest.mark.parametrize("name", list(SMALL))
 def test_forward_small_tcgen05(name, tiles):
     _need_gpu()
@@ -297,10 +298,27 @@ def test_forward_small_tcgen05(name, tiles):
     _check_full(prob, bufs)
 
 
-def test_null_experts_tcgen05():
+@pytest.mark.parametrize("tiles", [0, 24])
+def test_null_experts_tcgen05(tiles):
     _need_gpu()
     prob = make_problem(SMALL["ragged"], null_experts=[1, 3])
-    _, bufs = _gpu_forward(prob, ws=True, path=2)
+    _, bufs = _gpu_forward(prob, ws=True, path=2, tiles=tiles)
+    _check_full(prob, bufs)
+
+
+# Experts of 1 .. 400 rows on the pair kernel: every pass length 32 .. 192 and
+# several passes per expert, two column blocks of gate+up (I = 256).
+PAIR_CFG = MoEConfig("pairrows", hidden=512, inter=256, experts=12, topk=3, tokens=400,
+                     router="zipf", seed=25)
+
+
+@pytest.mark.parametrize("tiles", [24, 16])
+def test_forward_pair_kernel_pass_lengths(tiles):
+    _need_gpu()
+    prob = make_problem(PAIR_CFG)
+    counts = np.bincount(prob.topk_ids.reshape(-1), minlength=PAIR_CFG.experts)
+    assert counts.max() > 192 and counts[counts > 0].min() < 32
+    _, bufs = _gpu_forward(prob, ws=True, path=2, tiles=tiles)
     _check_full(prob, bufs)
 
 
@@ -616,7 +634,8 @@ def _gpu_forward_nongated(prob, activation, ws=False, null=(), **opts):
 
 # (path options): decode kernel automatic and forced shapes; tcgen05 16- and 128-row passes.
 NONGATED_PATHS = [dict(), dict(path=1, split=4, tiles=1, depth=2), dict(path=1, split=1, tiles=2, depth=3),
-                  dict(ws=True, path=2, tiles=2), dict(ws=True, path=2, tiles=16)]
+                  dict(ws=True, path=2, tiles=2), dict(ws=True, path=2, tiles=16),
+                  dict(ws=True, path=2, tiles=24)]
 
 
 @pytest.mark.parametrize("opts", NONGATED_PATHS, ids=lambda o: "-".join(f"{k}{v}" for k, v in o.items()) or "auto")
