@@ -19,13 +19,14 @@
 // consecutive rows n0 + 128 r .. + 127 of the one matrix.
 //
 // Roles (15 warps per CTA), synchronised by mbarriers only:
-//   warps 0-7   decoders: TMEM lane 32 (w % 4) + l, k half w / 4 of each
-//               64-k stage; 16 nibble bytes and 2 scales per stage from the
-//               weight tile in shared memory, exact E2M1 x E4M3 -> f16,
-//               tcgen05.st into a 4-stage A ring; each warp then arrives on the
-//               first CTA's full_a barrier (the peer's warps remotely);
-//   warp 8      first CTA: MMA issuer (one thread): waits for both CTAs' A
-//               stage and token tile, issues the pair MMAs into one of two D
+//   warps 0-7   decoders: TMEM lane 32 (w % 4) + l, the 64-k stages of parity
+//               w / 4; 32 nibble bytes and 4 scales per stage from the weight
+//               tile in shared memory, exact E2M1 x E4M3 -> f16, tcgen05.st
+//               into the A ring; each warp then arrives on the first CTA's
+//               full_a barrier (the peer's warps remotely);
+//   warp 8      first CTA: MMA issuer (one thread): waits for the stage's
+//               full_a barrier (both CTAs' A stage; one decoder lane folds in
+//               the token tile's arrival), issues the pair MMAs into one of two D
 //               buffers, commits each stage and each pass to barriers in both
 //               CTAs (multicast commit);
 //   warp 9      weight tiles by TMA (its CTA's 128 rows, 256 k per tile);
@@ -41,7 +42,7 @@
 
 namespace {
 
-constexpr int kPairNT = 192;                // token rows per pass of the pair (MMA N, max)
+constexpr int kPairNT = kTcPairRows;        // token rows per pass of the pair (MMA N, max)
 constexpr int kPairHalf = kPairNT / 2;      // token rows each CTA loads
 constexpr int kPairMmaWarp = 8;
 constexpr int kPairWLoadWarp = 9;
@@ -60,19 +61,23 @@ struct PairCfg {
   static constexpr int B_SLOT_BYTES = PLANES * B_PLANE_BYTES;
   static constexpr int A_COLS = 32;                                   // TMEM columns per A stage
   static constexpr int D_COLS = kPairNT;                              // per D buffer
-  static constexpr int SA = 4;
-  static constexpr int WS = 2;
+  static constexpr int ND = 2;                                        // D buffers
+  static constexpr int WS = 3;
   static constexpr int SB = MODE == kModeDown ? 4 : 8;
+  // A ring: the rest of tensor memory, at most SB stages (the completion ring
+  // of SB entries also tells the decoders when an A slot is free).
+  static constexpr int SA_TMEM = (512 - ND * D_COLS) / A_COLS;
+  static constexpr int SA = SA_TMEM < SB ? SA_TMEM : SB;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int OFF_W = 0;
   static constexpr int OFF_B = WS * kPairWSlot;
   static constexpr int OFF_BAR = OFF_B + SB * B_SLOT_BYTES;
-  // full_w[WS], empty_w[WS], full_b[SB], mma_done[SB], full_a[SA], done[2], dfree[2]
-  static constexpr int NBAR = 2 * WS + 2 * SB + SA + 4;
+  // full_w[WS], empty_w[WS], full_b[SB], mma_done[SB], full_a[SA], done[ND], dfree[ND]
+  static constexpr int NBAR = 2 * WS + 2 * SB + SA + 2 * ND;
   static constexpr int OFF_TMEM = OFF_BAR + 8 * NBAR;
   static constexpr int OFF_ABORT = OFF_TMEM + 16;
   static constexpr int SMEM = OFF_ABORT + 16 + 1024;
-  static_assert(2 * D_COLS + SA * A_COLS <= (int)TMEM_COLS, "TMEM budget");
+  static_assert(ND * D_COLS + SA * A_COLS <= (int)TMEM_COLS && SA >= 2, "TMEM budget");
   static_assert(B_PLANE_BYTES % 1024 == 0 && kPairWSlot % 1024 == 0, "TMA tiles stay 1024-byte aligned");
   static_assert(SB >= SA, "mma_done also tracks the A ring");
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
@@ -94,8 +99,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   const uint32_t full_b = empty_w + 8 * C::WS;   // used in the first CTA
   const uint32_t mma_done = full_b + 8 * C::SB;  // both CTAs (multicast commit)
   const uint32_t full_a = mma_done + 8 * C::SB;  // used in the first CTA
-  const uint32_t bar_done = full_a + 8 * C::SA;  // [2], both CTAs (multicast commit)
-  const uint32_t bar_dfree = bar_done + 16;      // [2], used in the first CTA
+  const uint32_t bar_done = full_a + 8 * C::SA;  // [ND], both CTAs (multicast commit)
+  const uint32_t bar_dfree = bar_done + 8 * C::ND;  // [ND], used in the first CTA
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_ABORT);
 
@@ -133,8 +138,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       mbar_init(full_b + 8 * s, 1);
       mbar_init(mma_done + 8 * s, 1);
     }
-    for (int s = 0; s < C::SA; ++s) mbar_init(full_a + 8 * s, 16);  // 8 decoder warps per CTA
-    for (int d = 0; d < 2; ++d) {
+    for (int s = 0; s < C::SA; ++s) mbar_init(full_a + 8 * s, 8);  // 4 decoder warps per stage per CTA
+    for (int d = 0; d < C::ND; ++d) {
       mbar_init(bar_done + 8 * d, 1);
       mbar_init(bar_dfree + 8 * d, 8);  // 4 epilogue warps per CTA
     }
@@ -150,17 +155,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   cluster_sync();  // the first CTA's barriers exist before any remote arrive or TMA signal
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t tmem_a = tmem + 2 * C::D_COLS;  // A ring after the two D buffers
+  const uint32_t tmem_a = tmem + C::ND * C::D_COLS;  // A ring after the D buffers
 
   auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+    if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if (mbar_wait(bar, parity)) return true;
-    *abort_flag = 1;
-    return false;
-  };
-  auto wait_cl = [&](uint32_t bar, uint32_t parity) -> bool {
-    if (*abort_flag) return false;
-    if (mbar_wait_cluster(bar, parity)) return true;
     *abort_flag = 1;
     return false;
   };
@@ -228,17 +228,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         }
       }
       // The last tiles are consumed by the pair's last MMAs: wait for their
-      // completion (which also means the loads have landed).
-      for (uint32_t i = issued > (uint32_t)C::SB ? issued - C::SB : 0; i < issued; ++i)
+      // completion.  The first CTA also waits for its full_b phases, which
+      // count both CTAs' bytes, so no TMA of either CTA still targets its
+      // barriers or the peer's shared memory when the pair exits.
+      for (uint32_t i = issued > (uint32_t)C::SB ? issued - C::SB : 0; i < issued; ++i) {
         mbar_wait(mma_done + 8 * (i % C::SB), (i / C::SB) & 1);
+        if (rank == 0) mbar_wait(full_b + 8 * (i % C::SB), (i / C::SB) & 1);
+      }
     }
   } else if (warp == kPairMmaWarp) {
     // ================= MMA issuer (first CTA) =================
     if (rank == 0 && lane == 0) {
       for (int g = 0; g < ngroups; ++g) {
-        const int db = g & 1;
-        if (g >= 2) {
-          wait_cl(bar_dfree + 8 * db, ((g >> 1) - 1) & 1);  // both epilogues read pass g - 2
+        const int db = g % C::ND;
+        if (g >= C::ND) {
+          wait(bar_dfree + 8 * db, (g / C::ND - 1) & 1);  // both epilogues read pass g - ND
           tc_fence_after();
         }
         const uint32_t idesc = idesc_f16_f32(256, pass_n(g));
@@ -246,8 +250,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         for (int st = 0; st < nst; ++st) {
           const uint32_t ga = (uint32_t)(g * nst + st);
           const uint32_t aslot = ga % C::SA, bslot = ga % C::SB;
-          if (!wait_cl(full_a + 8 * aslot, (ga / C::SA) & 1)) break;
-          if (!wait_cl(full_b + 8 * bslot, (ga / C::SB) & 1)) break;
+          // full_a completes only after the stage's token tile has landed too
+          // (one decoder lane of this CTA waits for it before arriving).
+          if (!wait(full_a + 8 * aslot, (ga / C::SA) & 1)) break;
           tc_fence_after();
           const uint32_t bbase = s_base + C::OFF_B + bslot * C::B_SLOT_BYTES;
           const uint32_t abase = tmem_a + aslot * C::A_COLS;
@@ -263,11 +268,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         tc_commit_pair(bar_done + 8 * db, 0x3);  // also after a timeout: nothing waits on MMAs in flight
       }
       // No MMA may still run when the tensor memory is freed.
-      mbar_wait(bar_done + 8 * ((ngroups - 1) & 1), ((ngroups - 1) >> 1) & 1);
+      mbar_wait(bar_done + 8 * ((ngroups - 1) % C::ND), ((ngroups - 1) / C::ND) & 1);
     }
   } else if (warp < 8) {
     // ================= decoders (both CTAs) =================
-    const int q = warp & 3, kh = warp >> 2;
+    // Warp w decodes TMEM lanes 32 (w % 4) .. + 31 of the stages of parity
+    // w / 4, all 64 k of each: two warps per lane quarter alternate stages, so
+    // each has two stages of MMA time to decode, store and report one.
+    const int q = warp & 3, par = warp >> 2;
     const int L = 32 * q + lane;  // TMEM lane = A row
     const int R = MODE == kModeGateUp ? ((L & 1) ? 64 + (L >> 1) : (L >> 1)) : L;  // row in the weight tile
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
@@ -281,37 +289,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const uint8_t* wtile = smem + C::OFF_W + wslot * kPairWSlot;
         const uint8_t* nrow = wtile + R * 128;
         const uint4 sc4 = *reinterpret_cast<const uint4*>(wtile + kPairWNib + R * 16);
-        const uint32_t scw[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int jj = 0; jj < 2; ++jj) {
+          const int j = 2 * jj + par;  // stage j of the tile (ga has the parity of j)
           const uint32_t ga = gw * 4 + j;
           const uint32_t aslot = ga % C::SA;
-          // k 64 j + 32 kh .. + 31 of this row: one 16-byte chunk, two block scales.
-          const uint4 qv = *reinterpret_cast<const uint4*>(nrow + (((2 * j + kh) ^ swz) << 4));
+          // k 64 j .. + 63 of this row: 16-byte chunks 2 j and 2 j + 1 (swizzled), four block scales.
+          const uint4 q0 = *reinterpret_cast<const uint4*>(nrow + (((2 * j) ^ swz) << 4));
+          const uint4 q1 = *reinterpret_cast<const uint4*>(nrow + (((2 * j + 1) ^ swz) << 4));
           uint32_t sclo, schi;  // f16x2 of scale bytes (4 j, 4 j + 1) and (4 j + 2, 4 j + 3)
-          e4m3x4_to_f16x2x2(scw[j], sclo, schi);
-          const uint32_t sc = kh ? schi : sclo;  // (first 16 k, second 16 k) of this half
-          const uint32_t wv[4] = {qv.x, qv.y, qv.z, qv.w};
-          uint32_t v[16];
+          e4m3x4_to_f16x2x2(par ? (jj ? sc4.w : sc4.y) : (jj ? sc4.z : sc4.x), sclo, schi);
+          uint32_t v[32];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t scl = i < 2 ? bcast_lo(sc) : bcast_hi(sc);
-            uint32_t dec[4];
-            e2m1x8_to_f16x2x4(wv[i], dec);
+          for (int h = 0; h < 2; ++h) {
+            const uint4 qv = h == 0 ? q0 : q1;
+            const uint32_t sc = h == 0 ? sclo : schi;
+            const uint32_t wv[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) v[i * 4 + jj] = hmul2_u32(dec[jj], scl);
+            for (int i = 0; i < 4; ++i) {
+              const uint32_t scl = i < 2 ? bcast_lo(sc) : bcast_hi(sc);
+              uint32_t dec[4];
+              e2m1x8_to_f16x2x4(wv[i], dec);
+#pragma unroll
+              for (int m = 0; m < 4; ++m) v[16 * h + i * 4 + m] = hmul2_u32(dec[m], scl);
+            }
           }
-          if (j == 3) {  // the weight tile is consumed
+          if (jj == 1) {  // this warp's last stage of the weight tile
             __syncwarp();
             if (lane == 0) mbar_arrive(empty_w + 8 * wslot);
           }
           if (ga >= (uint32_t)C::SA) wait_mma(ga - C::SA);  // the A slot's previous MMAs are done
           tc_fence_after();
-          tmem_st16(tmem_a + lane_off + aslot * C::A_COLS + 16 * kh, v);
+          tmem_st32(tmem_a + lane_off + aslot * C::A_COLS, v);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(lead_full_a + 8 * aslot);
+          if (lane == 0) {
+            // In the first CTA, warp 0 / 4 also reports the stage's token tile.
+            if (rank == 0 && q == 0) wait(full_b + 8 * (ga % C::SB), (ga / C::SB) & 1);
+            mbar_arrive_remote(lead_full_a + 8 * aslot);
+          }
         }
       }
     }
@@ -327,10 +344,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     const int n = MODE == kModeGateUp ? n_cta + (L >> 1) : n_cta + L;
     const int odd = lane & 1;
     for (int g = 0; g < ngroups; ++g) {
-      const int db = g & 1;
+      const int db = g % C::ND;
       const int g0 = row_lo + g * kPairNT;
       const int nrows = min(kPairNT, row_hi - g0);
-      bool ok = wait(bar_done + 8 * db, (g >> 1) & 1);
+      bool ok = wait(bar_done + 8 * db, (g / C::ND) & 1);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
       const uint32_t dcol = tmem + lane_off + db * C::D_COLS;
@@ -338,41 +355,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       for (int c0 = 0; c0 < nrows; c0 += 32) {
         // lane l holds the activation-row scale of token c0 + l
         const float xm_l = (c0 + lane < nrows) ? a.bexp[g0 + c0 + lane] : 0.0f;
-#pragma unroll 1
-        for (int tt = 0; tt < 32 && c0 + tt < nrows; tt += 8) {
-          uint32_t d[8];
-          tmem_ld8(dcol + c0 + tt, d);
-          tmem_wait_ld();
-          if constexpr (MODE == kModeGateUp) {
+        // 32 columns per wait (the D buffer holds 192 >= c0 + 32 columns).
+        uint32_t d[32];
 #pragma unroll
-            for (int j = 0; j < 8; j += 2) {
-              // Even lane: gate of tokens t, t + 1; odd lane: up of the same.
-              // After the swap the even lane holds (g, u) of token t, the odd
-              // lane (g, u) of token t + 1.
-              const float mine0 = __uint_as_float(d[j]), mine1 = __uint_as_float(d[j + 1]);
-              const float other = __shfl_xor_sync(0xffffffffu, odd ? mine0 : mine1, 1);
-              const float gv = odd ? other : mine0;
-              const float uv = odd ? mine1 : other;
-              const int tl = tt + j + odd;
-              const float xm = __shfl_sync(0xffffffffu, xm_l, tl);
-              const int t = c0 + tl;
-              if (ok && t < nrows) a.out[(size_t)(g0 + t) * N + n] = silu_f32(gv * xm * s2a) * (uv * xm * s2b);
-            }
-          } else {
+        for (int h = 0; h < 4; ++h) tmem_ld8(dcol + c0 + 8 * h, *reinterpret_cast<uint32_t(*)[8]>(d + 8 * h));
+        tmem_wait_ld();
+        if constexpr (MODE == kModeGateUp) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float xm = __shfl_sync(0xffffffffu, xm_l, tt + j);
-              const int t = c0 + tt + j;
-              float v = __uint_as_float(d[j]) * xm * s2a;
-              if constexpr (MODE == kModeUpAct) v = activation_f32(a.activation, v);
-              if (ok && t < nrows) a.out[(size_t)(g0 + t) * N + n] = v;
-            }
+          for (int j = 0; j < 32; j += 2) {
+            // Even lane: gate of tokens t, t + 1; odd lane: up of the same.
+            // After the swap the even lane holds (g, u) of token t, the odd
+            // lane (g, u) of token t + 1.
+            const float mine0 = __uint_as_float(d[j]), mine1 = __uint_as_float(d[j + 1]);
+            const float other = __shfl_xor_sync(0xffffffffu, odd ? mine0 : mine1, 1);
+            const float gv = odd ? other : mine0;
+            const float uv = odd ? mine1 : other;
+            const int tl = j + odd;
+            const float xm = __shfl_sync(0xffffffffu, xm_l, tl);
+            const int t = c0 + tl;
+            if (ok && t < nrows) a.out[(size_t)(g0 + t) * N + n] = silu_f32(gv * xm * s2a) * (uv * xm * s2b);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float xm = __shfl_sync(0xffffffffu, xm_l, j);
+            const int t = c0 + j;
+            float v = __uint_as_float(d[j]) * xm * s2a;
+            if constexpr (MODE == kModeUpAct) v = activation_f32(a.activation, v);
+            if (ok && t < nrows) a.out[(size_t)(g0 + t) * N + n] = v;
           }
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(lead_dfree + 8 * db);
+      if (lane == 0) mbar_arrive_remote(lead_dfree + 8 * db);
     }
   }
 

@@ -204,10 +204,12 @@ NVM_DEV uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
   return r;
 }
-// Arrive (release at cluster scope) on an mbarrier given by its shared::cluster
-// address: this CTA's own or the peer's.
-NVM_DEV void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+// Arrive on an mbarrier given by its shared::cluster address: this CTA's own
+// or the peer's.  Release at CTA scope: what the arrival orders is tensor-memory
+// work (tcgen05.st before an MMA, tcgen05.ld before the accumulator is reused),
+// which the tcgen05 fences around the barrier carry.
+NVM_DEV void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 NVM_DEV bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
   uint32_t ok;
