@@ -24,11 +24,12 @@
 //               tile in shared memory, exact E2M1 x E4M3 -> f16, tcgen05.st
 //               into the A ring; each warp then arrives on the first CTA's
 //               full_a barrier (the peer's warps remotely);
-//   warp 8      first CTA: MMA issuer (one thread): waits for the stage's
-//               full_a barrier (both CTAs' A stage; one decoder lane folds in
-//               the token tile's arrival), issues the pair MMAs into one of two D
-//               buffers, commits each stage and each pass to barriers in both
-//               CTAs (multicast commit);
+//   warp 8      first CTA: MMA issuer (one thread): per two stages, waits
+//               for their full_a barriers (both CTAs' A stage; one decoder
+//               lane folds in the token tile's arrival), issues the pair MMAs
+//               into one of two D buffers and commits once; each pass ends
+//               with a commit too; commits reach barriers in both CTAs
+//               (multicast commit);
 //   warp 9      weight tiles by TMA (its CTA's 128 rows, 256 k per tile);
 //   warp 10     token tiles by TMA, its half of each 64-k stage, completion
 //               signalled on the first CTA's full_b barrier (pair TMA form);
@@ -79,7 +80,7 @@ struct PairCfg {
   static constexpr int SMEM = OFF_ABORT + 16 + 1024;
   static_assert(ND * D_COLS + SA * A_COLS <= (int)TMEM_COLS && SA >= 2, "TMEM budget");
   static_assert(B_PLANE_BYTES % 1024 == 0 && kPairWSlot % 1024 == 0, "TMA tiles stay 1024-byte aligned");
-  static_assert(SB >= SA, "mma_done also tracks the A ring");
+  static_assert(SB >= SA && SB % 2 == 0, "mma_done (odd entries, one commit per two stages) also tracks the A ring");
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
 
@@ -165,7 +166,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     return false;
   };
   // MMAs of stage x have completed (frees B slot x % SB and A slot x % SA).
-  auto wait_mma = [&](uint32_t x) -> bool { return wait(mma_done + 8 * (x % C::SB), (x / C::SB) & 1); };
+  // Stages are committed in pairs: the commit after odd stage x | 1 covers x.
+  auto wait_mma = [&](uint32_t x) -> bool {
+    x |= 1u;
+    return wait(mma_done + 8 * (x % C::SB), (x / C::SB) & 1);
+  };
   // Token rows of pass g: the MMA's N is its rows rounded up to 32; each CTA
   // loads N / 2 of them.
   auto pass_n = [&](int g) -> int {
@@ -232,7 +237,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       // count both CTAs' bytes, so no TMA of either CTA still targets its
       // barriers or the peer's shared memory when the pair exits.
       for (uint32_t i = issued > (uint32_t)C::SB ? issued - C::SB : 0; i < issued; ++i) {
-        mbar_wait(mma_done + 8 * (i % C::SB), (i / C::SB) & 1);
+        mbar_wait(mma_done + 8 * ((i | 1) % C::SB), ((i | 1) / C::SB) & 1);
         if (rank == 0) mbar_wait(full_b + 8 * (i % C::SB), (i / C::SB) & 1);
       }
     }
@@ -247,23 +252,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         }
         const uint32_t idesc = idesc_f16_f32(256, pass_n(g));
         const uint32_t dcol = tmem + db * C::D_COLS;
-        for (int st = 0; st < nst; ++st) {
+        // Two stages per step: both A stages (each completes only after its
+        // token tile has landed too: one decoder lane of this CTA waits for
+        // it before arriving), 8 (down: 16) MMAs, one commit, which frees
+        // both stages' token slots and A slots.
+        for (int st = 0; st < nst; st += 2) {
           const uint32_t ga = (uint32_t)(g * nst + st);
-          const uint32_t aslot = ga % C::SA, bslot = ga % C::SB;
-          // full_a completes only after the stage's token tile has landed too
-          // (one decoder lane of this CTA waits for it before arriving).
-          if (!wait(full_a + 8 * aslot, (ga / C::SA) & 1)) break;
+          if (!wait(full_a + 8 * (ga % C::SA), (ga / C::SA) & 1)) break;
+          if (!wait(full_a + 8 * ((ga + 1) % C::SA), ((ga + 1) / C::SA) & 1)) break;
           tc_fence_after();
-          const uint32_t bbase = s_base + C::OFF_B + bslot * C::B_SLOT_BYTES;
-          const uint32_t abase = tmem_a + aslot * C::A_COLS;
 #pragma unroll
-          for (int s = 0; s < 4; ++s) {
-            const uint32_t acc = (st > 0 || s > 0) ? 1u : 0u;
-            tc_mma_pair_f16_ts(dcol, abase + s * 8, smem_desc_sw128(bbase + s * 32), idesc, acc);
-            if constexpr (MODE == kModeDown)
-              tc_mma_pair_f16_ts(dcol, abase + s * 8, smem_desc_sw128(bbase + C::B_PLANE_BYTES + s * 32), idesc, 1u);
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t gx = ga + h;
+            const uint32_t bbase = s_base + C::OFF_B + (gx % C::SB) * C::B_SLOT_BYTES;
+            const uint32_t abase = tmem_a + (gx % C::SA) * C::A_COLS;
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+              const uint32_t acc = (st + h > 0 || s > 0) ? 1u : 0u;
+              tc_mma_pair_f16_ts(dcol, abase + s * 8, smem_desc_sw128(bbase + s * 32), idesc, acc);
+              if constexpr (MODE == kModeDown)
+                tc_mma_pair_f16_ts(dcol, abase + s * 8, smem_desc_sw128(bbase + C::B_PLANE_BYTES + s * 32), idesc, 1u);
+            }
           }
-          tc_commit_pair(mma_done + 8 * bslot, 0x3);
+          tc_commit_pair(mma_done + 8 * ((ga + 1) % C::SB), 0x3);
         }
         tc_commit_pair(bar_done + 8 * db, 0x3);  // also after a timeout: nothing waits on MMAs in flight
       }
