@@ -52,7 +52,7 @@ DEFAULT_STEPS = {"tiny": 4000, "decode_m1": 4000, "decode_m32": 2000, "decode_m2
 # Sources of each projection kernel; their hash names the build an ncu capture
 # was taken from.
 KERNEL_SOURCES = {
-    "tcgen05": ["grouped_tc.cu", "tc_common.cuh", "common.cuh"],
+    "tcgen05": ["grouped_tc.cu", "grouped_tc_pair.cuh", "tc_common.cuh", "common.cuh"],
     "mma.sync": ["grouped_mma.cu", "common.cuh"],
 }
 
@@ -384,9 +384,10 @@ def run_ours(args, rank, world, local):
     gu_ms = ev0.elapsed_time(ev1) / (reps * len(layers))
     gu_bytes = 2 * (active + (1 if args.shared else 0)) * per_expert
     gu_flops = 2.0 * 2 * pairs_run * cfg.hidden * cfg.inter
+    rows = _tc_rows(args, pairs_run, experts_run) if tc else 0
     if prefill:
         achieved = gu_flops / (gu_ms * 1e-3) / 1e12
-        roofline = {"kernel": "nvfp4_moe_gate_up_silu_ws (tcgen05, 128-row passes)", "bound": "tensor",
+        roofline = {"kernel": f"nvfp4_moe_gate_up_silu_ws ({_tc_kernel_name(rows)})", "bound": "tensor",
                     "achieved": achieved, "peak": tflops, "unit": "TFLOP/s",
                     "frac": achieved / tflops, "peak_source": f"{peak_kind} bf16 burst",
                     "algorithmic_flops_per_launch": gu_flops, "launch_ms": gu_ms,
@@ -394,7 +395,7 @@ def run_ours(args, rank, world, local):
                     "traffic_source_hash": kernel_source_hash("tcgen05")}
     else:
         achieved = gu_bytes / (gu_ms * 1e-3) / 1e9
-        roofline = {"kernel": "nvfp4_moe_gate_up_silu_ws (tcgen05, 16-row passes)" if tc else
+        roofline = {"kernel": f"nvfp4_moe_gate_up_silu_ws ({_tc_kernel_name(rows)})" if tc else
                     "nvfp4_moe_gate_up_silu (register-fed mma.sync)", "bound": "hbm",
                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                     "peak_source": f"{peak_kind} HBM copy", "algorithmic_bytes_per_launch": gu_bytes,
@@ -417,7 +418,8 @@ def run_ours(args, rank, world, local):
                    "router": cfg.router, "active_experts": active,
                    "shared_expert": ({"rows_per_table_entry": base.rows_per_shared_slot(cfg.tokens),
                                       "table_entries": slots} if args.shared else None),
-                   "path": ("tcgen05-nt128" if prefill else "tcgen05-nt16") if tc else "mma.sync",
+                   "path": (f"tcgen05-pair-nt{rows}" if rows in (32, 192) else f"tcgen05-nt{rows}")
+                           if tc else "mma.sync",
                    "weight_replicas": len(layers),
                    "l2": f"weights rotate over {len(layers)} device replicas; "
                          f"{len(layers)} x {routed_bytes/1e6:.1f} MB routed >= 4 x L2 ({l2/1e6:.0f} MB)"
@@ -459,10 +461,21 @@ def _tc_path(args, cfg, pairs, experts):
 
 
 def _uses_prefill(args, pairs, experts):
-    """Many rows per expert: the tcgen05 kernel runs 128-row passes and is tensor-bound."""
-    if args.tiles:
-        return args.tiles * 8 > 16
+    """Many rows per expert: a dense contraction, tensor-bound (else HBM-bound)."""
     return (pairs + experts - 1) // experts > 16
+
+
+def _tc_rows(args, pairs, experts):
+    """Token rows per pass of the tcgen05 kernels (the library's rule): 16 / 128 on
+    the one-CTA kernel, 32 / 192 on the CTA-pair kernel."""
+    if args.tiles:
+        return args.tiles * 8
+    return 16 if (pairs + experts - 1) // experts <= 16 else 192
+
+
+def _tc_kernel_name(rows):
+    return (f"tcgen05 CTA pair, {rows}-row passes" if rows in (32, 192)
+            else f"tcgen05 one CTA, {rows}-row passes")
 
 
 def run_e2e(layers, prob, bufs, ws, dev, stream, steps, warmup, args, world):

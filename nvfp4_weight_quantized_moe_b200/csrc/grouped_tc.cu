@@ -776,10 +776,12 @@ cudaError_t launch_tc(int mode, int nt, const GroupedArgs& g, void* workspace, u
                       uint32_t hidden, uint32_t inter, uint32_t cap, cudaStream_t stream) {
   const uint64_t pairs = (uint64_t)tokens * g.topk;
   const WsLayout w = ws_layout(workspace, pairs, hidden, inter);
-  if (g.num_experts == 0 || g.num_experts > kMaxExperts || (nt != 16 && nt != 128 && nt != kPairNT))
+  if (g.num_experts == 0 || g.num_experts > kMaxExperts ||
+      (nt != 16 && nt != 128 && nt != kTcPairRows && nt != kTcPairRowsSmall))
     return cudaErrorInvalidValue;
-  // 192-row passes run the pair kernel: 64-row weight boxes, 96-row token boxes.
-  const bool pair = nt == kPairNT;
+  // Pair passes (192 or 32 rows) run the CTA-pair kernel: 64-row weight boxes,
+  // token boxes of half a pass.
+  const bool pair = nt == kTcPairRows || nt == kTcPairRowsSmall;
   TcArgs a{};
   a.packed0 = g.packed0;
   a.packed1 = g.packed1 != nullptr ? g.packed1 : g.packed0;
@@ -804,7 +806,7 @@ cudaError_t launch_tc(int mode, int nt, const GroupedArgs& g, void* workspace, u
   err = make_map_2d(&t_scale, workspace, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.N, g.K / 16, w_rows, kTileK / 16,
                     CU_TENSOR_MAP_SWIZZLE_NONE);
   if (err != cudaSuccess) return err;
-  const uint32_t box_rows = pair ? (uint32_t)kPairHalf : (uint32_t)nt;
+  const uint32_t box_rows = pair ? (uint32_t)nt / 2 : (uint32_t)nt;
 
   if (mode == kModeGateUp) {
     err = launch_pdl(pack_x_sorted_kernel, dim3((unsigned)((pairs + 7) / 8)), dim3(256), 0, stream,
@@ -820,7 +822,8 @@ cudaError_t launch_tc(int mode, int nt, const GroupedArgs& g, void* workspace, u
     b1 = b0;
     a.bexp = w.xexp;
     a.wmaps = w.maps_gu;
-    if (pair) return launch_tc_pair_impl<kModeGateUp>(a, b0, b1, cap, stream);
+    if (nt == kTcPairRows) return launch_tc_pair_impl<kModeGateUp, kTcPairRows>(a, b0, b1, cap, stream);
+    if (nt == kTcPairRowsSmall) return launch_tc_pair_impl<kModeGateUp, kTcPairRowsSmall>(a, b0, b1, cap, stream);
     if (nt == 16) return launch_tc_impl<kModeGateUp, 16>(a, b0, b1, cap, stream);
     return launch_tc_impl<kModeGateUp, 128>(a, b0, b1, cap, stream);
   }
@@ -839,7 +842,8 @@ cudaError_t launch_tc(int mode, int nt, const GroupedArgs& g, void* workspace, u
     b1 = b0;
     a.bexp = w.xexp;
     a.wmaps = w.maps_gu;
-    if (pair) return launch_tc_pair_impl<kModeUpAct>(a, b0, b1, cap, stream);
+    if (nt == kTcPairRows) return launch_tc_pair_impl<kModeUpAct, kTcPairRows>(a, b0, b1, cap, stream);
+    if (nt == kTcPairRowsSmall) return launch_tc_pair_impl<kModeUpAct, kTcPairRowsSmall>(a, b0, b1, cap, stream);
     if (nt == 16) return launch_tc_impl<kModeUpAct, 16>(a, b0, b1, cap, stream);
     return launch_tc_impl<kModeUpAct, 128>(a, b0, b1, cap, stream);
   }
@@ -865,7 +869,8 @@ cudaError_t launch_tc(int mode, int nt, const GroupedArgs& g, void* workspace, u
   if (err != cudaSuccess) return err;
   a.bexp = w.aexp;
   a.wmaps = w.maps_down;
-  if (pair) return launch_tc_pair_impl<kModeDown>(a, b0, b1, cap, stream);
+  if (nt == kTcPairRows) return launch_tc_pair_impl<kModeDown, kTcPairRows>(a, b0, b1, cap, stream);
+  if (nt == kTcPairRowsSmall) return launch_tc_pair_impl<kModeDown, kTcPairRowsSmall>(a, b0, b1, cap, stream);
   if (nt == 16) return launch_tc_impl<kModeDown, 16>(a, b0, b1, cap, stream);
   return launch_tc_impl<kModeDown, 128>(a, b0, b1, cap, stream);
 }

@@ -5,8 +5,8 @@
 //
 // A cluster of two CTAs runs tcgen05.mma.cta_group::2: M = 256 weight rows
 // (128 per CTA, each decoded into its own CTA's tensor memory) times N = up to
-// 192 token rows (each CTA loads half of the token tile into its own shared
-// memory), FP32 accumulators in both CTAs' tensor memory (each CTA holds its
+// NT token rows (192, or 32 for decode-shaped batches; each CTA loads half of
+// the token tile into its own shared memory), FP32 accumulators in both CTAs' tensor memory (each CTA holds its
 // 128 rows x all N columns).  Per FLOP this halves the decode work and the
 // tensor-memory stores of the one-CTA kernel at 128-token passes and cuts its
 // shared-memory traffic by a third, which is what bounded that kernel's MMA
@@ -43,8 +43,6 @@
 
 namespace {
 
-constexpr int kPairNT = kTcPairRows;        // token rows per pass of the pair (MMA N, max)
-constexpr int kPairHalf = kPairNT / 2;      // token rows each CTA loads
 constexpr int kPairMmaWarp = 8;
 constexpr int kPairWLoadWarp = 9;
 constexpr int kPairBLoadWarp = 10;
@@ -54,22 +52,27 @@ constexpr int kPairWBoxRows = 64;           // rows per weight TMA box
 constexpr int kPairWNib = 128 * 128;        // nibble bytes of a CTA's weight tile (128 rows x 256 k)
 constexpr int kPairWSlot = kPairWNib + 128 * 16;
 
-template <int MODE>
+// NT: token rows per pass of the pair (the MMA's N at most): 192 for experts
+// with many rows (one pair per SM pair), 32 for decode-shaped batches (two
+// pairs per SM pair, each with its own MMA issuer and weight stream).
+template <int MODE, int NT>
 struct PairCfg {
+  static constexpr int HALF = NT / 2;                                 // token rows each CTA loads
+  static constexpr int CTAS_PER_SM = NT > 32 ? 1 : 2;
   static constexpr int PLANES = MODE == kModeDown ? 2 : 1;           // down: f16 hi + lo
   static constexpr int ROWS_PER_PAIR = MODE == kModeGateUp ? 128 : 256;  // outputs n per pair
-  static constexpr int B_PLANE_BYTES = kPairHalf * kStageK * 2;      // 96 rows x 64 k f16
+  static constexpr int B_PLANE_BYTES = HALF * kStageK * 2;           // HALF rows x 64 k f16
   static constexpr int B_SLOT_BYTES = PLANES * B_PLANE_BYTES;
   static constexpr int A_COLS = 32;                                   // TMEM columns per A stage
-  static constexpr int D_COLS = kPairNT;                              // per D buffer
+  static constexpr int D_COLS = NT;                                   // per D buffer
   static constexpr int ND = 2;                                        // D buffers
   static constexpr int WS = 3;
-  static constexpr int SB = MODE == kModeDown ? 4 : 8;
-  // A ring: the rest of tensor memory, at most SB stages (the completion ring
-  // of SB entries also tells the decoders when an A slot is free).
-  static constexpr int SA_TMEM = (512 - ND * D_COLS) / A_COLS;
+  static constexpr int SB = (MODE == kModeDown && NT > 32) ? 4 : 8;
+  static constexpr uint32_t TMEM_COLS = 512 / CTAS_PER_SM;
+  // A ring: the rest of the CTA's tensor memory, at most SB stages (the
+  // completion ring of SB entries also tells the decoders when an A slot is free).
+  static constexpr int SA_TMEM = ((int)TMEM_COLS - ND * D_COLS) / A_COLS;
   static constexpr int SA = SA_TMEM < SB ? SA_TMEM : SB;
-  static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int OFF_W = 0;
   static constexpr int OFF_B = WS * kPairWSlot;
   static constexpr int OFF_BAR = OFF_B + SB * B_SLOT_BYTES;
@@ -81,16 +84,17 @@ struct PairCfg {
   static_assert(ND * D_COLS + SA * A_COLS <= (int)TMEM_COLS && SA >= 2, "TMEM budget");
   static_assert(B_PLANE_BYTES % 1024 == 0 && kPairWSlot % 1024 == 0, "TMA tiles stay 1024-byte aligned");
   static_assert(SB >= SA && SB % 2 == 0, "mma_done (odd entries, one commit per two stages) also tracks the A ring");
-  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+  static_assert(CTAS_PER_SM * (SMEM + 1024) <= 228 * 1024, "shared memory per SM");
+  static_assert(NT % 32 == 0 && NT >= 32 && NT <= 256, "pair MMA with A in tensor memory: N a multiple of 32");
 };
 
 }  // namespace
 
-template <int MODE>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
+template <int MODE, int NT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, NT > 32 ? 1 : 2)
     grouped_tc_pair_kernel(const TcArgs a, const __grid_constant__ CUtensorMap tm_b0,
                            const __grid_constant__ CUtensorMap tm_b1) {
-  using C = PairCfg<MODE>;
+  using C = PairCfg<MODE, NT>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
   const uint32_t s_base = (raw_base + 1023u) & ~1023u;
@@ -124,7 +128,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       a.out[(size_t)(row_lo + i / W) * N + n_cta + i % W] = 0.0f;
     return;
   }
-  const int ngroups = (row_hi - row_lo + kPairNT - 1) / kPairNT;
+  const int ngroups = (row_hi - row_lo + NT - 1) / NT;
   if (ngroups <= 0) return;
   const int nst = K / kStageK;
   const int ntile = K / kTileK;
@@ -174,7 +178,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   // Token rows of pass g: the MMA's N is its rows rounded up to 32; each CTA
   // loads N / 2 of them.
   auto pass_n = [&](int g) -> int {
-    const int rows = min(kPairNT, row_hi - (row_lo + g * kPairNT));
+    const int rows = min(NT, row_hi - (row_lo + g * NT));
     return (rows + 31) & ~31;
   };
 
@@ -219,7 +223,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       uint32_t issued = 0;
       for (int g = 0; g < ngroups && !*abort_flag; ++g) {
         const int half = pass_n(g) / 2;
-        const int y = row_lo + g * kPairNT + (int)rank * half;
+        const int y = row_lo + g * NT + (int)rank * half;
         for (int st = 0; st < nst; ++st) {
           const uint32_t slot = issued % C::SB, round = issued / C::SB;
           if (round > 0 && !wait_mma(issued - C::SB)) break;
@@ -356,8 +360,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     const int odd = lane & 1;
     for (int g = 0; g < ngroups; ++g) {
       const int db = g % C::ND;
-      const int g0 = row_lo + g * kPairNT;
-      const int nrows = min(kPairNT, row_hi - g0);
+      const int g0 = row_lo + g * NT;
+      const int nrows = min(NT, row_hi - g0);
       bool ok = wait(bar_done + 8 * db, (g / C::ND) & 1);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
@@ -366,7 +370,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       for (int c0 = 0; c0 < nrows; c0 += 32) {
         // lane l holds the activation-row scale of token c0 + l
         const float xm_l = (c0 + lane < nrows) ? a.bexp[g0 + c0 + lane] : 0.0f;
-        // 32 columns per wait (the D buffer holds 192 >= c0 + 32 columns).
+        // 32 columns per wait (the D buffer holds NT >= c0 + 32 columns).
         uint32_t d[32];
 #pragma unroll
         for (int h = 0; h < 4; ++h) tmem_ld8(dcol + c0 + 8 * h, *reinterpret_cast<uint32_t(*)[8]>(d + 8 * h));
@@ -414,11 +418,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 
 namespace {
 
-template <int MODE>
+template <int MODE, int NT>
 cudaError_t launch_tc_pair_impl(const TcArgs& a, const CUtensorMap& b0, const CUtensorMap& b1, uint32_t cap,
                                 cudaStream_t stream) {
-  using C = PairCfg<MODE>;
-  auto kern = grouped_tc_pair_kernel<MODE>;
+  using C = PairCfg<MODE, NT>;
+  auto kern = grouped_tc_pair_kernel<MODE, NT>;
   cudaError_t err = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::SMEM);
   if (err != cudaSuccess) return err;
   const dim3 grid(2 * (a.N / C::ROWS_PER_PAIR), cap);

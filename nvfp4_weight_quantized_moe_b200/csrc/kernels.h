@@ -20,8 +20,9 @@ constexpr uint64_t kMaxPairs = 1ull << 24;
 // Token rows per pass of the tcgen05 kernels: 16 for decode-shaped batches (a
 // few rows per expert, one-CTA kernel); 192 when experts carry many rows (the
 // CTA-pair kernel).  `tiles` > 0 (a launch option) forces tiles * 8: 2 -> 16,
-// 16 -> 128 (one-CTA kernel), 24 -> 192 (pair kernel).
+// 16 -> 128 (one-CTA kernel), 4 -> 32 and 24 -> 192 (pair kernel).
 constexpr int kTcPairRows = 192;
+constexpr int kTcPairRowsSmall = 32;
 inline int plan_tc_rows(uint64_t pairs, uint32_t num_experts, int tiles) {
   if (tiles > 0) return tiles * 8;
   const uint64_t mean = (pairs + num_experts - 1) / num_experts;

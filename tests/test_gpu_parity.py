@@ -288,8 +288,8 @@ def test_gate_up_four_tiles():
 
 
 # tcgen05 path: token rows per pass 16 (tiles=2) or 128 (tiles=16) on the one-CTA
-# kernel, 192 (tiles=24) on the CTA-pair kernel; 0 = from the shape.
-@pytest.mark.parametrize("tiles", [0, 2, 16, 24])
+# kernel, 32 (tiles=4) or 192 (tiles=24) on the CTA-pair kernel; 0 = from the shape.
+@pytest.mark.parametrize("tiles", [0, 2, 4, 16, 24])
 @pytest.mark.parametrize("name", list(SMALL))
 def test_forward_small_tcgen05(name, tiles):
     _need_gpu()
@@ -312,7 +312,7 @@ PAIR_CFG = MoEConfig("pairrows", hidden=512, inter=256, experts=12, topk=3, toke
                      router="zipf", seed=25)
 
 
-@pytest.mark.parametrize("tiles", [24, 16])
+@pytest.mark.parametrize("tiles", [24, 16, 4])
 def test_forward_pair_kernel_pass_lengths(tiles):
     _need_gpu()
     prob = make_problem(PAIR_CFG)
@@ -452,13 +452,16 @@ def _check_against(ref, bufs, cfg):
     np.testing.assert_array_equal(ob, bufs.out.bfloat16().float().cpu().numpy())
 
 
-@pytest.mark.parametrize("ws", [False, True], ids=["decode-path", "tcgen05"])
+@pytest.mark.parametrize("ws,tiles", [(False, 0), (True, 0), (True, 4)],
+                         ids=["decode-path", "tcgen05", "tcgen05-pair32"])
 @pytest.mark.parametrize("name", ["decode_m256", "prefill_m8192"])
-def test_forward_full_size_every_element(name, ws):
+def test_forward_full_size_every_element(name, ws, tiles):
     """Full-size launch, every element of act, y and out against the oracle's full forward."""
     _need_gpu()
+    if tiles and name != "decode_m256":
+        pytest.skip("32-row pair passes are the decode-shaped launch")
     prob = make_problem(name)
-    _, bufs = _gpu_forward(prob, ws=ws)
+    _, bufs = _gpu_forward(prob, ws=ws, **(dict(path=2, tiles=tiles) if tiles else {}))
     _check_against(_full_ref(name), bufs, prob.cfg)
 
 
@@ -635,7 +638,7 @@ def _gpu_forward_nongated(prob, activation, ws=False, null=(), **opts):
 # (path options): decode kernel automatic and forced shapes; tcgen05 16- and 128-row passes.
 NONGATED_PATHS = [dict(), dict(path=1, split=4, tiles=1, depth=2), dict(path=1, split=1, tiles=2, depth=3),
                   dict(ws=True, path=2, tiles=2), dict(ws=True, path=2, tiles=16),
-                  dict(ws=True, path=2, tiles=24)]
+                  dict(ws=True, path=2, tiles=4), dict(ws=True, path=2, tiles=24)]
 
 
 @pytest.mark.parametrize("opts", NONGATED_PATHS, ids=lambda o: "-".join(f"{k}{v}" for k, v in o.items()) or "auto")
