@@ -384,7 +384,7 @@ def run_ours(args, rank, world, local):
     gu_ms = ev0.elapsed_time(ev1) / (reps * len(layers))
     gu_bytes = 2 * (active + (1 if args.shared else 0)) * per_expert
     gu_flops = 2.0 * 2 * pairs_run * cfg.hidden * cfg.inter
-    rows = _tc_rows(args, pairs_run, experts_run) if tc else 0
+    rows = _tc_rows(args, cfg.tokens, pairs_run, experts_run) if tc else 0
     if prefill:
         achieved = gu_flops / (gu_ms * 1e-3) / 1e12
         roofline = {"kernel": f"nvfp4_moe_gate_up_silu_ws ({_tc_kernel_name(rows)})", "bound": "tensor",
@@ -465,12 +465,15 @@ def _uses_prefill(args, pairs, experts):
     return (pairs + experts - 1) // experts > 16
 
 
-def _tc_rows(args, pairs, experts):
+def _tc_rows(args, tokens, pairs, experts):
     """Token rows per pass of the tcgen05 kernels (the library's rule): 16 / 128 on
     the one-CTA kernel, 32 / 192 on the CTA-pair kernel."""
     if args.tiles:
         return args.tiles * 8
-    return 16 if (pairs + experts - 1) // experts <= 16 else 192
+    mean = (pairs + experts - 1) // experts
+    if mean > 16:
+        return 192
+    return 32 if tokens > 16 and mean <= 4 else 16
 
 
 def _tc_kernel_name(rows):
