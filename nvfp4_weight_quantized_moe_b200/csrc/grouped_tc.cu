@@ -308,6 +308,7 @@ struct TcArgs {
   const int32_t* active_count;
   uint32_t N, K;
   int activation;             // up+activation: kActRelu2 or kActSilu
+  uint32_t cap;               // pair kernel: active slots it may read
 };
 
 // Registers: 128-token tiles run one CTA per SM, 16-token tiles two.  The

@@ -113,25 +113,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, NT > 3
   const uint32_t rank = cluster_ctarank();
   griddep_wait();
   griddep_launch_dependents();
-  // Both CTAs of a pair read the same slot and expert, so they take the same
-  // early exits and the same loop counts.
-  const int slot_idx = blockIdx.y;
-  if (slot_idx >= *a.active_count) return;
-  const int e = a.active_experts[slot_idx];
-  const int row_lo = a.offsets[e], row_hi = a.offsets[e + 1];
   const int N = (int)a.N, K = (int)a.K;
-  const int n_cta = (int)(blockIdx.x >> 1) * C::ROWS_PER_PAIR + (int)rank * (C::ROWS_PER_PAIR / 2);
-  if (a.packed0[e] == nullptr || (MODE == kModeGateUp && a.packed1[e] == nullptr)) {
-    // NULL expert: this CTA's outputs of its rows are zero.
-    constexpr int W = C::ROWS_PER_PAIR / 2;
-    for (int i = tid; i < (row_hi - row_lo) * W; i += kPairThreads)
-      a.out[(size_t)(row_lo + i / W) * N + n_cta + i % W] = 0.0f;
-    return;
-  }
-  const int ngroups = (row_hi - row_lo + NT - 1) / NT;
-  if (ngroups <= 0) return;
   const int nst = K / kStageK;
   const int ntile = K / kTileK;
+  // Tasks: (active slot, column block of ROWS_PER_PAIR outputs), taken by the
+  // pairs in turn.  Both CTAs of a pair, and every role, walk the same list.
+  const int ncb = N / C::ROWS_PER_PAIR;
+  const int active = min(*a.active_count, (int)a.cap);
+  const int ntask = active * ncb;
+  const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
+  struct Task {
+    int e, row_lo, row_hi, n_cta, ngroups;
+    bool null_expert;
+  };
+  auto task = [&](int t) {
+    Task k;
+    const int slot = t / ncb, cb = t - slot * ncb;
+    k.e = a.active_experts[slot];
+    k.row_lo = a.offsets[k.e];
+    k.row_hi = a.offsets[k.e + 1];
+    k.n_cta = cb * C::ROWS_PER_PAIR + (int)rank * (C::ROWS_PER_PAIR / 2);
+    k.null_expert = a.packed0[k.e] == nullptr || (MODE == kModeGateUp && a.packed1[k.e] == nullptr);
+    k.ngroups = k.null_expert ? 0 : (k.row_hi - k.row_lo + NT - 1) / NT;
+    return k;
+  };
+  // Token rows of pass g of a task: the MMA's N is its rows rounded up to 32;
+  // each CTA loads N / 2 of them.
+  auto pass_n = [&](const Task& k, int g) -> int {
+    const int rows = min(NT, k.row_hi - (k.row_lo + g * NT));
+    return (rows + 31) & ~31;
+  };
 
   // ---- set-up: barriers, tensor memory, then both CTAs meet ----
   if (tid == 0) {
@@ -175,42 +186,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, NT > 3
     x |= 1u;
     return wait(mma_done + 8 * (x % C::SB), (x / C::SB) & 1);
   };
-  // Token rows of pass g: the MMA's N is its rows rounded up to 32; each CTA
-  // loads N / 2 of them.
-  auto pass_n = [&](int g) -> int {
-    const int rows = min(NT, row_hi - (row_lo + g * NT));
-    return (rows + 31) & ~31;
-  };
 
   if (warp == kPairWLoadWarp) {
     // ================= weight tile loader (both CTAs) =================
     if (lane == 0) {
-      const CUtensorMap* m = a.wmaps + (size_t)e * kMapsPerExpert;
-      const CUtensorMap* nib0 = m;
-      const CUtensorMap* sc0 = m + 1;
-      const CUtensorMap* nib1 = MODE == kModeGateUp ? m + 2 : m;
-      const CUtensorMap* sc1 = MODE == kModeGateUp ? m + 3 : m + 1;
-      tmap_acquire(nib0);
-      tmap_acquire(sc0);
-      if (MODE == kModeGateUp) {
-        tmap_acquire(nib1);
-        tmap_acquire(sc1);
-      }
-      // Gate+up: 64 gate rows then the same 64 up rows; else 128 rows in two boxes.
-      const int y0 = n_cta, y1 = MODE == kModeGateUp ? n_cta : n_cta + kPairWBoxRows;
       uint32_t issued = 0;
-      for (int g = 0; g < ngroups && !*abort_flag; ++g) {
-        for (int kt = 0; kt < ntile; ++kt) {
-          const uint32_t slot = issued % C::WS, round = issued / C::WS;
-          if (round > 0 && !wait(empty_w + 8 * slot, (round - 1) & 1)) break;
-          const uint32_t dst = s_base + C::OFF_W + slot * kPairWSlot;
-          const uint32_t bar = full_w + 8 * slot;
-          mbar_arrive_expect_tx(bar, kPairWSlot);
-          tma_load_2d(dst, nib0, kt * (kTileK / 2), y0, bar);
-          tma_load_2d(dst + kPairWNib / 2, nib1, kt * (kTileK / 2), y1, bar);
-          tma_load_2d(dst + kPairWNib, sc0, kt * (kTileK / 16), y0, bar);
-          tma_load_2d(dst + kPairWNib + kPairWBoxRows * 16, sc1, kt * (kTileK / 16), y1, bar);
-          ++issued;
+      for (int t = pair; t < ntask && !*abort_flag; t += npairs) {
+        const Task k = task(t);
+        if (k.ngroups == 0) continue;
+        const CUtensorMap* m = a.wmaps + (size_t)k.e * kMapsPerExpert;
+        const CUtensorMap* nib0 = m;
+        const CUtensorMap* sc0 = m + 1;
+        const CUtensorMap* nib1 = MODE == kModeGateUp ? m + 2 : m;
+        const CUtensorMap* sc1 = MODE == kModeGateUp ? m + 3 : m + 1;
+        tmap_acquire(nib0);
+        tmap_acquire(sc0);
+        if (MODE == kModeGateUp) {
+          tmap_acquire(nib1);
+          tmap_acquire(sc1);
+        }
+        // Gate+up: 64 gate rows then the same 64 up rows; else 128 rows in two boxes.
+        const int y0 = k.n_cta, y1 = MODE == kModeGateUp ? k.n_cta : k.n_cta + kPairWBoxRows;
+        for (int g = 0; g < k.ngroups && !*abort_flag; ++g) {
+          for (int kt = 0; kt < ntile; ++kt) {
+            const uint32_t slot = issued % C::WS, round = issued / C::WS;
+            if (round > 0 && !wait(empty_w + 8 * slot, (round - 1) & 1)) break;
+            const uint32_t dst = s_base + C::OFF_W + slot * kPairWSlot;
+            const uint32_t bar = full_w + 8 * slot;
+            mbar_arrive_expect_tx(bar, kPairWSlot);
+            tma_load_2d(dst, nib0, kt * (kTileK / 2), y0, bar);
+            tma_load_2d(dst + kPairWNib / 2, nib1, kt * (kTileK / 2), y1, bar);
+            tma_load_2d(dst + kPairWNib, sc0, kt * (kTileK / 16), y0, bar);
+            tma_load_2d(dst + kPairWNib + kPairWBoxRows * 16, sc1, kt * (kTileK / 16), y1, bar);
+            ++issued;
+          }
         }
       }
       for (uint32_t i = issued > (uint32_t)C::WS ? issued - C::WS : 0; i < issued; ++i)
@@ -221,19 +230,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, NT > 3
     if (lane == 0) {
       const uint32_t lead_full_b = mapa_shared(full_b, 0);
       uint32_t issued = 0;
-      for (int g = 0; g < ngroups && !*abort_flag; ++g) {
-        const int half = pass_n(g) / 2;
-        const int y = row_lo + g * NT + (int)rank * half;
-        for (int st = 0; st < nst; ++st) {
-          const uint32_t slot = issued % C::SB, round = issued / C::SB;
-          if (round > 0 && !wait_mma(issued - C::SB)) break;
-          const uint32_t dst = s_base + C::OFF_B + slot * C::B_SLOT_BYTES;
-          // The first CTA's barrier counts both CTAs' bytes.
-          if (rank == 0) mbar_arrive_expect_tx(full_b + 8 * slot, 2 * C::B_SLOT_BYTES);
-          tma_load_2d_pair(dst, &tm_b0, st * kStageK, y, lead_full_b + 8 * slot);
-          if constexpr (MODE == kModeDown)
-            tma_load_2d_pair(dst + C::B_PLANE_BYTES, &tm_b1, st * kStageK, y, lead_full_b + 8 * slot);
-          ++issued;
+      for (int t = pair; t < ntask && !*abort_flag; t += npairs) {
+        const Task k = task(t);
+        for (int g = 0; g < k.ngroups && !*abort_flag; ++g) {
+          const int half = pass_n(k, g) / 2;
+          const int y = k.row_lo + g * NT + (int)rank * half;
+          for (int st = 0; st < nst; ++st) {
+            const uint32_t slot = issued % C::SB, round = issued / C::SB;
+            if (round > 0 && !wait_mma(issued - C::SB)) break;
+            const uint32_t dst = s_base + C::OFF_B + slot * C::B_SLOT_BYTES;
+            // The first CTA's barrier counts both CTAs' bytes.
+            if (rank == 0) mbar_arrive_expect_tx(full_b + 8 * slot, 2 * C::B_SLOT_BYTES);
+            tma_load_2d_pair(dst, &tm_b0, st * kStageK, y, lead_full_b + 8 * slot);
+            if constexpr (MODE == kModeDown)
+              tma_load_2d_pair(dst + C::B_PLANE_BYTES, &tm_b1, st * kStageK, y, lead_full_b + 8 * slot);
+            ++issued;
+          }
         }
       }
       // The last tiles are consumed by the pair's last MMAs: wait for their
@@ -248,42 +260,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, NT > 3
   } else if (warp == kPairMmaWarp) {
     // ================= MMA issuer (first CTA) =================
     if (rank == 0 && lane == 0) {
-      for (int g = 0; g < ngroups; ++g) {
-        const int db = g % C::ND;
-        if (g >= C::ND) {
-          wait(bar_dfree + 8 * db, (g / C::ND - 1) & 1);  // both epilogues read pass g - ND
-          tc_fence_after();
-        }
-        const uint32_t idesc = idesc_f16_f32(256, pass_n(g));
-        const uint32_t dcol = tmem + db * C::D_COLS;
-        // Two stages per step: both A stages (each completes only after its
-        // token tile has landed too: one decoder lane of this CTA waits for
-        // it before arriving), 8 (down: 16) MMAs, one commit, which frees
-        // both stages' token slots and A slots.
-        for (int st = 0; st < nst; st += 2) {
-          const uint32_t ga = (uint32_t)(g * nst + st);
-          if (!wait(full_a + 8 * (ga % C::SA), (ga / C::SA) & 1)) break;
-          if (!wait(full_a + 8 * ((ga + 1) % C::SA), ((ga + 1) / C::SA) & 1)) break;
-          tc_fence_after();
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t gx = ga + h;
-            const uint32_t bbase = s_base + C::OFF_B + (gx % C::SB) * C::B_SLOT_BYTES;
-            const uint32_t abase = tmem_a + (gx % C::SA) * C::A_COLS;
-#pragma unroll
-            for (int s = 0; s < 4; ++s) {
-              const uint32_t acc = (st + h > 0 || s > 0) ? 1u : 0u;
-              tc_mma_pair_f16_ts(dcol, abase + s * 8, smem_desc_sw128(bbase + s * 32), idesc, acc);
-              if constexpr (MODE == kModeDown)
-                tc_mma_pair_f16_ts(dcol, abase + s * 8, smem_desc_sw128(bbase + C::B_PLANE_BYTES + s * 32), idesc, 1u);
-            }
+      uint32_t gp = 0, gs = 0;  // passes and stages issued so far (over every task)
+      for (int t = pair; t < ntask; t += npairs) {
+        const Task k = task(t);
+        for (int g = 0; g < k.ngroups; ++g, ++gp, gs += nst) {
+          const uint32_t db = gp % C::ND;
+          if (gp >= (uint32_t)C::ND) {
+            wait(bar_dfree + 8 * db, (gp / C::ND - 1) & 1);  // both epilogues read pass gp - ND
+            tc_fence_after();
           }
-          tc_commit_pair(mma_done + 8 * ((ga + 1) % C::SB), 0x3);
+          const uint32_t idesc = idesc_f16_f32(256, pass_n(k, g));
+          const uint32_t dcol = tmem + db * C::D_COLS;
+          // Two stages per step: both A stages (each completes only after its
+          // token tile has landed too: one decoder lane of this CTA waits for
+          // it before arriving), 8 (down: 16) MMAs, one commit, which frees
+          // both stages' token slots and A slots.
+          for (int st = 0; st < nst; st += 2) {
+            const uint32_t ga = gs + st;
+            if (!wait(full_a + 8 * (ga % C::SA), (ga / C::SA) & 1)) break;
+            if (!wait(full_a + 8 * ((ga + 1) % C::SA), ((ga + 1) / C::SA) & 1)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint32_t gx = ga + h;
+              const uint32_t bbase = s_base + C::OFF_B + (gx % C::SB) * C::B_SLOT_BYTES;
+              const uint32_t abase = tmem_a + (gx % C::SA) * C::A_COLS;
+#pragma unroll
+              for (int s = 0; s < 4; ++s) {
+                const uint32_t acc = (st + h > 0 || s > 0) ? 1u : 0u;
+                tc_mma_pair_f16_ts(dcol, abase + s * 8, smem_desc_sw128(bbase + s * 32), idesc, acc);
+                if constexpr (MODE == kModeDown)
+                  tc_mma_pair_f16_ts(dcol, abase + s * 8, smem_desc_sw128(bbase + C::B_PLANE_BYTES + s * 32), idesc,
+                                     1u);
+              }
+            }
+            tc_commit_pair(mma_done + 8 * ((ga + 1) % C::SB), 0x3);
+          }
+          tc_commit_pair(bar_done + 8 * db, 0x3);  // also after a timeout: nothing waits on MMAs in flight
         }
-        tc_commit_pair(bar_done + 8 * db, 0x3);  // also after a timeout: nothing waits on MMAs in flight
       }
       // No MMA may still run when the tensor memory is freed.
-      mbar_wait(bar_done + 8 * ((ngroups - 1) % C::ND), ((ngroups - 1) / C::ND) & 1);
+      if (gp > 0) mbar_wait(bar_done + 8 * ((gp - 1) % C::ND), ((gp - 1) / C::ND) & 1);
     }
   } else if (warp < 8) {
     // ================= decoders (both CTAs) =================
@@ -296,53 +313,56 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, NT > 3
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
     const int swz = R & 7;
     const uint32_t lead_full_a = mapa_shared(full_a, 0);
-    for (int g = 0; g < ngroups; ++g) {
-      for (int kt = 0; kt < ntile; ++kt) {
-        const uint32_t gw = (uint32_t)(g * ntile + kt);
-        const uint32_t wslot = gw % C::WS;
-        wait(full_w + 8 * wslot, (gw / C::WS) & 1);
-        const uint8_t* wtile = smem + C::OFF_W + wslot * kPairWSlot;
-        const uint8_t* nrow = wtile + R * 128;
-        const uint4 sc4 = *reinterpret_cast<const uint4*>(wtile + kPairWNib + R * 16);
+    uint32_t gw = 0;  // weight tiles consumed so far (over every task)
+    for (int t = pair; t < ntask; t += npairs) {
+      const Task k = task(t);
+      for (int g = 0; g < k.ngroups; ++g) {
+        for (int kt = 0; kt < ntile; ++kt, ++gw) {
+          const uint32_t wslot = gw % C::WS;
+          wait(full_w + 8 * wslot, (gw / C::WS) & 1);
+          const uint8_t* wtile = smem + C::OFF_W + wslot * kPairWSlot;
+          const uint8_t* nrow = wtile + R * 128;
+          const uint4 sc4 = *reinterpret_cast<const uint4*>(wtile + kPairWNib + R * 16);
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-          const int j = 2 * jj + par;  // stage j of the tile (ga has the parity of j)
-          const uint32_t ga = gw * 4 + j;
-          const uint32_t aslot = ga % C::SA;
-          // k 64 j .. + 63 of this row: 16-byte chunks 2 j and 2 j + 1 (swizzled), four block scales.
-          const uint4 q0 = *reinterpret_cast<const uint4*>(nrow + (((2 * j) ^ swz) << 4));
-          const uint4 q1 = *reinterpret_cast<const uint4*>(nrow + (((2 * j + 1) ^ swz) << 4));
-          uint32_t sclo, schi;  // f16x2 of scale bytes (4 j, 4 j + 1) and (4 j + 2, 4 j + 3)
-          e4m3x4_to_f16x2x2(par ? (jj ? sc4.w : sc4.y) : (jj ? sc4.z : sc4.x), sclo, schi);
-          uint32_t v[32];
+          for (int jj = 0; jj < 2; ++jj) {
+            const int j = 2 * jj + par;  // stage j of the tile (ga has the parity of j)
+            const uint32_t ga = gw * 4 + j;
+            const uint32_t aslot = ga % C::SA;
+            // k 64 j .. + 63 of this row: 16-byte chunks 2 j and 2 j + 1 (swizzled), four block scales.
+            const uint4 q0 = *reinterpret_cast<const uint4*>(nrow + (((2 * j) ^ swz) << 4));
+            const uint4 q1 = *reinterpret_cast<const uint4*>(nrow + (((2 * j + 1) ^ swz) << 4));
+            uint32_t sclo, schi;  // f16x2 of scale bytes (4 j, 4 j + 1) and (4 j + 2, 4 j + 3)
+            e4m3x4_to_f16x2x2(par ? (jj ? sc4.w : sc4.y) : (jj ? sc4.z : sc4.x), sclo, schi);
+            uint32_t v[32];
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint4 qv = h == 0 ? q0 : q1;
-            const uint32_t sc = h == 0 ? sclo : schi;
-            const uint32_t wv[4] = {qv.x, qv.y, qv.z, qv.w};
+            for (int h = 0; h < 2; ++h) {
+              const uint4 qv = h == 0 ? q0 : q1;
+              const uint32_t sc = h == 0 ? sclo : schi;
+              const uint32_t wv[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const uint32_t scl = i < 2 ? bcast_lo(sc) : bcast_hi(sc);
-              uint32_t dec[4];
-              e2m1x8_to_f16x2x4(wv[i], dec);
+              for (int i = 0; i < 4; ++i) {
+                const uint32_t scl = i < 2 ? bcast_lo(sc) : bcast_hi(sc);
+                uint32_t dec[4];
+                e2m1x8_to_f16x2x4(wv[i], dec);
 #pragma unroll
-              for (int m = 0; m < 4; ++m) v[16 * h + i * 4 + m] = hmul2_u32(dec[m], scl);
+                for (int m = 0; m < 4; ++m) v[16 * h + i * 4 + m] = hmul2_u32(dec[m], scl);
+              }
             }
-          }
-          if (jj == 1) {  // this warp's last stage of the weight tile
+            if (jj == 1) {  // this warp's last stage of the weight tile
+              __syncwarp();
+              if (lane == 0) mbar_arrive(empty_w + 8 * wslot);
+            }
+            if (ga >= (uint32_t)C::SA) wait_mma(ga - C::SA);  // the A slot's previous MMAs are done
+            tc_fence_after();
+            tmem_st32(tmem_a + lane_off + aslot * C::A_COLS, v);
+            tmem_wait_st();
+            tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(empty_w + 8 * wslot);
-          }
-          if (ga >= (uint32_t)C::SA) wait_mma(ga - C::SA);  // the A slot's previous MMAs are done
-          tc_fence_after();
-          tmem_st32(tmem_a + lane_off + aslot * C::A_COLS, v);
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            // In the first CTA, warp 0 / 4 also reports the stage's token tile.
-            if (rank == 0 && q == 0) wait(full_b + 8 * (ga % C::SB), (ga / C::SB) & 1);
-            mbar_arrive_remote(lead_full_a + 8 * aslot);
+            if (lane == 0) {
+              // In the first CTA, warp 0 / 4 also reports the stage's token tile.
+              if (rank == 0 && q == 0) wait(full_b + 8 * (ga % C::SB), (ga / C::SB) & 1);
+              mbar_arrive_remote(lead_full_a + 8 * aslot);
+            }
           }
         }
       }
@@ -351,59 +371,71 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, NT > 3
     // ================= epilogue (both CTAs) =================
     const int q = warp & 3;
     const int L = 32 * q + lane;
+    const int et = tid - 32 * kPairEpiWarp0;  // 0 .. 127
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
-    const float s2a = a.s2_0[e];
-    const float s2b = a.s2_1[e];
     const uint32_t lead_dfree = mapa_shared(bar_dfree, 0);
-    // Output n of this lane: gate+up pairs lanes (2j: gate, 2j + 1: up of n_cta + j).
-    const int n = MODE == kModeGateUp ? n_cta + (L >> 1) : n_cta + L;
     const int odd = lane & 1;
-    for (int g = 0; g < ngroups; ++g) {
-      const int db = g % C::ND;
-      const int g0 = row_lo + g * NT;
-      const int nrows = min(NT, row_hi - g0);
-      bool ok = wait(bar_done + 8 * db, (g / C::ND) & 1);
-      ok = __all_sync(0xffffffffu, ok);
-      tc_fence_after();
-      const uint32_t dcol = tmem + lane_off + db * C::D_COLS;
+    uint32_t gp = 0;  // passes drained so far (over every task)
+    for (int t = pair; t < ntask; t += npairs) {
+      const Task k = task(t);
+      if (k.null_expert) {
+        // NULL expert: this CTA's outputs of its rows are zero.
+        constexpr int W = C::ROWS_PER_PAIR / 2;
+        for (int i = et; i < (k.row_hi - k.row_lo) * W; i += 128)
+          a.out[(size_t)(k.row_lo + i / W) * N + k.n_cta + i % W] = 0.0f;
+        continue;
+      }
+      const float s2a = a.s2_0[k.e];
+      const float s2b = a.s2_1[k.e];
+      // Output n of this lane: gate+up pairs lanes (2j: gate, 2j + 1: up of n_cta + j).
+      const int n = MODE == kModeGateUp ? k.n_cta + (L >> 1) : k.n_cta + L;
+      for (int g = 0; g < k.ngroups; ++g, ++gp) {
+        const uint32_t db = gp % C::ND;
+        const int g0 = k.row_lo + g * NT;
+        const int nrows = min(NT, k.row_hi - g0);
+        bool ok = wait(bar_done + 8 * db, (gp / C::ND) & 1);
+        ok = __all_sync(0xffffffffu, ok);
+        tc_fence_after();
+        const uint32_t dcol = tmem + lane_off + db * C::D_COLS;
 #pragma unroll 1
-      for (int c0 = 0; c0 < nrows; c0 += 32) {
-        // lane l holds the activation-row scale of token c0 + l
-        const float xm_l = (c0 + lane < nrows) ? a.bexp[g0 + c0 + lane] : 0.0f;
-        // 32 columns per wait (the D buffer holds NT >= c0 + 32 columns).
-        uint32_t d[32];
+        for (int c0 = 0; c0 < nrows; c0 += 32) {
+          // lane l holds the activation-row scale of token c0 + l
+          const float xm_l = (c0 + lane < nrows) ? a.bexp[g0 + c0 + lane] : 0.0f;
+          // 32 columns per wait (the D buffer holds NT >= c0 + 32 columns).
+          uint32_t d[32];
 #pragma unroll
-        for (int h = 0; h < 4; ++h) tmem_ld8(dcol + c0 + 8 * h, *reinterpret_cast<uint32_t(*)[8]>(d + 8 * h));
-        tmem_wait_ld();
-        if constexpr (MODE == kModeGateUp) {
+          for (int h = 0; h < 4; ++h) tmem_ld8(dcol + c0 + 8 * h, *reinterpret_cast<uint32_t(*)[8]>(d + 8 * h));
+          tmem_wait_ld();
+          if constexpr (MODE == kModeGateUp) {
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            // Even lane: gate of tokens t, t + 1; odd lane: up of the same.
-            // After the swap the even lane holds (g, u) of token t, the odd
-            // lane (g, u) of token t + 1.
-            const float mine0 = __uint_as_float(d[j]), mine1 = __uint_as_float(d[j + 1]);
-            const float other = __shfl_xor_sync(0xffffffffu, odd ? mine0 : mine1, 1);
-            const float gv = odd ? other : mine0;
-            const float uv = odd ? mine1 : other;
-            const int tl = j + odd;
-            const float xm = __shfl_sync(0xffffffffu, xm_l, tl);
-            const int t = c0 + tl;
-            if (ok && t < nrows) a.out[(size_t)(g0 + t) * N + n] = silu_f32(gv * xm * s2a) * (uv * xm * s2b);
-          }
-        } else {
+            for (int j = 0; j < 32; j += 2) {
+              // Even lane: gate of tokens t, t + 1; odd lane: up of the same.
+              // After the swap the even lane holds (g, u) of token t, the odd
+              // lane (g, u) of token t + 1.
+              const float mine0 = __uint_as_float(d[j]), mine1 = __uint_as_float(d[j + 1]);
+              const float other = __shfl_xor_sync(0xffffffffu, odd ? mine0 : mine1, 1);
+              const float gv = odd ? other : mine0;
+              const float uv = odd ? mine1 : other;
+              const int tl = j + odd;
+              const float xm = __shfl_sync(0xffffffffu, xm_l, tl);
+              const int tt = c0 + tl;
+              if (ok && tt < nrows) a.out[(size_t)(g0 + tt) * N + n] = silu_f32(gv * xm * s2a) * (uv * xm * s2b);
+            }
+          } else {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float xm = __shfl_sync(0xffffffffu, xm_l, j);
-            const int t = c0 + j;
-            float v = __uint_as_float(d[j]) * xm * s2a;
-            if constexpr (MODE == kModeUpAct) v = activation_f32(a.activation, v);
-            if (ok && t < nrows) a.out[(size_t)(g0 + t) * N + n] = v;
+            for (int j = 0; j < 32; ++j) {
+              const float xm = __shfl_sync(0xffffffffu, xm_l, j);
+              const int tt = c0 + j;
+              float v = __uint_as_float(d[j]) * xm * s2a;
+              if constexpr (MODE == kModeUpAct) v = activation_f32(a.activation, v);
+              if (ok && tt < nrows) a.out[(size_t)(g0 + tt) * N + n] = v;
+            }
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(lead_dfree + 8 * db);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(lead_dfree + 8 * db);
     }
   }
 
@@ -418,6 +450,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, NT > 3
 
 namespace {
 
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 2) return 148;
+  return n;
+}
+
+// Persistent launch: one pair per two SMs (two at 32-row passes), or fewer
+// when there are fewer tasks than that.
 template <int MODE, int NT>
 cudaError_t launch_tc_pair_impl(const TcArgs& a, const CUtensorMap& b0, const CUtensorMap& b1, uint32_t cap,
                                 cudaStream_t stream) {
@@ -425,8 +466,13 @@ cudaError_t launch_tc_pair_impl(const TcArgs& a, const CUtensorMap& b0, const CU
   auto kern = grouped_tc_pair_kernel<MODE, NT>;
   cudaError_t err = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::SMEM);
   if (err != cudaSuccess) return err;
-  const dim3 grid(2 * (a.N / C::ROWS_PER_PAIR), cap);
-  return launch_pdl(kern, grid, dim3(kPairThreads), C::SMEM, stream, a, b0, b1);
+  const uint64_t tasks = (uint64_t)cap * (a.N / C::ROWS_PER_PAIR);
+  uint64_t pairs = (uint64_t)(sm_count() / 2) * C::CTAS_PER_SM;
+  if (pairs > tasks) pairs = tasks;
+  if (pairs == 0) return cudaSuccess;
+  TcArgs args = a;
+  args.cap = cap;
+  return launch_pdl(kern, dim3((unsigned)(2 * pairs)), dim3(kPairThreads), C::SMEM, stream, args, b0, b1);
 }
 
 }  // namespace
