@@ -109,6 +109,10 @@ def parse_args(argv=None):
                     help="use the calls without workspace (decode path only)")
     ap.add_argument("--replicas", type=int, default=0,
                     help="weight replicas to rotate over (0: enough to exceed 4 x L2)")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="override the workload's expert count (a reduced case for profiling)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the workload's token count (a reduced case for profiling)")
     return ap.parse_args(argv)
 
 
@@ -250,7 +254,7 @@ def run_ours(args, rank, world, local):
     from workloads import make_problem
     from workloads.device import upload_inputs, upload_layer
 
-    prob = make_problem(args.config)
+    prob = make_problem(args.config, **_overrides(args))
     cfg = prob.cfg
     steps = args.steps if args.steps is not None else DEFAULT_STEPS.get(cfg.name, 1000)
     warmup = max(args.warmup, 3)
@@ -413,7 +417,9 @@ def run_ours(args, rank, world, local):
         "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
         "steps": steps, "warmup": warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16-mma/f32-acc", "data": "synthetic",
-        "config": {"workload": cfg.name + ("+shared" if args.shared else ""), "hidden": cfg.hidden, "inter": cfg.inter,
+        "config": {"workload": cfg.name + ("+shared" if args.shared else "")
+                   + (" (reduced: experts/tokens overridden)" if _overrides(args) else ""),
+                   "hidden": cfg.hidden, "inter": cfg.inter,
                    "experts": cfg.experts, "topk": cfg.topk, "tokens": cfg.tokens,
                    "router": cfg.router, "active_experts": active,
                    "shared_expert": ({"rows_per_table_entry": base.rows_per_shared_slot(cfg.tokens),
@@ -445,6 +451,16 @@ def run_ours(args, rank, world, local):
     if world > 1:
         del g_steps, g_one, gu_graph
         dist.destroy_process_group()
+
+
+def _overrides(args):
+    """Reduced-case overrides (profiling): expert and token counts."""
+    out = {}
+    if args.experts:
+        out["experts"] = args.experts
+    if args.tokens:
+        out["tokens"] = args.tokens
+    return out
 
 
 def _opts(args):
@@ -640,7 +656,7 @@ def run_load_op(args, rank, world, local):
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    prob = make_problem(args.config)
+    prob = make_problem(args.config, **_overrides(args))
     cfg = prob.cfg
     layer = upload_layer(prob, dev)
     projs = (layer.gate, layer.up, layer.down)
