@@ -54,6 +54,8 @@ DEFAULT_STEPS = {"tiny": 4000, "decode_m1": 4000, "decode_m32": 2000, "decode_m2
 KERNEL_SOURCES = {
     "tcgen05": ["grouped_tc.cu", "grouped_tc_pair.cuh", "tc_common.cuh", "common.cuh"],
     "mma.sync": ["grouped_mma.cu", "common.cuh"],
+    "check_scales": ["check_scales.cu"],
+    "transpose_u8": ["transpose_u8.cu"],
 }
 
 # DRAM bytes (read + write) of one launch of the dominant kernel (gate+up
@@ -61,9 +63,19 @@ KERNEL_SOURCES = {
 # kernel, with the hash of that kernel's sources when it was captured.  An
 # entry whose hash no longer matches the sources is stale and not reported.
 NCU_TRAFFIC_BYTES = {
-    ("decode_m1", "mma.sync"): (28357888, "00f418d43112"),
-    ("decode_m32", "tcgen05"): (335457536, "5e2f82da6383"),
-    ("prefill_m8192", "tcgen05"): (4249585000, "5e2f82da6383"),
+    ("decode_m1", "mma.sync"): (28357376, "b043af2a146a"),       # 28.36 MB read, 0 written
+    ("decode_m32", "tcgen05"): (299103232, "ba425bfe1e4c"),      # 293.13 MB read, 5.97 MB written
+    # reduced case (64 experts, 64 tokens: the same 8 rows per expert) x 4 experts
+    ("decode_m256", "tcgen05"): (4519915520, "ba425bfe1e4c"),    # 4 x (1122.36 + 7.62) MB
+    ("prefill_m8192", "tcgen05"): (2114844000, "ba425bfe1e4c"),  # 1.7252 GB read, 0.3896 GB written
+}
+
+
+# The same for one launch of a load-time op's kernel (per projection for the
+# scale check; per transposed matrix for the twins), keyed by op and workload.
+NCU_OP_TRAFFIC_BYTES = {
+    ("check_scales", "prefill_m8192"): (50353152, "5b4491c5e4d3"),   # 50.34 MB read, 0.01 MB written
+    ("twins", "prefill_m8192"): (3150336, "07ac2b2c0b60"),           # packed part of one expert: 3.15 MB read
 }
 
 
@@ -453,6 +465,16 @@ def run_ours(args, rank, world, local):
         dist.destroy_process_group()
 
 
+def _op_traffic(op, workload):
+    """ncu DRAM bytes of one launch of a load-time op's kernel, or None when absent
+    or taken from other sources."""
+    entry = NCU_OP_TRAFFIC_BYTES.get((op, workload))
+    kernel = {"check_scales": "check_scales", "twins": "transpose_u8"}.get(op)
+    if entry is None or kernel is None or entry[1] != kernel_source_hash(kernel):
+        return None
+    return entry[0]
+
+
 def _overrides(args):
     """Reduced-case overrides (profiling): expert and token counts."""
     out = {}
@@ -735,7 +757,9 @@ def run_load_op(args, rank, world, local):
                      else "check_scales_kernel",
                      "bound": "hbm", "achieved": gbs, "peak": hbm,
                      "unit": "GB/s", "frac": gbs / hbm, "peak_source": f"{peak_kind} HBM copy",
-                     "traffic": None},
+                     "traffic": _op_traffic(args.op, cfg.name),
+                     "traffic_unit": "bytes per launch (one projection's scale table; one "
+                                     "transposed packed part)"},
         "gpu_launches": (4 * cfg.experts if twins else 6 if shard else 3) * steps,
         "clocks": clocks,
     }
