@@ -520,15 +520,16 @@ SHARED_CASES = [("tiny", 0, False), ("ragged", 2, True), ("hot", 16, True), ("zi
                 ("longk", 1, True)]
 
 
-@pytest.mark.parametrize("ws", [False, True], ids=["decode-path", "tcgen05"])
+@pytest.mark.parametrize("ws,tiles", [(False, 0), (True, 0), (True, 24)],
+                         ids=["decode-path", "tcgen05", "tcgen05-pair192"])
 @pytest.mark.parametrize("name,rows,weighted", SHARED_CASES)
-def test_forward_with_shared_expert(name, rows, weighted, ws):
+def test_forward_with_shared_expert(name, rows, weighted, ws, tiles):
     _need_gpu()
     prob = make_problem(SMALL[name])
     cfg = prob.cfg
     sw = (np.random.default_rng(cfg.seed).random(cfg.tokens).astype(np.float32)
           if weighted else None)
-    opts = dict(path=2) if ws else {}
+    opts = (dict(path=2, tiles=tiles) if tiles else dict(path=2)) if ws else {}
     layer, bufs = _gpu_forward_shared(prob, sw, rows, ws=ws, **opts)
     ref = _shared_ref(prob, sw)
     # The sort of the appended routing is bit-exact; the shared rows come last.
@@ -803,9 +804,16 @@ def _sum_over_ranks(prob, layers, ws, shared=False, **opts):
     return total.cpu().numpy()
 
 
-@pytest.mark.parametrize("ws", [False, True], ids=["decode-path", "tcgen05"])
+# Kernels of the sharded forwards: decode kernel; tcgen05 from the shape; the
+# CTA-pair kernel at 32- and 192-row passes (the shard widths I/tp = 768, 512,
+# 256 all divide into its 128 / 256-row column blocks).
+SHARD_PATHS = [dict(), dict(ws=True, path=2), dict(ws=True, path=2, tiles=4), dict(ws=True, path=2, tiles=24)]
+SHARD_IDS = ["decode-path", "tcgen05", "tcgen05-pair32", "tcgen05-pair192"]
+
+
+@pytest.mark.parametrize("opts", SHARD_PATHS, ids=SHARD_IDS)
 @pytest.mark.parametrize("tp", [2, 3, 6])
-def test_tensor_parallel_ranks_sum_to_the_full_forward(tp, ws):
+def test_tensor_parallel_ranks_sum_to_the_full_forward(tp, opts):
     _need_gpu()
     from workloads.device import upload_layer
     prob = make_problem(SHARD_CFG)
@@ -813,20 +821,22 @@ def test_tensor_parallel_ranks_sum_to_the_full_forward(tp, ws):
     full = upload_layer(prob, shared=True)
     layers = [full.tensor_parallel(r, tp) for r in range(tp)]
     assert layers[0].inter == cfg.inter // tp
-    got = _sum_over_ranks(prob, layers, ws, **(dict(path=2) if ws else {}))
+    opts = dict(opts)
+    got = _sum_over_ranks(prob, layers, opts.pop("ws", False), **opts)
     ref = _shared_ref(prob, None)["out"]
     _close(got, ref, f"sum of {tp} tensor-parallel ranks")
 
 
-@pytest.mark.parametrize("ws", [False, True], ids=["decode-path", "tcgen05"])
+@pytest.mark.parametrize("opts", SHARD_PATHS, ids=SHARD_IDS)
 @pytest.mark.parametrize("world", [2, 4])
-def test_expert_parallel_ranks_sum_to_the_full_forward(world, ws):
+def test_expert_parallel_ranks_sum_to_the_full_forward(world, opts):
     _need_gpu()
     from workloads.device import upload_layer
     prob = make_problem(SHARD_CFG)
     full = upload_layer(prob, shared=True)
     layers = [full.expert_parallel(r, world) for r in range(world)]
-    got = _sum_over_ranks(prob, layers, ws, **(dict(path=2) if ws else {}))
+    opts = dict(opts)
+    got = _sum_over_ranks(prob, layers, opts.pop("ws", False), **opts)
     ref = _shared_ref(prob, None)["out"]
     _close(got, ref, f"sum of {world} expert-parallel ranks")
 
