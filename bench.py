@@ -436,7 +436,7 @@ def run_ours(args, rank, world, local):
                    "router": cfg.router, "active_experts": active,
                    "shared_expert": ({"rows_per_table_entry": base.rows_per_shared_slot(cfg.tokens),
                                       "table_entries": slots} if args.shared else None),
-                   "path": (f"tcgen05-pair-nt{rows}" if rows in (32, 192) else f"tcgen05-nt{rows}")
+                   "path": (f"tcgen05-pair-nt{rows}" if rows in (32, 192, 256) else f"tcgen05-nt{rows}")
                            if tc else "mma.sync",
                    "weight_replicas": len(layers),
                    "l2": f"weights rotate over {len(layers)} device replicas; "
@@ -510,11 +510,13 @@ def _tc_rows(args, tokens, pairs, experts):
         return args.tiles * 8
     mean = (pairs + experts - 1) // experts
     if mean > 16:
-        return 192
+        return 256
     return 32 if tokens > 16 and mean <= 4 else 16
 
 
 def _tc_kernel_name(rows):
+    if rows == 256:
+        return "tcgen05 CTA pair, 256-row passes, A in shared memory"
     return (f"tcgen05 CTA pair, {rows}-row passes" if rows in (32, 192)
             else f"tcgen05 one CTA, {rows}-row passes")
 

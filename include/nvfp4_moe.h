@@ -216,8 +216,9 @@ NVFP4_MOE_API size_t nvfp4_moe_workspace_bytes(uint32_t num_tokens, uint32_t top
  * nvfp4_moe_workspace_bytes(num_tokens, topk, hidden, inter) bytes, 256-byte
  * aligned (NVFP4_MOE_EINVAL otherwise), owned by the caller, overwritten by
  * the call.  For the tcgen05
- * path opts->tiles selects the token rows per pass (2 -> 16, 16 -> 128; 0 =
- * from the shape).  Results equal the other path's within FP32 rounding.
+ * path opts->tiles selects the token rows per pass: 2 -> 16 and 16 -> 128 (one
+ * CTA per 128 or 256 output rows); 4 -> 32, 24 -> 192 and 32 -> 256 (a cluster
+ * of two CTAs sharing each MMA; down takes 192 for 32); 0 = from the shape.  Results equal the other path's within FP32 rounding.
  * Calls on one stream may share the workspace; concurrent calls may not.
  */
 NVFP4_MOE_API int nvfp4_moe_gate_up_silu_ws(

@@ -260,8 +260,8 @@ int nvfp4_moe_gate_up_silu_ws(const uint16_t* x, nvfp4_expert_tables gate, nvfp4
     return NVFP4_MOE_EINVAL;
   if (workspace_bytes < tc_workspace_bytes(num_tokens, topk, k_hidden, n_inter)) return NVFP4_MOE_EINVAL;
   if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return NVFP4_MOE_EINVAL;
-  const int nt = plan_tc_rows(num_tokens, pairs, num_experts, opts ? opts->tiles : 0);
-  if (nt != 16 && nt != 128 && nt != kTcPairRows && nt != kTcPairRowsSmall) return NVFP4_MOE_EINVAL;
+  const int nt = plan_tc_rows(num_tokens, pairs, num_experts, opts ? opts->tiles : 0, kModeGateUp);
+  if (nt != 16 && nt != 128 && nt != kTcPairRows && nt != kTcPairRowsSmall && nt != kTcPairRowsWide) return NVFP4_MOE_EINVAL;
   GroupedArgs a{};
   a.src = x;
   a.packed0 = gate.packed_ptrs;
@@ -306,7 +306,8 @@ int nvfp4_moe_down_ws(const float* act, nvfp4_expert_tables down, float* y,
     return NVFP4_MOE_EINVAL;
   if (workspace_bytes < tc_workspace_bytes(num_tokens, topk, n_hidden, k_inter)) return NVFP4_MOE_EINVAL;
   if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return NVFP4_MOE_EINVAL;
-  const int nt = plan_tc_rows(num_tokens, pairs, num_experts, opts ? opts->tiles : 0);
+  int nt = plan_tc_rows(num_tokens, pairs, num_experts, opts ? opts->tiles : 0, kModeDown);
+  if (nt == kTcPairRowsWide) nt = kTcPairRows;  // down's widest pair pass (A in tensor memory)
   if (nt != 16 && nt != 128 && nt != kTcPairRows && nt != kTcPairRowsSmall) return NVFP4_MOE_EINVAL;
   GroupedArgs a{};
   a.src = act;
@@ -387,8 +388,8 @@ int nvfp4_moe_up_act_ws(const uint16_t* x, nvfp4_expert_tables up, float* act,
     return NVFP4_MOE_EINVAL;
   if (workspace_bytes < tc_workspace_bytes(num_tokens, topk, k_hidden, n_inter)) return NVFP4_MOE_EINVAL;
   if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return NVFP4_MOE_EINVAL;
-  const int nt = plan_tc_rows(num_tokens, pairs, num_experts, opts ? opts->tiles : 0);
-  if (nt != 16 && nt != 128 && nt != kTcPairRows && nt != kTcPairRowsSmall) return NVFP4_MOE_EINVAL;
+  const int nt = plan_tc_rows(num_tokens, pairs, num_experts, opts ? opts->tiles : 0, kModeUpAct);
+  if (nt != 16 && nt != 128 && nt != kTcPairRows && nt != kTcPairRowsSmall && nt != kTcPairRowsWide) return NVFP4_MOE_EINVAL;
   GroupedArgs a{};
   a.src = x;
   a.packed0 = up.packed_ptrs;

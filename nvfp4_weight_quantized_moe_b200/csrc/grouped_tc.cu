@@ -778,11 +778,12 @@ cudaError_t launch_tc(int mode, int nt, const GroupedArgs& g, void* workspace, u
   const uint64_t pairs = (uint64_t)tokens * g.topk;
   const WsLayout w = ws_layout(workspace, pairs, hidden, inter);
   if (g.num_experts == 0 || g.num_experts > kMaxExperts ||
-      (nt != 16 && nt != 128 && nt != kTcPairRows && nt != kTcPairRowsSmall))
+      (nt != 16 && nt != 128 && nt != kTcPairRows && nt != kTcPairRowsSmall && nt != kTcPairRowsWide) ||
+      (nt == kTcPairRowsWide && mode == kModeDown))
     return cudaErrorInvalidValue;
-  // Pair passes (192 or 32 rows) run the CTA-pair kernel: 64-row weight boxes,
-  // token boxes of half a pass.
-  const bool pair = nt == kTcPairRows || nt == kTcPairRowsSmall;
+  // Pair passes (256, 192 or 32 rows) run the CTA-pair kernel: 64-row weight
+  // boxes, token boxes of half a pass.
+  const bool pair = nt == kTcPairRows || nt == kTcPairRowsSmall || nt == kTcPairRowsWide;
   TcArgs a{};
   a.packed0 = g.packed0;
   a.packed1 = g.packed1 != nullptr ? g.packed1 : g.packed0;
@@ -823,6 +824,7 @@ cudaError_t launch_tc(int mode, int nt, const GroupedArgs& g, void* workspace, u
     b1 = b0;
     a.bexp = w.xexp;
     a.wmaps = w.maps_gu;
+    if (nt == kTcPairRowsWide) return launch_tc_pair_impl<kModeGateUp, kTcPairRowsWide>(a, b0, b1, cap, stream);
     if (nt == kTcPairRows) return launch_tc_pair_impl<kModeGateUp, kTcPairRows>(a, b0, b1, cap, stream);
     if (nt == kTcPairRowsSmall) return launch_tc_pair_impl<kModeGateUp, kTcPairRowsSmall>(a, b0, b1, cap, stream);
     if (nt == 16) return launch_tc_impl<kModeGateUp, 16>(a, b0, b1, cap, stream);
@@ -843,6 +845,7 @@ cudaError_t launch_tc(int mode, int nt, const GroupedArgs& g, void* workspace, u
     b1 = b0;
     a.bexp = w.xexp;
     a.wmaps = w.maps_gu;
+    if (nt == kTcPairRowsWide) return launch_tc_pair_impl<kModeUpAct, kTcPairRowsWide>(a, b0, b1, cap, stream);
     if (nt == kTcPairRows) return launch_tc_pair_impl<kModeUpAct, kTcPairRows>(a, b0, b1, cap, stream);
     if (nt == kTcPairRowsSmall) return launch_tc_pair_impl<kModeUpAct, kTcPairRowsSmall>(a, b0, b1, cap, stream);
     if (nt == 16) return launch_tc_impl<kModeUpAct, 16>(a, b0, b1, cap, stream);

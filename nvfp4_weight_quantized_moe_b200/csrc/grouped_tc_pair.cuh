@@ -19,11 +19,13 @@
 // consecutive rows n0 + 128 r .. + 127 of the one matrix.
 //
 // Roles (15 warps per CTA), synchronised by mbarriers only:
-//   warps 0-7   decoders: TMEM lane 32 (w % 4) + l, the 64-k stages of parity
+//   warps 0-7   decoders: A row 32 (w % 4) + l, the 64-k stages of parity
 //               w / 4; 32 nibble bytes and 4 scales per stage from the weight
-//               tile in shared memory, exact E2M1 x E4M3 -> f16, tcgen05.st
-//               into the A ring; each warp then arrives on the first CTA's
-//               full_a barrier (the peer's warps remotely);
+//               tile in shared memory, exact E2M1 x E4M3 -> f16, into the A
+//               ring (tcgen05.st into tensor memory, or, at 256-row passes,
+//               128-byte-swizzled rows in shared memory); each warp then
+//               arrives on the first CTA's full_a barrier (the peer's warps
+//               remotely);
 //   warp 8      first CTA: MMA issuer (one thread): per two stages, waits
 //               for their full_a barriers (both CTAs' A stage; one decoder
 //               lane folds in the token tile's arrival), issues the pair MMAs
@@ -52,36 +54,43 @@ constexpr int kPairWBoxRows = 64;           // rows per weight TMA box
 constexpr int kPairWNib = 128 * 128;        // nibble bytes of a CTA's weight tile (128 rows x 256 k)
 constexpr int kPairWSlot = kPairWNib + 128 * 16;
 
-// NT: token rows per pass of the pair (the MMA's N at most): 192 for experts
-// with many rows (one pair per SM pair), 32 for decode-shaped batches (two
-// pairs per SM pair, each with its own MMA issuer and weight stream).
+// NT: token rows per pass of the pair (the MMA's N at most): 256 for gate+up
+// of experts with many rows, with the A operand in shared memory (two 256-column
+// accumulators fill tensor memory); 192 for down of such experts (A in tensor
+// memory; its hi + lo token planes leave no shared memory for A); 32 for
+// decode-shaped batches (two pairs per SM pair, each with its own MMA issuer
+// and weight stream; A in tensor memory).
 template <int MODE, int NT>
 struct PairCfg {
+  static constexpr bool SMEM_A = NT == 256;                           // A operand in shared memory
   static constexpr int HALF = NT / 2;                                 // token rows each CTA loads
   static constexpr int CTAS_PER_SM = NT > 32 ? 1 : 2;
   static constexpr int PLANES = MODE == kModeDown ? 2 : 1;           // down: f16 hi + lo
   static constexpr int ROWS_PER_PAIR = MODE == kModeGateUp ? 128 : 256;  // outputs n per pair
   static constexpr int B_PLANE_BYTES = HALF * kStageK * 2;           // HALF rows x 64 k f16
   static constexpr int B_SLOT_BYTES = PLANES * B_PLANE_BYTES;
-  static constexpr int A_COLS = 32;                                   // TMEM columns per A stage
+  static constexpr int A_COLS = 32;                                   // TMEM columns per A stage (A in TMEM)
+  static constexpr int A_STAGE_BYTES = 128 * kStageK * 2;             // 128 rows x 64 k f16 (A in smem)
   static constexpr int D_COLS = NT;                                   // per D buffer
   static constexpr int ND = 2;                                        // D buffers
-  static constexpr int WS = 3;
-  static constexpr int SB = (MODE == kModeDown && NT > 32) ? 4 : 8;
+  static constexpr int WS = SMEM_A ? 2 : 3;
+  static constexpr int SB = SMEM_A ? 6 : (MODE == kModeDown && NT > 32) ? 4 : 8;
   static constexpr uint32_t TMEM_COLS = 512 / CTAS_PER_SM;
   // A ring: the rest of the CTA's tensor memory, at most SB stages (the
   // completion ring of SB entries also tells the decoders when an A slot is free).
   static constexpr int SA_TMEM = ((int)TMEM_COLS - ND * D_COLS) / A_COLS;
-  static constexpr int SA = SA_TMEM < SB ? SA_TMEM : SB;
+  static constexpr int SA = SMEM_A ? 4 : (SA_TMEM < SB ? SA_TMEM : SB);
   static constexpr int OFF_W = 0;
   static constexpr int OFF_B = WS * kPairWSlot;
-  static constexpr int OFF_BAR = OFF_B + SB * B_SLOT_BYTES;
+  static constexpr int OFF_A = OFF_B + SB * B_SLOT_BYTES;             // A ring (A in smem only)
+  static constexpr int OFF_BAR = OFF_A + (SMEM_A ? SA * A_STAGE_BYTES : 0);
   // full_w[WS], empty_w[WS], full_b[SB], mma_done[SB], full_a[SA], done[ND], dfree[ND]
   static constexpr int NBAR = 2 * WS + 2 * SB + SA + 2 * ND;
   static constexpr int OFF_TMEM = OFF_BAR + 8 * NBAR;
   static constexpr int OFF_ABORT = OFF_TMEM + 16;
   static constexpr int SMEM = OFF_ABORT + 16 + 1024;
-  static_assert(ND * D_COLS + SA * A_COLS <= (int)TMEM_COLS && SA >= 2, "TMEM budget");
+  static_assert(ND * D_COLS + (SMEM_A ? 0 : SA * A_COLS) <= (int)TMEM_COLS && SA >= 2, "TMEM budget");
+  static_assert(!SMEM_A || (MODE != kModeDown && CTAS_PER_SM == 1), "A in shared memory: gate+up / up+activation");
   static_assert(B_PLANE_BYTES % 1024 == 0 && kPairWSlot % 1024 == 0, "TMA tiles stay 1024-byte aligned");
   static_assert(SB >= SA && SB % 2 == 0, "mma_done (odd entries, one commit per two stages) also tracks the A ring");
   static_assert(CTAS_PER_SM * (SMEM + 1024) <= 228 * 1024, "shared memory per SM");
@@ -284,11 +293,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, NT > 3
             for (int h = 0; h < 2; ++h) {
               const uint32_t gx = ga + h;
               const uint32_t bbase = s_base + C::OFF_B + (gx % C::SB) * C::B_SLOT_BYTES;
-              const uint32_t abase = tmem_a + (gx % C::SA) * C::A_COLS;
+              const uint32_t abase = C::SMEM_A ? s_base + C::OFF_A + (gx % C::SA) * C::A_STAGE_BYTES
+                                               : tmem_a + (gx % C::SA) * C::A_COLS;
 #pragma unroll
               for (int s = 0; s < 4; ++s) {
                 const uint32_t acc = (st + h > 0 || s > 0) ? 1u : 0u;
-                tc_mma_pair_f16_ts(dcol, abase + s * 8, smem_desc_sw128(bbase + s * 32), idesc, acc);
+                if constexpr (C::SMEM_A)
+                  tc_mma_pair_f16_ss(dcol, smem_desc_sw128(abase + s * 32), smem_desc_sw128(bbase + s * 32), idesc, acc);
+                else
+                  tc_mma_pair_f16_ts(dcol, abase + s * 8, smem_desc_sw128(bbase + s * 32), idesc, acc);
                 if constexpr (MODE == kModeDown)
                   tc_mma_pair_f16_ts(dcol, abase + s * 8, smem_desc_sw128(bbase + C::B_PLANE_BYTES + s * 32), idesc,
                                      1u);
@@ -353,10 +366,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, NT > 3
               if (lane == 0) mbar_arrive(empty_w + 8 * wslot);
             }
             if (ga >= (uint32_t)C::SA) wait_mma(ga - C::SA);  // the A slot's previous MMAs are done
-            tc_fence_after();
-            tmem_st32(tmem_a + lane_off + aslot * C::A_COLS, v);
-            tmem_wait_st();
-            tc_fence_before();
+            if constexpr (C::SMEM_A) {
+              // Row L of the stage's K-major tile, 128-byte swizzle: 16-byte
+              // chunk c (k 8 c .. 8 c + 7) at chunk position c ^ (L % 8).
+              uint8_t* arow = smem + C::OFF_A + aslot * C::A_STAGE_BYTES + L * 128;
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(arow + ((c ^ (L & 7)) << 4)) =
+                    make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+              fence_proxy_async_smem();  // generic-proxy writes -> the MMA's async-proxy reads
+            } else {
+              tc_fence_after();
+              tmem_st32(tmem_a + lane_off + aslot * C::A_COLS, v);
+              tmem_wait_st();
+              tc_fence_before();
+            }
             __syncwarp();
             if (lane == 0) {
               // In the first CTA, warp 0 / 4 also reports the stage's token tile.

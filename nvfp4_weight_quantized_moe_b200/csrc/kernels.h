@@ -18,7 +18,9 @@ constexpr uint32_t kMaxExperts = 1024;
 constexpr uint64_t kMaxPairs = 1ull << 24;
 
 // Token rows per pass of the tcgen05 kernels, from the host-known sizes:
-//   * more than 16 rows per expert on average: 192 (the CTA-pair kernel);
+//   * more than 16 rows per expert on average: the CTA-pair kernel at 256-row
+//     passes for gate+up and up+activation (A operand in shared memory), 192
+//     for down (A in tensor memory);
 //   * batches of at most 16 tokens (no expert can have more rows), or 5..16
 //     rows per expert on average: 16 (one-CTA kernel, one pass per expert);
 //   * more than 16 tokens spread at most 4 per expert on average, where a
@@ -27,13 +29,15 @@ constexpr uint64_t kMaxPairs = 1ull << 24;
 // Measured on B200: 32-row pair passes 12 % faster than 16-row passes on the
 // skewed decode M=32 workload (2 rows per expert on average), 13 % slower on
 // decode M=256 (8 per expert, uniform).  `tiles` > 0 (a launch option) forces
-// tiles * 8: 2 -> 16, 16 -> 128 (one-CTA kernel), 4 -> 32, 24 -> 192 (pair).
+// tiles * 8: 2 -> 16, 16 -> 128 (one-CTA kernel), 4 -> 32, 24 -> 192 and (not
+// for down) 32 -> 256 (pair kernel).
 constexpr int kTcPairRows = 192;
 constexpr int kTcPairRowsSmall = 32;
-inline int plan_tc_rows(uint64_t tokens, uint64_t pairs, uint32_t num_experts, int tiles) {
+constexpr int kTcPairRowsWide = 256;
+inline int plan_tc_rows(uint64_t tokens, uint64_t pairs, uint32_t num_experts, int tiles, int mode) {
   if (tiles > 0) return tiles * 8;
   const uint64_t mean = (pairs + num_experts - 1) / num_experts;
-  if (mean > 16) return kTcPairRows;
+  if (mean > 16) return mode == kModeDown ? kTcPairRows : kTcPairRowsWide;
   if (tokens > 16 && mean <= 4) return kTcPairRowsSmall;
   return 16;
 }

@@ -82,7 +82,7 @@ extern "C" int nvfp4_moe_gate_up_silu_noalloc(
   if (static_scratch_address(&scratch) != cudaSuccess) return NVFP4_MOE_ECUDA;
   // Nothing in the scratch has to start at zero: the pack kernel writes every
   // packed row and scale before the projection kernel reads them.
-  const int nt = plan_tc_rows(num_tokens, pairs, num_experts, 0);  // the _ws call's rule
+  const int nt = plan_tc_rows(num_tokens, pairs, num_experts, 0, kModeGateUp);  // the _ws call's rule
   GroupedArgs a{};
   a.src = x;
   a.packed0 = gate.packed_ptrs;

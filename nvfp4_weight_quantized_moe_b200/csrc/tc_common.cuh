@@ -264,6 +264,19 @@ NVM_DEV void tc_mma_pair_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_des
       "r"(0u), "r"(0u)
       : "memory");
 }
+// The same with A from shared memory too (each CTA's 128 rows at the address
+// its descriptor gives, K-major).
+NVM_DEV void tc_mma_pair_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8, %9, %10, %11, %12}, p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u), "r"(0u), "r"(0u),
+      "r"(0u), "r"(0u)
+      : "memory");
+}
 // Arrive on the mbarrier at shared::cta offset `bar` in every CTA of `cta_mask`
 // once all pair MMAs this thread issued have completed.
 NVM_DEV void tc_commit_pair(uint32_t bar, uint16_t cta_mask) {

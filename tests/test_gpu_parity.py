@@ -288,8 +288,9 @@ def test_gate_up_four_tiles():
 
 
 # tcgen05 path: token rows per pass 16 (tiles=2) or 128 (tiles=16) on the one-CTA
-# kernel, 32 (tiles=4) or 192 (tiles=24) on the CTA-pair kernel; 0 = from the shape.
-@pytest.mark.parametrize("tiles", [0, 2, 4, 16, 24])
+# kernel, 32 (tiles=4), 192 (tiles=24) or 256 (tiles=32: gate+up with A in shared
+# memory, down at 192) on the CTA-pair kernel; 0 = from the shape.
+@pytest.mark.parametrize("tiles", [0, 2, 4, 16, 24, 32])
 @pytest.mark.parametrize("name", list(SMALL))
 def test_forward_small_tcgen05(name, tiles):
     _need_gpu()
@@ -312,7 +313,7 @@ PAIR_CFG = MoEConfig("pairrows", hidden=512, inter=256, experts=12, topk=3, toke
                      router="zipf", seed=25)
 
 
-@pytest.mark.parametrize("tiles", [24, 16, 4])
+@pytest.mark.parametrize("tiles", [32, 24, 16, 4])
 def test_forward_pair_kernel_pass_lengths(tiles):
     _need_gpu()
     prob = make_problem(PAIR_CFG)
@@ -520,8 +521,8 @@ SHARED_CASES = [("tiny", 0, False), ("ragged", 2, True), ("hot", 16, True), ("zi
                 ("longk", 1, True)]
 
 
-@pytest.mark.parametrize("ws,tiles", [(False, 0), (True, 0), (True, 24)],
-                         ids=["decode-path", "tcgen05", "tcgen05-pair192"])
+@pytest.mark.parametrize("ws,tiles", [(False, 0), (True, 0), (True, 24), (True, 32)],
+                         ids=["decode-path", "tcgen05", "tcgen05-pair192", "tcgen05-pair256"])
 @pytest.mark.parametrize("name,rows,weighted", SHARED_CASES)
 def test_forward_with_shared_expert(name, rows, weighted, ws, tiles):
     _need_gpu()
@@ -639,7 +640,8 @@ def _gpu_forward_nongated(prob, activation, ws=False, null=(), **opts):
 # (path options): decode kernel automatic and forced shapes; tcgen05 16- and 128-row passes.
 NONGATED_PATHS = [dict(), dict(path=1, split=4, tiles=1, depth=2), dict(path=1, split=1, tiles=2, depth=3),
                   dict(ws=True, path=2, tiles=2), dict(ws=True, path=2, tiles=16),
-                  dict(ws=True, path=2, tiles=4), dict(ws=True, path=2, tiles=24)]
+                  dict(ws=True, path=2, tiles=4), dict(ws=True, path=2, tiles=24),
+                  dict(ws=True, path=2, tiles=32)]
 
 
 @pytest.mark.parametrize("opts", NONGATED_PATHS, ids=lambda o: "-".join(f"{k}{v}" for k, v in o.items()) or "auto")
@@ -807,8 +809,9 @@ def _sum_over_ranks(prob, layers, ws, shared=False, **opts):
 # Kernels of the sharded forwards: decode kernel; tcgen05 from the shape; the
 # CTA-pair kernel at 32- and 192-row passes (the shard widths I/tp = 768, 512,
 # 256 all divide into its 128 / 256-row column blocks).
-SHARD_PATHS = [dict(), dict(ws=True, path=2), dict(ws=True, path=2, tiles=4), dict(ws=True, path=2, tiles=24)]
-SHARD_IDS = ["decode-path", "tcgen05", "tcgen05-pair32", "tcgen05-pair192"]
+SHARD_PATHS = [dict(), dict(ws=True, path=2), dict(ws=True, path=2, tiles=4), dict(ws=True, path=2, tiles=24),
+               dict(ws=True, path=2, tiles=32)]
+SHARD_IDS = ["decode-path", "tcgen05", "tcgen05-pair32", "tcgen05-pair192", "tcgen05-pair256"]
 
 
 @pytest.mark.parametrize("opts", SHARD_PATHS, ids=SHARD_IDS)
