@@ -136,17 +136,15 @@ NVM_DEV uint32_t pack_f16x2(float a, float b) {
 // Activation packing (once per call)
 // ---------------------------------------------------------------------------
 
-// One warp per sorted row r < offsets[E]: xs[r] = f16(x[t] * 2^-e), t the
-// row's token, xexp[r] = 2^e.
+// One warp per token t < M: texp[t] = e, the power of two that brings the
+// token's row of x into the f16 range (f16_range_exponent of its max |value|).
+// A token's row is packed once per routed slot, so its exponent is found once.
 __global__ void __launch_bounds__(256)
-    pack_x_sorted_kernel(const uint16_t* __restrict__ x, int P, int K, int topk,
-                         const int32_t* __restrict__ sorted_pair_ids, const int32_t* __restrict__ kept_rows,
-                         uint16_t* __restrict__ xs, float* __restrict__ xexp) {
+    token_exp_kernel(const uint16_t* __restrict__ x, int M, int K, int32_t* __restrict__ texp) {
   griddep_wait();
   griddep_launch_dependents();
-  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (row >= P || row >= *kept_rows) return;
-  const int t = sorted_pair_ids[row] / topk;
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (t >= M) return;
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * K);
   float m = 0.0f;
   for (int i = lane; i < K / 8; i += 32) {
@@ -159,7 +157,23 @@ __global__ void __launch_bounds__(256)
     }
   }
   const int e = f16_range_exponent(warp_max(m));
+  if (lane == 0) texp[t] = e;
+}
+
+// One warp per sorted row r < offsets[E]: xs[r] = f16(x[t] * 2^-e), t the
+// row's token and e = texp[t]; xexp[r] = 2^e.
+__global__ void __launch_bounds__(256)
+    pack_x_sorted_kernel(const uint16_t* __restrict__ x, int P, int K, int topk,
+                         const int32_t* __restrict__ sorted_pair_ids, const int32_t* __restrict__ kept_rows,
+                         const int32_t* __restrict__ texp, uint16_t* __restrict__ xs, float* __restrict__ xexp) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= P || row >= *kept_rows) return;
+  const int t = sorted_pair_ids[row] / topk;
+  const int e = texp[t];
   const float mul = exp2i(-e);
+  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * K);
   uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)row * K);
   for (int i = lane; i < K / 8; i += 32) {
     const uint4 v = src[i];
@@ -731,11 +745,14 @@ cudaError_t launch_tc_impl(const TcArgs& a, const CUtensorMap& b0, const CUtenso
 
 uint64_t al256(uint64_t v) { return (v + 255) & ~uint64_t(255); }
 
-// Workspace regions, in this order: gate+up [xs | xexp | weight maps], then
-// down [act hi | act lo | aexp | weight maps].
+// Workspace regions, in this order: gate+up [xs | xexp | texp | weight maps],
+// then down [act hi | act lo | aexp | weight maps].  texp holds one exponent
+// per token; it is sized by the pairs (tokens <= pairs), which is all the
+// gate+up part's size may depend on.
 struct WsLayout {
   uint16_t* xs;
   float* xexp;
+  int32_t* texp;
   CUtensorMap* maps_gu;
   uint16_t* act_hi;
   uint16_t* act_lo;
@@ -748,6 +765,8 @@ WsLayout ws_layout(void* ws, uint64_t pairs, uint64_t hidden, uint64_t inter) {
   l.xs = reinterpret_cast<uint16_t*>(p);
   p += al256(pairs * hidden * 2);
   l.xexp = reinterpret_cast<float*>(p);
+  p += al256(pairs * 4);
+  l.texp = reinterpret_cast<int32_t*>(p);
   p += al256(pairs * 4);
   l.maps_gu = reinterpret_cast<CUtensorMap*>(p);
   p += kMapBytes;
@@ -764,7 +783,7 @@ WsLayout ws_layout(void* ws, uint64_t pairs, uint64_t hidden, uint64_t inter) {
 }  // namespace
 
 size_t tc_gate_up_workspace_bytes(uint64_t pairs, uint64_t hidden) {
-  return al256(pairs * hidden * 2) + al256(pairs * 4) + kMapBytes;
+  return al256(pairs * hidden * 2) + 2 * al256(pairs * 4) + kMapBytes;
 }
 
 size_t tc_workspace_bytes(uint64_t tokens, uint64_t topk, uint64_t hidden, uint64_t inter) {
@@ -811,9 +830,12 @@ cudaError_t launch_tc(int mode, int nt, const GroupedArgs& g, void* workspace, u
   const uint32_t box_rows = pair ? (uint32_t)nt / 2 : (uint32_t)nt;
 
   if (mode == kModeGateUp) {
+    err = launch_pdl(token_exp_kernel, dim3((unsigned)((tokens + 7) / 8)), dim3(256), 0, stream,
+                     static_cast<const uint16_t*>(g.src), (int)tokens, (int)g.K, w.texp);
+    if (err != cudaSuccess) return err;
     err = launch_pdl(pack_x_sorted_kernel, dim3((unsigned)((pairs + 7) / 8)), dim3(256), 0, stream,
                      static_cast<const uint16_t*>(g.src), (int)pairs, (int)g.K, (int)g.topk, g.sorted_pair_ids,
-                     g.offsets + g.num_experts, w.xs, w.xexp);
+                     g.offsets + g.num_experts, w.texp, w.xs, w.xexp);
     if (err != cudaSuccess) return err;
     err = launch_pdl(build_weight_maps_kernel, dim3(g.num_experts), dim3(128), 0, stream, t_nib, t_scale,
                      g.packed0, g.scale0, g.packed1, g.scale1, 4, w.maps_gu);
@@ -832,9 +854,12 @@ cudaError_t launch_tc(int mode, int nt, const GroupedArgs& g, void* workspace, u
   }
   if (mode == kModeUpAct) {
     // x packed as for gate+up; one weight table, two row halves per CTA.
+    err = launch_pdl(token_exp_kernel, dim3((unsigned)((tokens + 7) / 8)), dim3(256), 0, stream,
+                     static_cast<const uint16_t*>(g.src), (int)tokens, (int)g.K, w.texp);
+    if (err != cudaSuccess) return err;
     err = launch_pdl(pack_x_sorted_kernel, dim3((unsigned)((pairs + 7) / 8)), dim3(256), 0, stream,
                      static_cast<const uint16_t*>(g.src), (int)pairs, (int)g.K, (int)g.topk, g.sorted_pair_ids,
-                     g.offsets + g.num_experts, w.xs, w.xexp);
+                     g.offsets + g.num_experts, w.texp, w.xs, w.xexp);
     if (err != cudaSuccess) return err;
     err = launch_pdl(build_weight_maps_kernel, dim3(g.num_experts), dim3(128), 0, stream, t_nib, t_scale,
                      g.packed0, g.scale0, g.packed0, g.scale0, 2, w.maps_gu);
