@@ -117,6 +117,8 @@ def parse_args(argv=None):
     ap.add_argument("--split", type=int, default=0)
     ap.add_argument("--tiles", type=int, default=0)
     ap.add_argument("--depth", type=int, default=0)
+    ap.add_argument("--staging", type=int, default=0,
+                    help="decode path: 1 whole-K activation staging, 2 two-chunk ring, 0 auto")
     ap.add_argument("--no-workspace", action="store_true",
                     help="use the calls without workspace (decode path only)")
     ap.add_argument("--replicas", type=int, default=0,
@@ -486,7 +488,8 @@ def _overrides(args):
 
 
 def _opts(args):
-    return dict(path=args.path, split=args.split, tiles=args.tiles, depth=args.depth)
+    return dict(path=args.path, split=args.split, tiles=args.tiles, depth=args.depth,
+                staging=args.staging)
 
 
 def _tc_path(args, cfg, pairs, experts):

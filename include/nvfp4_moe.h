@@ -105,14 +105,21 @@ typedef struct {
  *   tiles    decode path: 8-row token tiles per pass over an expert, 1, 2 or 4
  *            (gate+up) / 1 or 2 (down); 4 takes depth = 2.
  *   depth    decode path: weight chunks each warp keeps in flight, 2 or 3.
+ *   staging  decode path: how a pass holds its token rows in shared memory.
+ *            1: every 256-wide K chunk is converted up front, then the
+ *            weights stream with no CTA-wide step (needs K/256 x 4 KB per
+ *            8-row tile, twice that for down, within 200 KB); 2: a two-chunk
+ *            ring refilled chunk by chunk.  Automatic: 1 when it fits in 72 KB.
  * Every choice computes the same function; it affects speed and the FP32
- * summation order only.
+ * summation order only.  A choice the shapes do not allow returns
+ * NVFP4_MOE_EINVAL.
  */
 typedef struct {
   int32_t path;
   int32_t split;
   int32_t tiles;
   int32_t depth;
+  int32_t staging;
 } nvfp4_moe_launch_opts;
 
 /*

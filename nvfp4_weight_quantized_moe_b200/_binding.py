@@ -39,7 +39,7 @@ class ExpertTables(ctypes.Structure):
 class LaunchOpts(ctypes.Structure):
     """nvfp4_moe_launch_opts."""
     _fields_ = [("path", ctypes.c_int32), ("split", ctypes.c_int32), ("tiles", ctypes.c_int32),
-                ("depth", ctypes.c_int32)]
+                ("depth", ctypes.c_int32), ("staging", ctypes.c_int32)]
 
 
 class Buffers(ctypes.Structure):
@@ -153,10 +153,10 @@ def _stream(stream) -> Optional[int]:
     return int(stream)
 
 
-def _opts(path=0, split=0, tiles=0, depth=0):
-    if not (path or split or tiles or depth):
+def _opts(path=0, split=0, tiles=0, depth=0, staging=0):
+    if not (path or split or tiles or depth or staging):
         return None
-    return ctypes.byref(LaunchOpts(path, split, tiles, depth))
+    return ctypes.byref(LaunchOpts(path, split, tiles, depth, staging))
 
 
 def active_cap(num_experts: int, num_pairs: int) -> int:
@@ -178,7 +178,7 @@ def route_sort(topk_ids, num_experts, expert_offsets, sorted_pair_ids, pair_pos,
 
 def gate_up_silu(x, gate: ExpertTables, up: ExpertTables, act, expert_offsets, sorted_pair_ids,
                  active_experts, active_count, n_inter, k_hidden, cap, num_tokens, topk,
-                 path=0, split=0, tiles=0, depth=0, stream=None) -> None:
+                 path=0, split=0, tiles=0, depth=0, staging=0, stream=None) -> None:
     if x.dtype not in (torch.bfloat16, torch.uint16, torch.int16):
         raise TypeError("x: expected bf16 (or its uint16 bits)")
     _check("nvfp4_moe_gate_up_silu_ex", _lib.nvfp4_moe_gate_up_silu_ex(
@@ -187,19 +187,19 @@ def gate_up_silu(x, gate: ExpertTables, up: ExpertTables, act, expert_offsets, s
         _ptr(sorted_pair_ids, torch.int32, "sorted_pair_ids"),
         _ptr(active_experts, torch.int32, "active_experts"),
         _ptr(active_count, torch.int32, "active_count"),
-        n_inter, k_hidden, cap, num_tokens, topk, _opts(path, split, tiles, depth),
+        n_inter, k_hidden, cap, num_tokens, topk, _opts(path, split, tiles, depth, staging),
         _stream(stream)))
 
 
 def down(act, down_w: ExpertTables, y, expert_offsets, active_experts, active_count,
-         n_hidden, k_inter, cap, num_tokens, topk, path=0, split=0, tiles=0, depth=0,
+         n_hidden, k_inter, cap, num_tokens, topk, path=0, split=0, tiles=0, depth=0, staging=0,
          stream=None) -> None:
     _check("nvfp4_moe_down_ex", _lib.nvfp4_moe_down_ex(
         _ptr(act, torch.float32, "act"), down_w, _ptr(y, torch.float32, "y"),
         _ptr(expert_offsets, torch.int32, "expert_offsets"),
         _ptr(active_experts, torch.int32, "active_experts"),
         _ptr(active_count, torch.int32, "active_count"),
-        n_hidden, k_inter, cap, num_tokens, topk, _opts(path, split, tiles, depth),
+        n_hidden, k_inter, cap, num_tokens, topk, _opts(path, split, tiles, depth, staging),
         _stream(stream)))
 
 
@@ -350,7 +350,7 @@ def _ws(workspace):
 
 def gate_up_silu_ws(x, gate: ExpertTables, up: ExpertTables, act, expert_offsets, sorted_pair_ids,
                     active_experts, active_count, n_inter, k_hidden, cap, num_tokens, topk,
-                    num_experts, workspace, path=0, split=0, tiles=0, depth=0, stream=None) -> None:
+                    num_experts, workspace, path=0, split=0, tiles=0, depth=0, staging=0, stream=None) -> None:
     if x.dtype not in (torch.bfloat16, torch.uint16, torch.int16):
         raise TypeError("x: expected bf16 (or its uint16 bits)")
     wp, wn = _ws(workspace)
@@ -361,11 +361,11 @@ def gate_up_silu_ws(x, gate: ExpertTables, up: ExpertTables, act, expert_offsets
         _ptr(active_experts, torch.int32, "active_experts"),
         _ptr(active_count, torch.int32, "active_count"),
         n_inter, k_hidden, cap, num_tokens, topk, num_experts,
-        _opts(path, split, tiles, depth), wp, wn, _stream(stream)))
+        _opts(path, split, tiles, depth, staging), wp, wn, _stream(stream)))
 
 
 def down_ws(act, down_w: ExpertTables, y, expert_offsets, active_experts, active_count, n_hidden,
-            k_inter, cap, num_tokens, topk, num_experts, workspace, path=0, split=0, tiles=0, depth=0,
+            k_inter, cap, num_tokens, topk, num_experts, workspace, path=0, split=0, tiles=0, depth=0, staging=0,
             stream=None) -> None:
     wp, wn = _ws(workspace)
     _check("nvfp4_moe_down_ws", _lib.nvfp4_moe_down_ws(
@@ -374,12 +374,12 @@ def down_ws(act, down_w: ExpertTables, y, expert_offsets, active_experts, active
         _ptr(active_experts, torch.int32, "active_experts"),
         _ptr(active_count, torch.int32, "active_count"),
         n_hidden, k_inter, cap, num_tokens, topk, num_experts,
-        _opts(path, split, tiles, depth), wp, wn, _stream(stream)))
+        _opts(path, split, tiles, depth, staging), wp, wn, _stream(stream)))
 
 
 def forward(x, topk_ids, topk_weights, gate: ExpertTables, up: ExpertTables, down: ExpertTables,
             buffers: Buffers, num_experts, hidden, inter, workspace=None, path=0, split=0, tiles=0,
-            depth=0, stream=None) -> None:
+            depth=0, staging=0, stream=None) -> None:
     """nvfp4_moe_forward: the four steps of one layer in one library call.
     ``buffers`` is a :class:`Buffers` of device pointers (see ``MoEBuffers.c_buffers``)."""
     if x.dtype not in (torch.bfloat16, torch.uint16, torch.int16):
@@ -389,7 +389,7 @@ def forward(x, topk_ids, topk_weights, gate: ExpertTables, up: ExpertTables, dow
     _check("nvfp4_moe_forward", _lib.nvfp4_moe_forward(
         _ptr(x, None, "x"), _ptr(topk_ids, torch.int32, "topk_ids"),
         _ptr(topk_weights, torch.float32, "topk_weights"), gate, up, down, ctypes.byref(buffers),
-        m, k, num_experts, hidden, inter, _opts(path, split, tiles, depth), wp, wn, _stream(stream)))
+        m, k, num_experts, hidden, inter, _opts(path, split, tiles, depth, staging), wp, wn, _stream(stream)))
 
 
 def _activation(activation) -> int:
@@ -399,7 +399,7 @@ def _activation(activation) -> int:
 
 
 def up_act(x, up: ExpertTables, act, expert_offsets, sorted_pair_ids, active_experts, active_count,
-           n_inter, k_hidden, cap, num_tokens, topk, activation, path=0, split=0, tiles=0, depth=0,
+           n_inter, k_hidden, cap, num_tokens, topk, activation, path=0, split=0, tiles=0, depth=0, staging=0,
            stream=None) -> None:
     """nvfp4_moe_up_act: act = f(x Wu^T) by sorted position (non-gated experts)."""
     if x.dtype not in (torch.bfloat16, torch.uint16, torch.int16):
@@ -411,12 +411,12 @@ def up_act(x, up: ExpertTables, act, expert_offsets, sorted_pair_ids, active_exp
         _ptr(active_experts, torch.int32, "active_experts"),
         _ptr(active_count, torch.int32, "active_count"),
         n_inter, k_hidden, cap, num_tokens, topk, _activation(activation),
-        _opts(path, split, tiles, depth), _stream(stream)))
+        _opts(path, split, tiles, depth, staging), _stream(stream)))
 
 
 def up_act_ws(x, up: ExpertTables, act, expert_offsets, sorted_pair_ids, active_experts,
               active_count, n_inter, k_hidden, cap, num_tokens, topk, num_experts, activation,
-              workspace, path=0, split=0, tiles=0, depth=0, stream=None) -> None:
+              workspace, path=0, split=0, tiles=0, depth=0, staging=0, stream=None) -> None:
     """nvfp4_moe_up_act_ws: nvfp4_moe_up_act with a workspace (tcgen05 path)."""
     if x.dtype not in (torch.bfloat16, torch.uint16, torch.int16):
         raise TypeError("x: expected bf16 (or its uint16 bits)")
@@ -428,12 +428,12 @@ def up_act_ws(x, up: ExpertTables, act, expert_offsets, sorted_pair_ids, active_
         _ptr(active_experts, torch.int32, "active_experts"),
         _ptr(active_count, torch.int32, "active_count"),
         n_inter, k_hidden, cap, num_tokens, topk, num_experts, _activation(activation),
-        _opts(path, split, tiles, depth), wp, wn, _stream(stream)))
+        _opts(path, split, tiles, depth, staging), wp, wn, _stream(stream)))
 
 
 def forward_nongated(x, topk_ids, topk_weights, up: ExpertTables, down: ExpertTables,
                      buffers: Buffers, num_experts, hidden, inter, activation, workspace=None,
-                     path=0, split=0, tiles=0, depth=0, stream=None) -> None:
+                     path=0, split=0, tiles=0, depth=0, staging=0, stream=None) -> None:
     """nvfp4_moe_forward_nongated: the four steps of a layer of non-gated experts."""
     if x.dtype not in (torch.bfloat16, torch.uint16, torch.int16):
         raise TypeError("x: expected bf16 (or its uint16 bits)")
@@ -442,5 +442,5 @@ def forward_nongated(x, topk_ids, topk_weights, up: ExpertTables, down: ExpertTa
     _check("nvfp4_moe_forward_nongated", _lib.nvfp4_moe_forward_nongated(
         _ptr(x, None, "x"), _ptr(topk_ids, torch.int32, "topk_ids"),
         _ptr(topk_weights, torch.float32, "topk_weights"), up, down, ctypes.byref(buffers),
-        m, k, num_experts, hidden, inter, _activation(activation), _opts(path, split, tiles, depth),
+        m, k, num_experts, hidden, inter, _activation(activation), _opts(path, split, tiles, depth, staging),
         wp, wn, _stream(stream)))

@@ -42,7 +42,7 @@ constexpr int kSmsEstimate = 148;
 // mean.  With one tile, the CTA's warps split K when the grid would otherwise
 // leave SMs short of weight streams.
 DecodePlan plan_decode(int mode, uint64_t tokens, uint64_t pairs, uint32_t num_experts,
-                       uint32_t cap, uint32_t n, const nvfp4_moe_launch_opts* o) {
+                       uint32_t cap, uint32_t n, uint32_t k, const nvfp4_moe_launch_opts* o) {
   DecodePlan p{};
   const uint64_t max_rows = tokens < pairs ? tokens : pairs;
   const uint64_t mean = (pairs + num_experts - 1) / num_experts;
@@ -66,7 +66,17 @@ DecodePlan plan_decode(int mode, uint64_t tokens, uint64_t pairs, uint32_t num_e
   if (o && o->split) p.split = o->split;
   p.depth = 2;
   if (o && o->depth) p.depth = o->depth;
+  // Whole-K staging when the token rows of a pass fit in shared memory next to
+  // three CTAs per SM; the ring otherwise.
+  p.xres = grouped_xres_smem(mode, p, k) <= kDecodeXresAuto ? 1 : 0;
+  if (o && o->staging) p.xres = o->staging == 1 ? 1 : o->staging == 2 ? 0 : -1;
   return p;
+}
+
+// A plan the decode kernels have an instance for and whose staging fits.
+bool plan_ok(int mode, const DecodePlan& p, uint32_t k) {
+  if (p.xres < 0 || !grouped_plan_supported(mode, p)) return false;
+  return !p.xres || grouped_xres_smem(mode, p, k) <= kDecodeSmemMax;
 }
 
 }  // namespace
@@ -126,8 +136,9 @@ int nvfp4_moe_gate_up_silu_ex(const uint16_t* x, nvfp4_expert_tables gate,
     return NVFP4_MOE_EINVAL;
   const int path = opts ? opts->path : 0;
   if (path != 0 && path != 1) return NVFP4_MOE_EINVAL;
-  const DecodePlan plan = plan_decode(kModeGateUp, num_tokens, pairs, cap, cap, n_inter, opts);
-  if (!grouped_plan_supported(kModeGateUp, plan)) return NVFP4_MOE_EINVAL;
+  const DecodePlan plan =
+      plan_decode(kModeGateUp, num_tokens, pairs, cap, cap, n_inter, k_hidden, opts);
+  if (!plan_ok(kModeGateUp, plan, k_hidden)) return NVFP4_MOE_EINVAL;
   GroupedArgs a{};
   a.src = x;
   a.packed0 = gate.packed_ptrs;
@@ -175,8 +186,9 @@ int nvfp4_moe_down_ex(const float* act, nvfp4_expert_tables down, float* y,
     return NVFP4_MOE_EINVAL;
   const int path = opts ? opts->path : 0;
   if (path != 0 && path != 1) return NVFP4_MOE_EINVAL;
-  const DecodePlan plan = plan_decode(kModeDown, num_tokens, pairs, cap, cap, n_hidden, opts);
-  if (!grouped_plan_supported(kModeDown, plan)) return NVFP4_MOE_EINVAL;
+  const DecodePlan plan =
+      plan_decode(kModeDown, num_tokens, pairs, cap, cap, n_hidden, k_inter, opts);
+  if (!plan_ok(kModeDown, plan, k_inter)) return NVFP4_MOE_EINVAL;
   GroupedArgs a{};
   a.src = act;
   a.packed0 = down.packed_ptrs;
@@ -343,8 +355,9 @@ int nvfp4_moe_up_act(const uint16_t* x, nvfp4_expert_tables up, float* act,
     return NVFP4_MOE_EINVAL;
   const int path = opts ? opts->path : 0;
   if (path != 0 && path != 1) return NVFP4_MOE_EINVAL;
-  const DecodePlan plan = plan_decode(kModeUpAct, num_tokens, pairs, cap, cap, n_inter, opts);
-  if (!grouped_plan_supported(kModeUpAct, plan)) return NVFP4_MOE_EINVAL;
+  const DecodePlan plan =
+      plan_decode(kModeUpAct, num_tokens, pairs, cap, cap, n_inter, k_hidden, opts);
+  if (!plan_ok(kModeUpAct, plan, k_hidden)) return NVFP4_MOE_EINVAL;
   GroupedArgs a{};
   a.src = x;
   a.packed0 = up.packed_ptrs;

@@ -7,6 +7,7 @@
 #include <cuda_bf16.h>
 
 #define NVM_DEV __device__ __forceinline__
+#define NVM_HD __host__ __device__ __forceinline__
 
 namespace nvm {
 

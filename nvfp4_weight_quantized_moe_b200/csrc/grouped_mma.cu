@@ -39,11 +39,19 @@
 // Pipeline.  A CTA (4 warps) owns 64 (gate+up) or 128 (down, up+activation) output rows of one
 // expert over all of K; with S > 1 its warps split K S ways over 64/S or 128/S
 // rows and add their sums through shared memory at the end (one row per
-// expert needs that parallelism).  Per 256-k chunk, the activation rows of the
-// group are copied raw with cp.async two chunks ahead into a ring that only the
-// copying lane reads back, converted one chunk ahead into the MMA layout, and
-// consumed after one CTA barrier; the weights run DEPTH chunks ahead in
-// registers.  No load is waited on in the same iteration that issues it.
+// expert needs that parallelism).  The weights run DEPTH chunks ahead in
+// registers.  The activation rows of a group are staged in one of two ways
+// (same arithmetic, same result):
+//   * whole K, when every 256-k chunk of the group fits in shared memory (K/256
+//     x 4 KB per 8-row tile, twice that for down's hi and lo planes): the warps
+//     load all (chunk, row) pieces at once, convert them into the MMA layout,
+//     meet at one CTA barrier, and then each warp runs over its own chunks
+//     with nothing to wait for but its weight loads;
+//   * a ring otherwise: per 256-k chunk the rows are copied raw with cp.async
+//     two chunks ahead into a ring that only the copying lane reads back,
+//     converted one chunk ahead into the MMA layout, and consumed after one
+//     CTA barrier per chunk.
+// No load is waited on in the same iteration that issues it.
 
 #include "common.cuh"
 #include "kernels.h"
@@ -74,7 +82,23 @@ struct Cfg {
   static constexpr int OFF_ROWSRC = OFF_XMUL + 2 * ITEMS * 4;
   static constexpr int OFF_RED = OFF_ROWSRC + GROUP * 4;
   static constexpr int SMEM = OFF_RED + RED_BYTES;
+  // Whole-K staging: every 256-k chunk of the group's rows in MMA layout.
+  static constexpr int XCH_BYTES = PLANES * TILES * kTileChunkBytes;  // one chunk
 };
+
+// Shared-memory layout of whole-K staging for K / 256 = nch chunks: fragments,
+// per-(chunk, row) scale factors, row sources, split-K sums.
+struct XresLayout {
+  int xmul, rowsrc, red, total;
+};
+NVM_HD XresLayout xres_layout(int planes, int split, int tiles, int nch) {
+  XresLayout l;
+  l.xmul = nch * planes * tiles * kTileChunkBytes;
+  l.rowsrc = l.xmul + nch * 8 * tiles * 4;
+  l.red = (l.rowsrc + 8 * tiles * 4 + 15) & ~15;
+  l.total = l.red + (split > 1 ? 128 * 2 * tiles * 4 * 4 : 0);
+  return l;
+}
 
 // Byte offset of the 8-byte unit holding k = 64c + 4j .. +3 of token `r` (0..7)
 // inside one token tile's chunk (u = 16c + j).
@@ -99,17 +123,89 @@ NVM_DEV void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// One (row, 256-k chunk) of the activation operand, as the warp holds it (lane
+// l: bytes [16 l, 16 l + 16) of each 512-byte half), scaled by 2^-e into the
+// f16 range and stored in the MMA layout: `dst` is the row's token tile in the
+// chunk, `lo_off` the offset of the lo plane (down), `xm` the row's 2^e slot.
+template <int MODE>
+NVM_DEV void stage_piece(const uint4 (&v)[MODE == kModeDown ? 2 : 1], uint8_t* dst, int lo_off,
+                         int r, float* xm, int lane) {
+  float f[8];
+  int u0[2];  // first 4-k unit of each 16-byte piece
+  if (MODE != kModeDown) {
+    const uint32_t wv[4] = {v[0].x, v[0].y, v[0].z, v[0].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = bf16_bits_to_f32(wv[i] & 0xFFFFu);
+      f[2 * i + 1] = bf16_bits_to_f32(wv[i] >> 16);
+    }
+    u0[0] = 2 * lane;  // 8 bf16 = units 2 lane, 2 lane + 1
+    u0[1] = 2 * lane + 1;
+  } else {
+    f[0] = __uint_as_float(v[0].x); f[1] = __uint_as_float(v[0].y);
+    f[2] = __uint_as_float(v[0].z); f[3] = __uint_as_float(v[0].w);
+    f[4] = __uint_as_float(v[1].x); f[5] = __uint_as_float(v[1].y);
+    f[6] = __uint_as_float(v[1].z); f[7] = __uint_as_float(v[1].w);
+    u0[0] = lane;
+    u0[1] = 32 + lane;
+  }
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
+  const int ex = f16_range_exponent(warp_max(m));
+  const float mul = exp2i(-ex);
+  if (MODE != kModeDown) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint2 o;
+      o.x = pack_f16x2(f[4 * h] * mul, f[4 * h + 1] * mul);
+      o.y = pack_f16x2(f[4 * h + 2] * mul, f[4 * h + 3] * mul);
+      *reinterpret_cast<uint2*>(dst + unit_offset(r & 7, u0[h])) = o;
+    }
+  } else {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float hv[4], lv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float sv = f[4 * h + i] * mul;
+        hv[i] = __half2float(__float2half_rn(sv));
+        lv[i] = sv - hv[i];
+      }
+      uint2 oh, ol;
+      oh.x = pack_f16x2(hv[0], hv[1]);
+      oh.y = pack_f16x2(hv[2], hv[3]);
+      ol.x = pack_f16x2(lv[0], lv[1]);
+      ol.y = pack_f16x2(lv[2], lv[3]);
+      const int off = unit_offset(r & 7, u0[h]);
+      *reinterpret_cast<uint2*>(dst + off) = oh;
+      *reinterpret_cast<uint2*>(dst + lo_off + off) = ol;
+    }
+  }
+  if (lane == 0) *xm = exp2i(ex);
+}
+
 }  // namespace
 
-template <int MODE, int S, int TILES, int DEPTH>
-__global__ void __launch_bounds__(128) grouped_mma_kernel(GroupedArgs a) {
+// One-tile, depth-2 instances (one token row per expert: many CTAs, all of
+// which should be resident at once) are held to three CTAs per SM, 168
+// registers; the whole-K form would otherwise take more for its longer-lived
+// weight buffers.
+template <int MODE, int S, int TILES, int DEPTH, bool XR>
+__global__ void __launch_bounds__(128, (TILES == 1 && DEPTH == 2) ? 3 : 1)
+    grouped_mma_kernel(GroupedArgs a) {
   using C = Cfg<MODE, S, TILES>;
   extern __shared__ __align__(16) uint8_t smem[];
+  const int nch = (int)a.K >> 8;
+  const XresLayout xl = xres_layout(C::PLANES, S, TILES, nch);
+  static_assert(C::XCH_BYTES == C::PLANES * TILES * kTileChunkBytes &&
+                    C::RED_BYTES == (S > 1 ? 128 * 2 * TILES * 4 * 4 : 0),
+                "whole-K staging layout");
   uint8_t* frag = smem;
   uint8_t* raw = smem + C::OFF_RAW;
-  float* xmul = reinterpret_cast<float*>(smem + C::OFF_XMUL);
-  int* rowsrc = reinterpret_cast<int*>(smem + C::OFF_ROWSRC);
-  float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
+  float* xmul = reinterpret_cast<float*>(smem + (XR ? xl.xmul : C::OFF_XMUL));
+  int* rowsrc = reinterpret_cast<int*>(smem + (XR ? xl.rowsrc : C::OFF_ROWSRC));
+  float* red = reinterpret_cast<float*>(smem + (XR ? xl.red : C::OFF_RED));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int s = warp % S, q = warp / S;
@@ -182,7 +278,6 @@ __global__ void __launch_bounds__(128) grouped_mma_kernel(GroupedArgs a) {
   const float s2a = a.s2_0[e];
   const float s2b = MODE == kModeGateUp ? a.s2_1[e] : s2a;
 
-  const int nch = K >> 8;
   const int my_ch0 = s * nch / S;
   const int my_nch = (s + 1) * nch / S - my_ch0;
   const int iters = (nch + S - 1) / S;
@@ -221,10 +316,10 @@ __global__ void __launch_bounds__(128) grouped_mma_kernel(GroupedArgs a) {
   for (int g0 = row_lo; g0 < row_hi; g0 += C::GROUP) {
     const int nrows = min(C::GROUP, row_hi - g0);
     const int ntiles = (nrows + 7) >> 3;
-    // Split-K CTAs (short K slices) put their first DEPTH weight chunks in
-    // flight before the token rows are looked up; full-K CTAs do it after, which
-    // keeps those registers free during the look-up.
-    if (S > 1 && warp_on) {
+    // Split-K CTAs (short K slices) and whole-K staging put their first DEPTH
+    // weight chunks in flight before the token rows are looked up; full-K ring
+    // CTAs do it after, which keeps those registers free during the look-up.
+    if ((S > 1 || XR) && warp_on) {
 #pragma unroll
       for (int d = 0; d < DEPTH; ++d)
         if (d < my_nch) load_chunk(d, wbuf[d], sbuf[d]);
@@ -257,78 +352,60 @@ __global__ void __launch_bounds__(128) grouped_mma_kernel(GroupedArgs a) {
         const int ss = item / C::GROUP, r = item % C::GROUP;
         const int cnt = (ss + 1) * nch / S - ss * nch / S;
         if (r >= nrows || it >= cnt) continue;
-        const uint8_t* rp = raw + stage * C::RAW_BYTES + item * 256 * C::BPE;
-        uint8_t* dst = frag + buf * C::FRAG_BYTES + (ss * TILES + (r >> 3)) * kTileChunkBytes;
-        float f[8];
-        int u0[C::BPE / 2];  // first 4-k unit of each 16-byte piece
-        if (MODE != kModeDown) {
-          const uint4 v = *reinterpret_cast<const uint4*>(rp + lane * 16);
-          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+        const uint8_t* rp = raw + stage * C::RAW_BYTES + item * 256 * C::BPE + lane * 16;
+        uint4 v[C::PLANES];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            f[2 * i] = bf16_bits_to_f32(wv[i] & 0xFFFFu);
-            f[2 * i + 1] = bf16_bits_to_f32(wv[i] >> 16);
-          }
-          u0[0] = 2 * lane;  // 8 bf16 = units 2 lane, 2 lane + 1
-        } else {
-          const float4 v0 = *reinterpret_cast<const float4*>(rp + lane * 16);
-          const float4 v1 = *reinterpret_cast<const float4*>(rp + 512 + lane * 16);
-          f[0] = v0.x; f[1] = v0.y; f[2] = v0.z; f[3] = v0.w;
-          f[4] = v1.x; f[5] = v1.y; f[6] = v1.z; f[7] = v1.w;
-          u0[0] = lane;
-          u0[1] = 32 + lane;
-        }
-        float m = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
-        const int ex = f16_range_exponent(warp_max(m));
-        const float mul = exp2i(-ex);
-        if (MODE != kModeDown) {
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint2 o;
-            o.x = pack_f16x2(f[4 * h] * mul, f[4 * h + 1] * mul);
-            o.y = pack_f16x2(f[4 * h + 2] * mul, f[4 * h + 3] * mul);
-            *reinterpret_cast<uint2*>(dst + unit_offset(r & 7, u0[0] + h)) = o;
-          }
-        } else {
-          uint8_t* dst_lo = dst + S * TILES * kTileChunkBytes;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            float hv[4], lv[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float sv = f[4 * h + i] * mul;
-              hv[i] = __half2float(__float2half_rn(sv));
-              lv[i] = sv - hv[i];
-            }
-            uint2 oh, ol;
-            oh.x = pack_f16x2(hv[0], hv[1]);
-            oh.y = pack_f16x2(hv[2], hv[3]);
-            ol.x = pack_f16x2(lv[0], lv[1]);
-            ol.y = pack_f16x2(lv[2], lv[3]);
-            const int off = unit_offset(r & 7, u0[h]);
-            *reinterpret_cast<uint2*>(dst + off) = oh;
-            *reinterpret_cast<uint2*>(dst_lo + off) = ol;
-          }
-        }
-        if (lane == 0) xmul[buf * C::ITEMS + item] = exp2i(ex);
+        for (int h = 0; h < C::PLANES; ++h) v[h] = *reinterpret_cast<const uint4*>(rp + h * 512);
+        stage_piece<MODE>(v, frag + buf * C::FRAG_BYTES + (ss * TILES + (r >> 3)) * kTileChunkBytes,
+                          S * TILES * kTileChunkBytes, r, xmul + buf * C::ITEMS + item, lane);
       }
     };
 
-    // ---- prologue: raw chunks 0 and 1 and weights 0..DEPTH-1 in flight ----
-    copy_raw(0, 0);
-    cp_async_commit();
-    if (S == 1 && warp_on) {
+    if (XR) {
+      // ---- whole-K staging: every (chunk, row) of the group is loaded (XU per
+      // warp in flight at once) and converted, then one barrier; the main loop
+      // below then waits on nothing but its own weight loads ----
+      constexpr int XU = MODE == kModeDown ? 2 : 4;
+      const int nitems = nch * nrows;
+      for (int i0 = warp; i0 < nitems; i0 += C::WARPS * XU) {
+        uint4 v[XU][C::PLANES];
 #pragma unroll
-      for (int d = 0; d < DEPTH; ++d)
-        if (d < my_nch) load_chunk(d, wbuf[d], sbuf[d]);
+        for (int u = 0; u < XU; ++u) {
+          const int item = i0 + u * C::WARPS;
+          if (item < nitems) {
+            const int ch = item / nrows, r = item - ch * nrows;
+            const uint8_t* src = static_cast<const uint8_t*>(a.src) +
+                                 ((size_t)rowsrc[r] * K + ((size_t)ch << 8)) * C::BPE + lane * 16;
+#pragma unroll
+            for (int h = 0; h < C::PLANES; ++h) v[u][h] = ld_stream_v4(src + h * 512);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < XU; ++u) {
+          const int item = i0 + u * C::WARPS;
+          if (item < nitems) {
+            const int ch = item / nrows, r = item - ch * nrows;
+            stage_piece<MODE>(v[u], frag + (size_t)ch * C::XCH_BYTES + (r >> 3) * kTileChunkBytes,
+                              TILES * kTileChunkBytes, r, xmul + ch * C::GROUP + r, lane);
+          }
+        }
+      }
+      __syncthreads();
+    } else {
+      // ---- prologue: raw chunks 0 and 1 and weights 0..DEPTH-1 in flight ----
+      copy_raw(0, 0);
+      cp_async_commit();
+      if (S == 1 && warp_on) {
+#pragma unroll
+        for (int d = 0; d < DEPTH; ++d)
+          if (d < my_nch) load_chunk(d, wbuf[d], sbuf[d]);
+      }
+      copy_raw(1, 1);
+      cp_async_commit();
+      cp_async_wait<1>();
+      convert(0, 0, 0);
+      __syncthreads();
     }
-    copy_raw(1, 1);
-    cp_async_commit();
-    cp_async_wait<1>();
-    convert(0, 0, 0);
-    __syncthreads();
 
     float acc[2][TILES][4];
 #pragma unroll
@@ -338,16 +415,21 @@ __global__ void __launch_bounds__(128) grouped_mma_kernel(GroupedArgs a) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[t][u][i] = 0.0f;
 
+    // Whole-K staging has no CTA-wide step per chunk, so each warp runs over
+    // its own chunks only.
+    const int nloop = XR ? (warp_on ? my_nch : 0) : iters;
 #pragma unroll 1
-    for (int base = 0; base < iters; base += DEPTH) {
+    for (int base = 0; base < nloop; base += DEPTH) {
 #pragma unroll
       for (int d = 0; d < DEPTH; ++d) {
         const int it = base + d;
-        if (it < iters) {
+        if (it < nloop) {
           const int buf = it & 1;
-          // Raw chunk it + 2 reuses the stage of chunk it (converted last iteration).
-          copy_raw(it + 2, it & 1);
-          cp_async_commit();
+          if (!XR) {
+            // Raw chunk it + 2 reuses the stage of chunk it (converted last iteration).
+            copy_raw(it + 2, it & 1);
+            cp_async_commit();
+          }
           if (warp_on && it < my_nch) {
             float pacc[2][TILES][4];
 #pragma unroll
@@ -364,7 +446,9 @@ __global__ void __launch_bounds__(128) grouped_mma_kernel(GroupedArgs a) {
 #pragma unroll
               for (int r = 0; r < 2; ++r) e4m3x4_to_f16x2x2(sbuf[d][t][r], scl[t][r][0], scl[t][r][1]);
 
-            const uint8_t* xb = frag + buf * C::FRAG_BYTES + s * TILES * kTileChunkBytes;
+            const uint8_t* xb = XR ? frag + (size_t)(my_ch0 + it) * C::XCH_BYTES
+                                   : frag + buf * C::FRAG_BYTES + s * TILES * kTileChunkBytes;
+            constexpr int kLoOff = (XR ? 1 : S) * TILES * kTileChunkBytes;
 #pragma unroll
             for (int m = 0; m < 8; ++m) {  // word m of each row's 32 bytes: steps j = 2m, 2m+1
               uint32_t dec[2][2][4];
@@ -400,7 +484,7 @@ __global__ void __launch_bounds__(128) grouped_mma_kernel(GroupedArgs a) {
                     mma_f16_16816(pacc[1][u], A[1], b.x, b.y);
                     if (MODE == kModeDown) {
                       const uint2 bl =
-                          *reinterpret_cast<const uint2*>(xt + S * TILES * kTileChunkBytes + boff);
+                          *reinterpret_cast<const uint2*>(xt + kLoOff + boff);
                       mma_f16_16816(pacc[0][u], A[0], bl.x, bl.y);
                       mma_f16_16816(pacc[1][u], A[1], bl.x, bl.y);
                     }
@@ -411,7 +495,7 @@ __global__ void __launch_bounds__(128) grouped_mma_kernel(GroupedArgs a) {
             // The registers of slot d are free again: refill them DEPTH chunks ahead.
             if (it + DEPTH < my_nch) load_chunk(it + DEPTH, wbuf[d], sbuf[d]);
             // Undo the chunk's activation scaling (columns 2c, 2c+1 of each tile).
-            const float* xm = xmul + buf * C::ITEMS + s * C::GROUP;
+            const float* xm = XR ? xmul + (my_ch0 + it) * C::GROUP : xmul + buf * C::ITEMS + s * C::GROUP;
 #pragma unroll
             for (int u = 0; u < TILES; ++u) {
               if (u < ntiles) {
@@ -426,14 +510,16 @@ __global__ void __launch_bounds__(128) grouped_mma_kernel(GroupedArgs a) {
               }
             }
           }
-          // Chunk it + 1: its raw copy was issued two iterations ago.
-          cp_async_wait<1>();
-          if (it + 1 < iters) convert(it + 1, (it + 1) & 1, buf ^ 1);
-          __syncthreads();
+          if (!XR) {
+            // Chunk it + 1: its raw copy was issued two iterations ago.
+            cp_async_wait<1>();
+            if (it + 1 < iters) convert(it + 1, (it + 1) & 1, buf ^ 1);
+            __syncthreads();
+          }
         }
       }
     }
-    cp_async_wait<0>();
+    if (!XR) cp_async_wait<0>();
 
     if (S > 1) {
       // Split-K: warps with s > 0 publish their sums, s == 0 adds them in split order.
@@ -487,21 +573,24 @@ __global__ void __launch_bounds__(128) grouped_mma_kernel(GroupedArgs a) {
   }
 }
 
-template <int MODE, int S, int TILES, int DEPTH>
+template <int MODE, int S, int TILES, int DEPTH, bool XR>
 cudaError_t launch_grouped_impl(const GroupedArgs& a, uint32_t cap, cudaStream_t stream) {
   using C = Cfg<MODE, S, TILES>;
-  auto kern = grouped_mma_kernel<MODE, S, TILES, DEPTH>;
-  cudaError_t err = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::SMEM);
+  auto kern = grouped_mma_kernel<MODE, S, TILES, DEPTH, XR>;
+  const int smem = XR ? xres_layout(C::PLANES, S, TILES, (int)(a.K >> 8)).total : C::SMEM;
+  if (smem > kDecodeSmemMax) return cudaErrorInvalidValue;
+  cudaError_t err = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), smem);
   if (err != cudaSuccess) return err;
   const dim3 grid((a.N + C::ROWS_PER_CTA - 1) / C::ROWS_PER_CTA, cap);
-  return launch_pdl(kern, grid, dim3(C::THREADS), C::SMEM, stream, a);
+  return launch_pdl(kern, grid, dim3(C::THREADS), smem, stream, a);
 }
 
 cudaError_t launch_grouped(int mode, const DecodePlan& p, const GroupedArgs& a, uint32_t cap,
                            cudaStream_t stream) {
-#define NVM_CASE(M, SS, T, D)                                               \
-  if (mode == M && p.split == SS && p.tiles == T && p.depth == D)           \
-    return launch_grouped_impl<M, SS, T, D>(a, cap, stream);
+#define NVM_CASE(M, SS, T, D)                                                       \
+  if (mode == M && p.split == SS && p.tiles == T && p.depth == D)                   \
+    return p.xres ? launch_grouped_impl<M, SS, T, D, true>(a, cap, stream)          \
+                  : launch_grouped_impl<M, SS, T, D, false>(a, cap, stream);
   // One row per expert: K split over the CTA's warps.
   NVM_CASE(kModeGateUp, 4, 1, 2)
   NVM_CASE(kModeGateUp, 2, 1, 2)
@@ -538,6 +627,10 @@ bool grouped_plan_supported(int mode, const DecodePlan& p) {
 
 int grouped_rows_per_cta(int mode, int split) {
   return (4 / split) * (mode == kModeGateUp ? 16 : 32);
+}
+
+int grouped_xres_smem(int mode, const DecodePlan& p, uint32_t k) {
+  return xres_layout(mode == kModeDown ? 2 : 1, p.split, p.tiles, (int)(k >> 8)).total;
 }
 
 }  // namespace nvm

@@ -72,12 +72,19 @@ struct DecodePlan {
   int split;
   int tiles;
   int depth;
+  int xres;  // 1: each pass stages every K chunk of its token rows up front
 };
 
 cudaError_t launch_grouped(int mode, const DecodePlan& plan, const GroupedArgs& a, uint32_t cap,
                            cudaStream_t stream);
 bool grouped_plan_supported(int mode, const DecodePlan& plan);
 int grouped_rows_per_cta(int mode, int split);
+// Dynamic shared memory of whole-K staging for this plan and K.
+int grouped_xres_smem(int mode, const DecodePlan& plan, uint32_t k);
+// Largest dynamic shared memory a decode launch takes; automatic plans stage
+// whole K only up to kDecodeXresAuto (three CTAs per SM).
+constexpr int kDecodeSmemMax = 200 * 1024;
+constexpr int kDecodeXresAuto = 72 * 1024;
 
 // tcgen05 path (grouped_tc.cu): activation packing and per-expert weight
 // tensor maps into `workspace` (256-byte aligned), then the projection kernel

@@ -268,13 +268,13 @@ class NVFP4MoE:
     def forward(self, x: torch.Tensor, topk_ids: torch.Tensor, topk_weights: torch.Tensor,
                 bufs: Optional[MoEBuffers] = None, path: int = 0, split: int = 0,
                 tiles: int = 0, depth: int = 0, workspace: Optional[torch.Tensor] = None,
-                stream=None, steps: bool = False,
+                stream=None, steps: bool = False, staging: int = 0,
                 shared_weights: Optional[torch.Tensor] = None) -> MoEBuffers:
         """Run the four steps on ``stream``; results land in ``bufs`` (returned).
         One library call (nvfp4_moe_forward) by default; ``steps=True`` makes the
         four single-step calls instead (same kernels, same results).
 
-        path / split / tiles / depth are the launch options of the two
+        path / split / tiles / depth / staging are the launch options of the two
         projections (0 = chosen from the shape); see nvfp4_moe_launch_opts.
         With a ``workspace`` (see :meth:`workspace`) the projections may take
         the tcgen05 path.  With a shared expert, the routing is first extended
@@ -287,7 +287,7 @@ class NVFP4MoE:
             raise ValueError("buffers were sized for fewer tokens")
         if self.gate is None:
             return self._forward_nongated(x, topk_ids, topk_weights, bufs, path, split, tiles,
-                                          depth, workspace, stream, steps, shared_weights)
+                                          depth, staging, workspace, stream, steps, shared_weights)
         gate_t, up_t, down_t = self.gate.tables, self.up.tables, self.down.tables
         topk, num_experts = self.topk, self.num_experts
         if self.shared is not None:
@@ -306,14 +306,14 @@ class NVFP4MoE:
         if not steps:
             B.forward(x, topk_ids, topk_weights, gate_t, up_t, down_t, bufs.c_buffers, num_experts,
                       self.hidden, self.inter, workspace=workspace, path=path, split=split,
-                      tiles=tiles, depth=depth, stream=stream)
+                      tiles=tiles, depth=depth, staging=staging, stream=stream)
             return bufs
         p = m * topk
         cap = B.active_cap(num_experts, p)
         B.route_sort(topk_ids, num_experts, bufs.expert_offsets[:num_experts + 1],
                      bufs.sorted_pair_ids, bufs.pair_pos, bufs.active_experts[:num_experts],
                      bufs.active_count, bufs.status, stream=stream)
-        opts = dict(path=path, split=split, tiles=tiles, depth=depth, stream=stream)
+        opts = dict(path=path, split=split, tiles=tiles, depth=depth, staging=staging, stream=stream)
         if workspace is None:
             B.gate_up_silu(x, gate_t, up_t, bufs.act, bufs.expert_offsets, bufs.sorted_pair_ids,
                            bufs.active_experts, bufs.active_count, self.inter, self.hidden, cap, m,
@@ -331,10 +331,11 @@ class NVFP4MoE:
         return bufs
 
     def _forward_nongated(self, x, topk_ids, topk_weights, bufs, path, split, tiles, depth,
-                          workspace, stream, steps, shared_weights) -> MoEBuffers:
+                          staging, workspace, stream, steps, shared_weights) -> MoEBuffers:
         if shared_weights is not None:
             raise ValueError("shared_weights given to a layer without a shared expert")
-        opts = dict(path=path, split=split, tiles=tiles, depth=depth, stream=stream)
+        opts = dict(path=path, split=split, tiles=tiles, depth=depth, staging=staging,
+                    stream=stream)
         if not steps:
             B.forward_nongated(x, topk_ids, topk_weights, self.up.tables, self.down.tables,
                                bufs.c_buffers, self.num_experts, self.hidden, self.inter,

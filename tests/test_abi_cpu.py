@@ -82,6 +82,12 @@ def test_host_validation_rejects_bad_shapes_without_a_gpu(lib):
         bad = B.LaunchOpts(*opts)
         assert L.nvfp4_moe_down_ex(p8, ok_t, p8, p8, p8, p8, 128, 256, 1, 1, 1,
                                    ctypes.byref(bad), None) == 1, opts
+    # staging: unknown choice; whole-K staging past the shared-memory limit
+    # (K = 16384 on two tiles: 64 chunks x 8 KB) is refused before any launch
+    for opts, k in (((1, 0, 0, 0, 3), 256), ((1, 1, 2, 2, 1), 16384)):
+        bad = B.LaunchOpts(*opts)
+        assert L.nvfp4_moe_gate_up_silu_ex(p8, ok_t, ok_t, p8, p8, p8, p8, p8, 64, k, 1, 1, 1,
+                                           ctypes.byref(bad), None) == 1, opts
 
 
 def test_nongated_calls_check_activation_and_shapes_on_the_host(lib):

@@ -250,21 +250,27 @@ SMALL = {
 }
 
 
-# Decode launch shapes: (split, tiles, depth); zeros pick from the shape.
-PLANS = [(0, 0, 0), (4, 1, 2), (2, 1, 2), (1, 1, 2), (1, 1, 3), (1, 2, 2), (1, 2, 3)]
+# Decode launch shapes: (split, tiles, depth, staging); zeros pick from the shape.
+# Staging 1 holds every K chunk of a pass's token rows in shared memory, 2 a
+# two-chunk ring; every forced shape runs both ways.
+PLANS = [(0, 0, 0, 0)] + [(s, t, d, g) for (s, t, d) in
+                          [(4, 1, 2), (2, 1, 2), (1, 1, 2), (1, 1, 3), (1, 2, 2), (1, 2, 3)]
+                          for g in (1, 2)]
 
 
-@pytest.mark.parametrize("plan", PLANS, ids=lambda p: "s%d-t%d-d%d" % p)
+@pytest.mark.parametrize("plan", PLANS, ids=lambda p: "s%d-t%d-d%d-x%d" % p)
 @pytest.mark.parametrize("name", list(SMALL))
 def test_forward_small(name, plan):
     _need_gpu()
     prob = make_problem(SMALL[name])
-    split, tiles, depth = plan
-    _, bufs = _gpu_forward(prob, path=1 if any(plan) else 0, split=split, tiles=tiles, depth=depth)
+    split, tiles, depth, staging = plan
+    _, bufs = _gpu_forward(prob, path=1 if any(plan) else 0, split=split, tiles=tiles, depth=depth,
+                           staging=staging)
     _check_full(prob, bufs)
 
 
-def test_gate_up_four_tiles():
+@pytest.mark.parametrize("staging", [1, 2])
+def test_gate_up_four_tiles(staging):
     """Gate+up holding 32 rows per pass (the 17..32-token shape)."""
     _need_gpu()
     prob = make_problem(SMALL["hot"])
@@ -279,7 +285,8 @@ def test_gate_up_four_tiles():
     cap = nvm.active_cap(cfg.experts, cfg.pairs)
     nvm.gate_up_silu(x, layer.gate.tables, layer.up.tables, bufs.act, bufs.expert_offsets,
                      bufs.sorted_pair_ids, bufs.active_experts, bufs.active_count, cfg.inter,
-                     cfg.hidden, cap, cfg.tokens, cfg.topk, path=1, split=1, tiles=4, depth=2)
+                     cfg.hidden, cap, cfg.tokens, cfg.topk, path=1, split=1, tiles=4, depth=2,
+                     staging=staging)
     torch.cuda.synchronize()
     ref = orc.moe_forward(prob.x_bf16, prob.topk_ids, prob.topk_weights, cfg.experts, *_fns(prob),
                           hidden=cfg.hidden, inter=cfg.inter)
@@ -638,7 +645,10 @@ def _gpu_forward_nongated(prob, activation, ws=False, null=(), **opts):
 
 
 # (path options): decode kernel automatic and forced shapes; tcgen05 16- and 128-row passes.
-NONGATED_PATHS = [dict(), dict(path=1, split=4, tiles=1, depth=2), dict(path=1, split=1, tiles=2, depth=3),
+NONGATED_PATHS = [dict(), dict(path=1, split=4, tiles=1, depth=2, staging=1),
+                  dict(path=1, split=4, tiles=1, depth=2, staging=2),
+                  dict(path=1, split=1, tiles=2, depth=3, staging=1),
+                  dict(path=1, split=1, tiles=2, depth=3, staging=2),
                   dict(ws=True, path=2, tiles=2), dict(ws=True, path=2, tiles=16),
                   dict(ws=True, path=2, tiles=4), dict(ws=True, path=2, tiles=24),
                   dict(ws=True, path=2, tiles=32)]
