@@ -63,11 +63,11 @@ KERNEL_SOURCES = {
 # kernel, with the hash of that kernel's sources when it was captured.  An
 # entry whose hash no longer matches the sources is stale and not reported.
 NCU_TRAFFIC_BYTES = {
-    ("decode_m1", "mma.sync"): (28357376, "b043af2a146a"),       # 28.36 MB read, 0 written
-    ("decode_m32", "tcgen05"): (299103232, "ba425bfe1e4c"),      # 293.13 MB read, 5.97 MB written
+    ("decode_m1", "mma.sync"): (28362496, "75ef290dff45"),       # 28.36 MB read, 0.002 MB written
+    ("decode_m32", "tcgen05"): (297943296, "18e52bb5eee3"),      # 293.13 MB read, 4.82 MB written
     # reduced case (64 experts, 64 tokens: the same 8 rows per expert) x 4 experts
-    ("decode_m256", "tcgen05"): (4519915520, "ba425bfe1e4c"),    # 4 x (1122.36 + 7.62) MB
-    ("prefill_m8192", "tcgen05"): (2114844000, "ba425bfe1e4c"),  # 1.7252 GB read, 0.3896 GB written
+    ("decode_m256", "tcgen05"): (4518880256, "18e52bb5eee3"),    # 4 x (1122.32 + 7.40) MB
+    ("prefill_m8192", "tcgen05"): (3190343424, "18e52bb5eee3"),  # 2.8000 GB read, 0.3903 GB written
 }
 
 
