@@ -69,6 +69,11 @@ NCU_TRAFFIC_BYTES = {
     ("decode_m256", "tcgen05"): (4518880256, "18e52bb5eee3"),    # 4 x (1122.32 + 7.40) MB
     ("prefill_m8192", "tcgen05"): (3190343424, "18e52bb5eee3"),  # 2.8000 GB read, 0.3903 GB written
 }
+# Entries not captured on the workload itself: how the figure was obtained.
+NCU_TRAFFIC_SCALED = {
+    ("decode_m256", "tcgen05"): "4 x one launch of a 64-expert, 64-token case of the same "
+                                "per-expert shape (the full workload is too large to capture)",
+}
 
 
 # The same for one launch of a load-time op's kernel (per projection for the
@@ -401,6 +406,17 @@ def run_ours(args, rank, world, local):
     torch.cuda.synchronize(dev)
     gu_ms = ev0.elapsed_time(ev1) / (reps * len(layers))
     gu_bytes = 2 * (active + (1 if args.shared else 0)) * per_expert
+    # Stored traffic describes the default launch of the captured workload only.
+    default_launch = not _overrides(args) and not args.shared and not any(
+        v for k, v in _opts(args).items())
+
+    def traffic(kernel):
+        t = ncu_traffic(cfg.name, kernel) if default_launch else None
+        out = {"traffic": t, "traffic_source_hash": kernel_source_hash(kernel)}
+        if t is not None and (cfg.name, kernel) in NCU_TRAFFIC_SCALED:
+            out["traffic_scaled"] = NCU_TRAFFIC_SCALED[(cfg.name, kernel)]
+        return out
+
     gu_flops = 2.0 * 2 * pairs_run * cfg.hidden * cfg.inter
     rows = _tc_rows(args, cfg.tokens, pairs_run, experts_run) if tc else 0
     if prefill:
@@ -409,17 +425,14 @@ def run_ours(args, rank, world, local):
                     "achieved": achieved, "peak": tflops, "unit": "TFLOP/s",
                     "frac": achieved / tflops, "peak_source": f"{peak_kind} bf16 burst",
                     "algorithmic_flops_per_launch": gu_flops, "launch_ms": gu_ms,
-                    "traffic": ncu_traffic(cfg.name, "tcgen05"),
-                    "traffic_source_hash": kernel_source_hash("tcgen05")}
+                    **traffic("tcgen05")}
     else:
         achieved = gu_bytes / (gu_ms * 1e-3) / 1e9
         roofline = {"kernel": f"nvfp4_moe_gate_up_silu_ws ({_tc_kernel_name(rows)})" if tc else
                     "nvfp4_moe_gate_up_silu (register-fed mma.sync)", "bound": "hbm",
                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                     "peak_source": f"{peak_kind} HBM copy", "algorithmic_bytes_per_launch": gu_bytes,
-                    "launch_ms": gu_ms,
-                    "traffic": ncu_traffic(cfg.name, "tcgen05" if tc else "mma.sync"),
-                    "traffic_source_hash": kernel_source_hash("tcgen05" if tc else "mma.sync")}
+                    "launch_ms": gu_ms, **traffic("tcgen05" if tc else "mma.sync")}
 
     e2e = None if args.no_e2e else run_e2e(layers, prob, bufs, ws, dev, stream, steps, warmup, args, world)
 

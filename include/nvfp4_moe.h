@@ -252,14 +252,15 @@ NVFP4_MOE_API int nvfp4_moe_down_ws(
  * workspace.  The packed token rows go to a fixed scratch array inside the
  * library: 8 MiB of device memory on every GPU that loads the library, held
  * until the process exits.  Requests needing more than that (P * k_hidden * 2
- * bytes plus P * 4, each rounded up to 256, plus 512 KiB of tensor maps,
- * P = num_tokens * topk) return NVFP4_MOE_ESHAPE before anything is launched; so do widths the
- * tcgen05 path does not take (n_inter % 128, k_hidden % 256).  The call never
- * allocates memory.  Its first call on a device looks the scratch array's
- * device address up (cudaGetSymbolAddress) with that device current; make
- * that first call before any stream capture.  The address is kept for the
- * life of the process: after cudaDeviceReset of a device, do not call this
- * entry point on that device again.  All calls share the one array
+ * bytes of rows, plus two arrays of P * 4 bytes for the row and token scale
+ * exponents, each rounded up to 256, plus 512 KiB of tensor maps, P =
+ * num_tokens * topk) return NVFP4_MOE_ESHAPE before anything is launched; so
+ * do widths the tcgen05 path does not take (n_inter % 128, k_hidden % 256).
+ * The call never allocates memory.  Its first call on a device looks the
+ * scratch array's device address up (cudaGetSymbolAddress) with that device
+ * current; make that first call before any stream capture.  The address is
+ * kept for the life of the process: after cudaDeviceReset of a device, do not
+ * call this entry point on that device again.  All calls share the one array
  * and each call leaves its packed rows there: calls whose kernels overlap on
  * the GPU (different streams, or different host threads) race on it.
  */
