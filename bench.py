@@ -64,10 +64,10 @@ KERNEL_SOURCES = {
 # entry whose hash no longer matches the sources is stale and not reported.
 NCU_TRAFFIC_BYTES = {
     ("decode_m1", "mma.sync"): (28362496, "75ef290dff45"),       # 28.36 MB read, 0.002 MB written
-    ("decode_m32", "tcgen05"): (297943296, "18e52bb5eee3"),      # 293.13 MB read, 4.82 MB written
+    ("decode_m32", "tcgen05"): (297321728, "f284aa1030ca"),      # 293.13 MB read, 4.19 MB written
     # reduced case (64 experts, 64 tokens: the same 8 rows per expert) x 4 experts
-    ("decode_m256", "tcgen05"): (4518880256, "18e52bb5eee3"),    # 4 x (1122.32 + 7.40) MB
-    ("prefill_m8192", "tcgen05"): (3190343424, "18e52bb5eee3"),  # 2.8000 GB read, 0.3903 GB written
+    ("decode_m256", "tcgen05"): (4515166208, "f284aa1030ca"),    # 4 x (1122.08 + 6.71) MB
+    ("prefill_m8192", "tcgen05"): (3189124864, "f284aa1030ca"),  # 2.7995 GB read, 0.3896 GB written
 }
 # Entries not captured on the workload itself: how the figure was obtained.
 NCU_TRAFFIC_SCALED = {

@@ -136,6 +136,9 @@ NVM_DEV uint32_t pack_f16x2(float a, float b) {
 // Activation packing (once per call)
 // ---------------------------------------------------------------------------
 
+// 16-byte loads each lane of the x pack kernels keeps in flight.
+constexpr int kPackLoads = 4;
+
 // One warp per token t < M: texp[t] = e, the power of two that brings the
 // token's row of x into the f16 range (f16_range_exponent of its max |value|).
 // A token's row is packed once per routed slot, so its exponent is found once.
@@ -146,14 +149,24 @@ __global__ void __launch_bounds__(256)
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (t >= M) return;
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * K);
+  const int n = K / 8;
   float m = 0.0f;
-  for (int i = lane; i < K / 8; i += 32) {
-    const uint4 v = src[i];
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  // kPackLoads 16-byte pieces per lane in flight before any is used.
+  for (int i0 = lane; i0 < n; i0 += 32 * kPackLoads) {
+    uint4 v[kPackLoads];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      m = fmaxf(m, fabsf(bf16_bits_to_f32(w[j] & 0xFFFFu)));
-      m = fmaxf(m, fabsf(bf16_bits_to_f32(w[j] >> 16)));
+    for (int u = 0; u < kPackLoads; ++u) {
+      const int i = i0 + 32 * u;
+      v[u] = i < n ? src[i] : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < kPackLoads; ++u) {
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        m = fmaxf(m, fabsf(bf16_bits_to_f32(w[j] & 0xFFFFu)));
+        m = fmaxf(m, fabsf(bf16_bits_to_f32(w[j] >> 16)));
+      }
     }
   }
   const int e = f16_range_exponent(warp_max(m));
@@ -175,15 +188,26 @@ __global__ void __launch_bounds__(256)
   const float mul = exp2i(-e);
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * K);
   uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)row * K);
-  for (int i = lane; i < K / 8; i += 32) {
-    const uint4 v = src[i];
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint4 o;
-    uint32_t* op = &o.x;
+  const int n = K / 8;
+  for (int i0 = lane; i0 < n; i0 += 32 * kPackLoads) {
+    uint4 v[kPackLoads];
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-      op[j] = pack_f16x2(bf16_bits_to_f32(w[j] & 0xFFFFu) * mul, bf16_bits_to_f32(w[j] >> 16) * mul);
-    dst[i] = o;
+    for (int u = 0; u < kPackLoads; ++u) {
+      const int i = i0 + 32 * u;
+      if (i < n) v[u] = src[i];
+    }
+#pragma unroll
+    for (int u = 0; u < kPackLoads; ++u) {
+      const int i = i0 + 32 * u;
+      if (i >= n) continue;
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      uint4 o;
+      uint32_t* op = &o.x;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        op[j] = pack_f16x2(bf16_bits_to_f32(w[j] & 0xFFFFu) * mul, bf16_bits_to_f32(w[j] >> 16) * mul);
+      dst[i] = o;
+    }
   }
   if (lane == 0) xexp[row] = exp2i(e);
 }

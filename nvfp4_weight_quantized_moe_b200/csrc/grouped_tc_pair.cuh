@@ -4,10 +4,11 @@
 // arguments.
 //
 // A cluster of two CTAs runs tcgen05.mma.cta_group::2: M = 256 weight rows
-// (128 per CTA, each decoded into its own CTA's tensor memory) times N = up to
-// NT token rows (192, or 32 for decode-shaped batches; each CTA loads half of
-// the token tile into its own shared memory), FP32 accumulators in both CTAs' tensor memory (each CTA holds its
-// 128 rows x all N columns).  Per FLOP this halves the decode work and the
+// (128 per CTA, each decoded into its own CTA's tensor or shared memory) times
+// N = up to NT token rows (256 or 192 for prefill-shaped batches, 32 for
+// decode-shaped ones; each CTA loads half of the token tile into its own
+// shared memory), FP32 accumulators in both CTAs' tensor memory (each CTA
+// holds its 128 rows x all N columns).  Per FLOP this halves the decode work and the
 // tensor-memory stores of the one-CTA kernel at 128-token passes and cuts its
 // shared-memory traffic by a third, which is what bounded that kernel's MMA
 // rate.
