@@ -216,17 +216,18 @@ NVFP4_MOE_API size_t nvfp4_moe_workspace_bytes(uint32_t num_tokens, uint32_t top
  * f16 hi + lo pair; each row scaled by a power of two into the f16 range),
  * per-expert TMA tensor maps of the weights are built on the device from the
  * tables, and the projection kernel loads weight and activation tiles with
- * TMA, decodes the weights into tensor memory and runs tcgen05.mma with FP32
- * accumulators in tensor memory.  Arguments as for the calls without
- * _ws, plus num_experts (the length of the expert tables; it bounds the
- * offsets read) and `workspace`: device memory of at least
- * nvfp4_moe_workspace_bytes(num_tokens, topk, hidden, inter) bytes, 256-byte
- * aligned (NVFP4_MOE_EINVAL otherwise), owned by the caller, overwritten by
- * the call.  For the tcgen05
- * path opts->tiles selects the token rows per pass: 2 -> 16 and 16 -> 128 (one
- * CTA per 128 or 256 output rows); 4 -> 32, 24 -> 192 and 32 -> 256 (a cluster
- * of two CTAs sharing each MMA; down takes 192 for 32); 0 = from the shape.  Results equal the other path's within FP32 rounding.
- * Calls on one stream may share the workspace; concurrent calls may not.
+ * TMA, decodes the weights into tensor memory (or, at 256-row passes, shared
+ * memory) and runs tcgen05.mma with FP32 accumulators in tensor memory.
+ * Arguments as for the calls without _ws, plus num_experts (the length of the
+ * expert tables; it bounds the offsets read) and `workspace`: device memory of
+ * at least nvfp4_moe_workspace_bytes(num_tokens, topk, hidden, inter) bytes,
+ * 256-byte aligned (NVFP4_MOE_EINVAL otherwise), owned by the caller,
+ * overwritten by the call.  For the tcgen05 path opts->tiles selects the
+ * token rows per pass: 2 -> 16 and 16 -> 128 (one CTA per 128 or 256 output
+ * rows); 4 -> 32, 24 -> 192 and 32 -> 256 (a cluster of two CTAs sharing each
+ * MMA; down takes 192 for 32); 0 = from the shape.  Results equal the other
+ * path's within FP32 rounding.  Calls on one stream may share the workspace;
+ * concurrent calls may not.
  */
 NVFP4_MOE_API int nvfp4_moe_gate_up_silu_ws(
     const uint16_t* x, nvfp4_expert_tables gate, nvfp4_expert_tables up, float* act,
