@@ -437,6 +437,17 @@ def test_forward_full_decode(name, ws):
     _check_full(prob, bufs)
 
 
+@pytest.mark.parametrize("name,staging", [("decode_m1", 2), ("decode_m32", 1)],
+                         ids=["decode_m1-ring", "decode_m32-whole-k"])
+def test_forward_full_decode_other_staging(name, staging):
+    """The activation staging the automatic plan does not take at this size:
+    the two-chunk ring at decode M=1, whole-K staging at decode M=32."""
+    _need_gpu()
+    prob = make_problem(name)
+    _, bufs = _gpu_forward(prob, path=1, staging=staging)
+    _check_full(prob, bufs)
+
+
 # The oracle's full result at the two large sizes, computed once per session
 # (expert blocks spread over host processes; see _oracle_pool.py).
 _FULL_REF = {}
